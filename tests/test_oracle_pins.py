@@ -1,0 +1,206 @@
+"""Pins for the CPU oracle: facts that do not come from the oracle's own formulas.
+
+Each test names the passage of the ARCHead paper (arXiv 2608.02703 HTML) it follows.
+A plausible slip in the oracle -- swapped nibble order, wrong group index, a transposed
+factor, a dropped term, a wrong scale -- makes at least one of these fail.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from workloads import random_canonical_head
+
+
+def _empty_head(V, D, r_c, r_r, g):
+    G = D // g
+    return {
+        "V": V, "D": D, "r_c": r_c, "r_r": r_r, "g": g,
+        "r_nib": np.zeros((V, D // 2), np.uint8),
+        "r_code": np.zeros((V, G), np.uint8),
+        "r_super": np.zeros(V, np.uint16),
+        "Ac": np.zeros((V, r_c), np.int8), "sAc": np.zeros(V, np.float32),
+        "Bc": np.zeros((r_c, D), np.int8), "sBc": np.zeros((r_c, G), np.float32),
+        "Aw": np.zeros((V, r_r), np.int8), "sAw": np.zeros(V, np.float32),
+        "Bw": np.zeros((r_r, D), np.int8), "sBw": np.zeros((r_r, G), np.float32),
+    }
+
+
+def _bf16_bits_of(x):
+    """BF16 bit patterns of values exactly representable in BF16 (torch does the rounding)."""
+    t = torch.tensor(np.asarray(x, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def _identity_H(D):
+    return _bf16_bits_of(np.eye(D, dtype=np.float32))
+
+
+def test_bf16_decoding_matches_torch_on_all_patterns():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ours = oracle.bf16_bits_to_f64(bits)
+    ref = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan], ref[~nan])
+
+
+def test_int4_decoding_all_bytes():
+    """Sec. 3 'packed signed-INT4': each byte splits into two values in [-8, 7] whose
+    4-bit two's-complement patterns reassemble the byte (low nibble = even column)."""
+    b = np.arange(256, dtype=np.uint8)
+    vals = oracle.decode_int4_bytes(b[:, None])
+    assert vals.shape == (256, 2)
+    lo, hi = vals[:, 0].astype(np.int64), vals[:, 1].astype(np.int64)
+    assert lo.min() == -8 and lo.max() == 7 and hi.min() == -8 and hi.max() == 7
+    assert np.array_equal(((lo & 0xF) | ((hi & 0xF) << 4)).astype(np.uint8), b)
+
+
+def _pack_test(q):
+    """Inverse of the canonical nibble layout, written from its definition."""
+    q = np.asarray(q, np.int64)
+    return ((q[:, 0::2] & 0xF) | ((q[:, 1::2] & 0xF) << 4)).astype(np.uint8)
+
+
+def test_unit_scale_head_is_exact_integer_matmul():
+    """r_c = r_r = 0 with codes 1 and super-scale 1 leaves a plain INT4 matrix Q, so the
+    logits are H Q^T: an exact integer product (Sec. 3 final formula with empty factors)."""
+    rng = np.random.default_rng(1)
+    V, D, g, N = 37, 256, 64, 5
+    Q = rng.integers(-8, 8, size=(V, D))
+    head = _empty_head(V, D, 0, 0, g)
+    head["r_nib"] = _pack_test(Q)
+    head["r_code"][:] = 1
+    head["r_super"][:] = _bf16_bits_of(np.ones(V))
+    Hi = rng.integers(-100, 101, size=(N, D))
+    Y = oracle.logits(head, _bf16_bits_of(Hi))
+    assert np.array_equal(Y, (Hi @ Q.T).astype(np.float64))
+
+
+@pytest.mark.parametrize("v,d,qv", [(3, 137, -5), (0, 0, 7), (4, 255, -8), (2, 64, 1)])
+def test_single_residual_entry(v, d, qv):
+    """One nonzero nibble: W_hat has exactly one entry q * code[v, d // g] * S_v."""
+    V, D, g = 5, 256, 64
+    rng = np.random.default_rng(v * 1000 + d)
+    head = _empty_head(V, D, 0, 0, g)
+    Q = np.zeros((V, D), np.int64)
+    Q[v, d] = qv
+    head["r_nib"] = _pack_test(Q)
+    head["r_code"] = rng.integers(1, 256, size=(V, D // g)).astype(np.uint8)
+    head["r_super"][:] = _bf16_bits_of(np.full(V, 0.375))
+    Y = oracle.logits(head, _identity_H(D))  # row n of Y = column n of W_hat^T
+    expect = np.zeros((D, V))
+    expect[d, v] = qv * int(head["r_code"][v, d // g]) * 0.375
+    assert np.array_equal(Y, expect)
+
+
+def test_group_code_mapping():
+    """Every nibble = 1, super-scale 1: W_hat[v, d] = code[v, d // g] (group index pin)."""
+    V, D, g = 6, 256, 32
+    rng = np.random.default_rng(7)
+    head = _empty_head(V, D, 0, 0, g)
+    head["r_nib"] = _pack_test(np.ones((V, D), np.int64))
+    head["r_code"] = rng.integers(0, 256, size=(V, D // g)).astype(np.uint8)
+    head["r_super"][:] = _bf16_bits_of(np.ones(V))
+    Y = oracle.logits(head, _identity_H(D))
+    for vv in range(V):
+        for dd in range(D):
+            assert Y[dd, vv] == head["r_code"][vv, dd // g]
+
+
+def test_single_factor_entries():
+    """Core and correction factors each with one entry: W_hat[v, d] = (a s_A)(b s_B[group]).
+    Fixes the row-wise scale of A, the group-wise scale of B and both orientations."""
+    V, D, g = 4, 128, 64
+    head = _empty_head(V, D, 2, 3, g)
+    head["Ac"][2, 1] = 7
+    head["sAc"][:] = [1.0, 2.0, 0.5, 4.0]
+    head["Bc"][1, 70] = -3
+    head["sBc"][1] = [0.125, 0.25]          # column 70 is in group 1
+    head["Aw"][1, 2] = -11
+    head["sAw"][:] = [0.75, 0.0625, 1.5, 3.0]
+    head["Bw"][2, 5] = 9
+    head["sBw"][2] = [0.5, 8.0]             # column 5 is in group 0
+    W = oracle.dense_head_rows(head)
+    expect = np.zeros((V, D))
+    expect[2, 70] = (7 * 0.5) * (-3 * 0.25)
+    expect[1, 5] = (-11 * 0.0625) * (9 * 0.5)
+    assert np.array_equal(W, expect)
+    Y = oracle.logits(head, _identity_H(D))
+    assert np.array_equal(Y, expect.T)
+
+
+def test_factored_equals_dense():
+    """Sec. 3: Y = H W_d^T + (H B_w^T) A_w^T equals H (W_d + A_w B_w)^T."""
+    head = random_canonical_head(96, 256, 8, 8, 64, seed=3)
+    rng = np.random.default_rng(4)
+    H = _bf16_bits_of(rng.standard_normal((7, 256)).astype(np.float32))
+    Y1 = oracle.logits(head, H)
+    Y2 = oracle.logits_factored(head, H)
+    assert np.max(np.abs(Y1 - Y2)) <= 1e-10 * np.max(np.abs(Y1))
+
+
+def test_vocab_subsets_and_chunks_agree():
+    head = random_canonical_head(100, 128, 4, 4, 64, seed=5, zero_rows=3)
+    rng = np.random.default_rng(6)
+    H = _bf16_bits_of(rng.standard_normal((3, 128)).astype(np.float32))
+    Y = oracle.logits(head, H)
+    Yc = oracle.logits(head, H, chunk=7)
+    tol = 1e-12 * np.max(np.abs(Y))   # BLAS may sum in another order per slice shape
+    assert np.max(np.abs(Y - Yc)) <= tol
+    rows = np.array([99, 0, 17, 42])
+    assert np.max(np.abs(oracle.logits(head, H, rows=rows) - Y[:, rows])) <= tol
+
+
+def test_zero_super_scale_row_has_no_residual():
+    head = random_canonical_head(16, 128, 2, 2, 64, seed=8)
+    head["r_super"][5] = 0
+    W = oracle.unpack_residual(head)
+    assert np.all(W[5] == 0) and np.any(W[4] != 0)
+
+
+def test_residual_entries_exact_in_single_precision():
+    """q * c * S has at most 4 + 8 + 8 significant bits, so it is exact in IEEE single."""
+    head = random_canonical_head(64, 256, 0, 0, 64, seed=9)
+    R = oracle.unpack_residual(head)
+    assert np.array_equal(R.astype(np.float32).astype(np.float64), R)
+
+
+def test_nll_constant_logits_is_log_vocab():
+    Y = np.full((3, 1000), 2.5)
+    out = oracle.nll_from_logits(Y, np.array([0, 999, 500]))
+    assert np.allclose(out, math.log(1000), rtol=0, atol=1e-12)
+
+
+def test_nll_shift_invariance_and_dominant_logit():
+    rng = np.random.default_rng(10)
+    Y = rng.standard_normal((4, 50))
+    t = np.array([3, 7, 0, 49])
+    a = oracle.nll_from_logits(Y, t)
+    b = oracle.nll_from_logits(Y + 123.0, t)
+    assert np.allclose(a, b, atol=1e-12)
+    Y2 = Y.copy()
+    Y2[np.arange(4), t] = 1e3
+    assert np.all(oracle.nll_from_logits(Y2, t) < 1e-300 + 1e-12)
+
+
+def test_nll_matches_library_cross_entropy():
+    rng = np.random.default_rng(11)
+    Y = rng.standard_normal((6, 333)) * 4
+    t = rng.integers(0, 333, size=6)
+    ref = torch.nn.functional.cross_entropy(torch.from_numpy(Y), torch.from_numpy(t),
+                                            reduction="none").numpy()
+    assert np.allclose(oracle.nll_from_logits(Y, t), ref, rtol=0, atol=1e-12)
+
+
+def test_int8_dequant_is_single_precision_product():
+    """The dequantised INT8 factor is the IEEE-single product of value and FP32 scale,
+    the same single multiply a GPU performs with round-to-nearest-even."""
+    q = np.array([[127, -127, 3]], np.int8)
+    s = np.array([0.1], np.float32)
+    out = oracle.dequant_int8_rowwise(q, s)
+    ref = torch.tensor(q, dtype=torch.float32) * torch.tensor(s)[:, None]
+    assert np.array_equal(out, ref.double().numpy())
+    assert out[0, 0] != 127 * 0.1  # not the exact real product
