@@ -1,0 +1,406 @@
+#!/usr/bin/env python
+"""Benchmark: packed LM-head tokens/s with the decode HBM / prefill tensor roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the logit path (prologue, residual contraction with the rank
+epilogue) over each token batch of the workload: for the Qwen3-8B-shaped decode head that
+is one archead_logits call at each of N = 1, 4, 16, 64 (85 tokens).  Inputs are seeded
+synthetic data of the workload's shapes; the head is built by the construction (Algorithm
+1) on the GPU before timing.  Under torchrun every rank holds its own replica of the head
+and evaluates its own tokens (replicas only, weak scaling, no collective on the data
+path); rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (fp64, host cores) on a bounded vocabulary sample of
+the same workload, scaled to the full vocabulary.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import (WORKLOADS, bf16_bits, make_channel_scales, make_hidden,  # noqa: E402
+                       make_targets, make_weight)
+
+L2_BYTES = 126 * 2 ** 20
+METRIC = "packed LM-head tokens/s; decode HBM GB/s and prefill TFLOP/s vs B200 roofline"
+MAIN_KERNEL_SRC = ["packed_int4_lm_b200/csrc/residual_mma.cu",
+                   "packed_int4_lm_b200/csrc/archead_internal.cuh"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qwen_decode", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    return ap.parse_args()
+
+
+DEFAULT_STEPS = {"tiny": (500, 20), "qwen_decode": (600, 20), "qwen_prefill": (20, 3),
+                 "llama_batched": (100, 5), "wide_nll": (10, 3)}
+
+
+# ----------------------------------------------------------------------------------------
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm": d["hbm_gbs"], "bf16": d["bf16_tflops"],
+                "bf16_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for f in MAIN_KERNEL_SRC:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per launch of the main kernel from the committed ncu summary, or None
+    when the kernel source changed since those counters were taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(workload)
+    if not d or d.get("source_sha") != kernel_source_sha():
+        return None
+    return d.get("bytes_per_launch")
+
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, v in zip(self.NAMES, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------------------
+def build_head(w, device):
+    from packed_int4_lm_b200 import pack
+    W = make_weight(w.V, w.D, w.rank, w.sigma0, w.noise, w.seed_w, device=device)
+    s = make_channel_scales(w.D, w.sigma_s, w.n_outliers, w.outlier_mult, w.seed_scales)
+    Hc = make_hidden(w.n_cal, s, w.seed_hcal).to(device)
+    head = pack.build_head(W, Hc, w.r_c, w.r_r, w.g, w.p, w.lam, seed=w.seed_rsvd)
+    del W, Hc
+    torch.cuda.empty_cache()
+    return head, s
+
+
+def main_kernel_bytes(head, N):
+    """Algorithmic bytes one launch of the residual kernel must move: the packed rows it
+    reads (nibbles, codes, super-scales, A_c / A_w and their scales), the FP16 hidden
+    states and t, and the FP32 logits it writes (none in NLL mode)."""
+    per_head = sum(head[k].nbytes for k in ("r_nib", "r_code", "r_super", "Ac", "sAc", "Aw", "sAw"))
+    RR = head["r_c"] + head["r_r"]
+    return per_head + 2 * N * head["D"] + 4 * N * RR
+
+
+def flops(head, N):
+    V, D, RR = head["V"], head["D"], head["r_c"] + head["r_r"]
+    return 2.0 * N * V * D + 2.0 * N * RR * (V + D)
+
+
+def oracle_step(head, Hs, targets, Ns, nll_mode, rows):
+    """One step of the CPU oracle on the first `rows` vocabulary rows; returns seconds."""
+    import oracle
+    t0 = time.perf_counter()
+    for N in Ns:
+        Y = oracle.logits(head, Hs[N], rows=slice(0, rows))
+        if nll_mode:
+            oracle.nll_from_logits(Y, np.minimum(targets[N], rows - 1))
+    return time.perf_counter() - t0
+
+
+def oracle_rows_for(head, Hs, targets, Ns, nll_mode, budget_s):
+    """Vocabulary rows whose oracle step takes about budget_s (from a small probe)."""
+    V = head["V"]
+    probe_rows = min(V, 1024)
+    tp = oracle_step(head, Hs, targets, Ns, nll_mode, probe_rows)
+    return int(min(V, max(128, probe_rows * budget_s / max(tp, 1e-4))))
+
+
+def cpu_oracle_rate(head, Hs, targets, Ns, nll_mode, budget_s):
+    """Oracle tokens/s on a vocabulary sample, time scaled to the full vocabulary."""
+    rows = oracle_rows_for(head, Hs, targets, Ns, nll_mode, budget_s)
+    t = oracle_step(head, Hs, targets, Ns, nll_mode, rows)
+    return sum(Ns) / (t * head["V"] / rows), rows, t
+
+
+def main():
+    a = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = WORKLOADS[a.workload]
+    K, Wm = DEFAULT_STEPS[a.workload]
+    K = a.steps if a.steps is not None else K
+    Wm = a.warmup if a.warmup is not None else Wm
+    Ns = list(w.Ns)
+    nll_mode = w.nll
+    cfg = {"workload": f"{w.name}: V={w.V} D={w.D} N={','.join(map(str, Ns))} "
+                       f"r_c={w.r_c} r_r={w.r_r} g={w.g} p={w.p} lam={w.lam}"
+                       + (" fused NLL" if nll_mode else ""),
+           "V": w.V, "D": w.D, "tokens_per_step_per_gpu": sum(Ns), "parallelism": f"replicas{world}"}
+
+    if a.impl == "reference":
+        if rank != 0:
+            return
+        torch.cuda.set_device(local)
+        head, s = build_head(w, torch.device("cuda", local))
+        Hs = {N: bf16_bits(make_hidden(N, s, w.seed_heval)) for N in Ns}
+        tg = {N: make_targets(N, w.V, w.seed_targets).numpy() for N in Ns}
+        import oracle  # noqa: F401
+        budget = max(0.02, 150.0 / (K + Wm))  # whole run within a few minutes
+        rows_used = oracle_rows_for(head, Hs, tg, Ns, nll_mode, budget)
+        vals = []
+        for i in range(Wm + K):
+            t = oracle_step(head, Hs, tg, Ns, nll_mode, rows_used)
+            if i >= Wm:
+                vals.append(t * w.V / rows_used)  # scaled to the full vocabulary
+        ms = 1e3 * statistics.mean(vals)
+        value = sum(Ns) / (ms / 1e3)
+        cores = len(os.sched_getaffinity(0))
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": a.gpus,
+                "steps": K, "warmup": Wm, "ms_per_step": ms, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": cfg, "impl": "reference",
+                "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
+                                 "kind": "oracle",
+                                 "sample": f"{sum(Ns)} tokens x {rows_used} of {w.V} vocab rows "
+                                           "per step, time scaled by V/rows"},
+                "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import packed_int4_lm_b200 as ah
+
+    if world > 1:
+        torch.distributed.init_process_group(
+            "nccl", timeout=datetime.timedelta(seconds=180),
+            device_id=torch.device("cuda", local))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    head, s = build_head(w, dev)
+    dh = ah.DeviceHead.from_canonical(head, dev)
+    # each rank evaluates its own tokens
+    Hcpu = {N: make_hidden(N, s, w.seed_heval + 7919 * rank) for N in Ns}
+    H = {N: Hcpu[N].to(dev) for N in Ns}
+    tg = {N: make_targets(N, w.V, w.seed_targets + 7919 * rank) for N in Ns}
+    tgd = {N: tg[N].to(dev) for N in Ns}
+    Y = {N: torch.empty(N, w.V, device=dev) for N in Ns} if not nll_mode else None
+    out = {N: torch.empty(N, device=dev) for N in Ns} if nll_mode else None
+    stream = torch.cuda.current_stream()
+
+    def step():
+        launches = 0
+        for N in Ns:
+            if nll_mode:
+                ah.nll(H[N], dh, tgd[N], out=out[N])
+            else:
+                ah.logits(H[N], dh, out=Y[N])
+            launches += ah.last_launches()
+        return launches
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(Wm):
+        step()
+    ah.check()
+    barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    ah.profile(True)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    launches = 0
+    for _ in range(K):
+        launches += step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ah.profile(False)
+    ck = clocks.stop()
+    ah.check()
+    elapsed_ms = e0.elapsed_time(e1)
+    main_ms, main_n = ah.profile_read()
+    t = torch.tensor([elapsed_ms], device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    elapsed_ms = float(t.item())
+    tokens = sum(Ns) * K * world
+    value = tokens / (elapsed_ms / 1e3)
+    peaks = load_peaks()
+
+    # roofline of the residual kernel over the timed launches
+    bytes_step = sum(main_kernel_bytes(head, N) + (0 if nll_mode else 4 * N * w.V) for N in Ns)
+    flops_step = sum(flops(head, N) for N in Ns)
+    mean_launch_s = (main_ms / 1e3) / max(main_n, 1)
+    launches_per_step = len(Ns)
+    if w.name in ("qwen_decode", "tiny") or max(Ns) <= 64:
+        achieved = bytes_step / launches_per_step / mean_launch_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm"]}
+    else:
+        achieved = flops_step / launches_per_step / mean_launch_s / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_sustained"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_sustained"]}
+    roof["peak_source"] = peaks["source"]
+    roof["kernel"] = "residual_mma_kernel"
+    roof["traffic"] = profiled_traffic(w.name)
+    roof["main_kernel_share"] = main_ms / max(elapsed_ms, 1e-9)
+
+    # per-N detail (not part of the headline)
+    per_n = {}
+    for N in Ns:
+        ah.profile(True)
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        reps = max(5, min(200, K))
+        f0.record(stream)
+        for _ in range(reps):
+            if nll_mode:
+                ah.nll(H[N], dh, tgd[N], out=out[N])
+            else:
+                ah.logits(H[N], dh, out=Y[N])
+        f1.record(stream)
+        torch.cuda.synchronize()
+        ah.profile(False)
+        kms, kn = ah.profile_read()
+        call_ms = f0.elapsed_time(f1) / reps
+        kern_ms = kms / max(kn, 1)
+        b = main_kernel_bytes(head, N) + (0 if nll_mode else 4 * N * w.V)
+        per_n[str(N)] = {"call_us": 1e3 * call_ms, "main_kernel_us": 1e3 * kern_ms,
+                         "tokens_per_s": N / (call_ms / 1e3),
+                         "main_GBps": b / (kern_ms / 1e3) / 1e9,
+                         "hbm_frac": b / (kern_ms / 1e3) / 1e9 / peaks["hbm"],
+                         "main_TFLOPs": flops(head, N) / (kern_ms / 1e3) / 1e12}
+
+    # end to end through the host-buffer entry points
+    Hpin = {N: Hcpu[N].pin_memory() for N in Ns}
+    tgpin = {N: tg[N].pin_memory() for N in Ns}
+    Yh = {N: torch.empty(N, w.V, pin_memory=True) for N in Ns} if not nll_mode else None
+    oh = {N: torch.empty(N, pin_memory=True) for N in Ns} if nll_mode else None
+
+    def step_host():
+        for N in Ns:
+            if nll_mode:
+                ah.nll_host(Hpin[N], dh, tgpin[N], out=oh[N])
+            else:
+                ah.logits_host(Hpin[N], dh, out=Yh[N])
+
+    KE = max(1, min(a.e2e_steps, K))
+    for _ in range(3):
+        step_host()
+    barrier()
+    torch.cuda.synchronize()
+    g0 = torch.cuda.Event(enable_timing=True)
+    g1 = torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for _ in range(KE):
+        step_host()
+    g1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    te = torch.tensor([g0.elapsed_time(g1)], device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
+    e2e_value = sum(Ns) * KE * world / (float(te.item()) / 1e3)
+    h2d = sum(N * w.D * 2 + (4 * N if nll_mode else 0) for N in Ns)
+    d2h = sum(4 * N if nll_mode else 4 * N * w.V for N in Ns)
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        Hs = {N: bf16_bits(Hcpu[N]) for N in Ns}
+        tgs = {N: tg[N].numpy() for N in Ns}
+        rate, rows, tcpu = cpu_oracle_rate(head, Hs, tgs, Ns, nll_mode, 15.0)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": len(os.sched_getaffinity(0)),
+               "kind": "oracle",
+               "sample": f"{sum(Ns)} tokens x {rows} of {w.V} vocab rows ({tcpu:.1f} s), "
+                         "time scaled by V/rows"}
+
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "warmup": Wm, "ms_per_step": elapsed_ms / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+            "config": dict(cfg, l2=("inputs larger than L2: packed head %.1f MB > 126 MB L2, "
+                                    "no flush" % (sum(head[k].nbytes for k in head
+                                                      if isinstance(head[k], np.ndarray)) / 1e6))),
+            "roofline": roof, "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": KE},
+            "gpu_launches": launches, "clocks": ck, "per_n": per_n}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,189 @@
+/*
+ * archead.h -- C ABI of the ARCHead packed LM-head logit library (NVIDIA B200, sm_100a).
+ *
+ * The operation (ARCHead: Activation-Metric Residual Correction for Large Language Model
+ * Output Heads, Sec. 3, the final approximation / logit formula and the inference
+ * statement after Algorithm 1):
+ *
+ *     W_d = Q8(A_c) Q8(B_c) + SC4(R)          (INT8 low-rank core + packed INT4 residual)
+ *     Y   = H W_d^T + (H B_w^T) A_w^T         (A_w row-wise INT8, B_w group-wise INT8)
+ *
+ * evaluated straight from packed storage; the dense V x D head never exists on the device.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor arguments are DEVICE pointers unless the name ends in _host; the caller
+ *    owns every buffer it passes and the library never frees or retains them.
+ *  - Row-major, densely packed.  BF16 and FP16 travel as uint16_t bit patterns.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  All work is enqueued
+ *    on it and the calls return without synchronising, except archead_check and the
+ *    _host variants.
+ *  - Return value: ARCHEAD_OK (0) or a negative ARCHEAD_ERR_* code.  Argument errors are
+ *    detected on the host before anything is enqueued.  Errors detected by a kernel
+ *    (ARCHEAD_ERR_RANGE_H, ARCHEAD_ERR_TARGET) set a per-device error word; the affected
+ *    outputs are non-finite; archead_check() reports and clears the word.
+ *  - Temporary device memory (the N x (r_c + r_r) prologue product t, the FP16 copy of H,
+ *    the NLL partials) is taken with cudaMallocAsync from a library-owned pool on
+ *    `stream` and returned with cudaFreeAsync on the same stream.
+ *  - Limits: g in {32, 64, 128, 256}; D % 128 == 0 and D % g == 0; 0 <= r_c, r_r <= 128;
+ *    1 <= V <= 8388480 (65535 blocks of 128 rows); 0 <= N < 2^31; N == 0 is a successful
+ *    no-op.  V needs no multiple of
+ *    any tile: the vocabulary tail is predicated.
+ *  - |H| must stay within the FP16 range (|h| <= 65504); larger or non-finite entries
+ *    raise ARCHEAD_ERR_RANGE_H (see archead_logits).
+ */
+#ifndef ARCHEAD_H_
+#define ARCHEAD_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ARCHEAD_ABI_VERSION 1
+
+enum archead_status {
+  ARCHEAD_OK = 0,
+  ARCHEAD_ERR_NULLPTR = -1,     /* a required pointer is NULL                         */
+  ARCHEAD_ERR_ALIGN = -2,       /* a pointer is not 16-byte aligned                   */
+  ARCHEAD_ERR_SHAPE = -3,       /* sizes disagree with the head or break a limit      */
+  ARCHEAD_ERR_RANGE_H = -4,     /* an entry of H is outside the FP16 range / not finite */
+  ARCHEAD_ERR_TARGET = -5,      /* a target id is outside [0, V)                      */
+  ARCHEAD_ERR_TIMEOUT = -6,     /* a bounded device wait gave up                      */
+  ARCHEAD_ERR_CUDA = -7,        /* a CUDA runtime call or launch failed               */
+  ARCHEAD_ERR_UNSUPPORTED = -8, /* no kernel for this device / configuration          */
+  ARCHEAD_ERR_NOMEM = -9        /* stream-ordered allocation failed                   */
+};
+
+/*
+ * The packed head (the serialised module of Sec. 3: the SC4 residual and its scales, the
+ * quantized core factors, the quantized correction factors and the shape metadata; no
+ * dense head).  Every pointer is a device pointer, 16-byte aligned, owned by the caller.
+ *
+ *   r_nib   uint8  V x D/2  signed INT4 residual nibbles in the DEVICE layout written by
+ *                           archead_repack_residual (see there)
+ *   r_code  uint8  V x D/g  UINT8 code c of each residual group (g columns)
+ *   r_super bf16   V        per-row BF16 super-scale S; residual entry = q * c * S
+ *   Ac int8 V x r_c, sAc f32 V         core left factor, one FP32 scale per row
+ *   Bc int8 r_c x D, sBc f32 r_c x D/g core right factor, one FP32 scale per g columns
+ *   Aw int8 V x r_r, sAw f32 V         correction left factor, row-wise
+ *   Bw int8 r_r x D, sBw f32 r_r x D/g correction right factor, group-wise
+ * A factor entry's value is the IEEE-single product of the INT8 value and its scale.
+ * Factor pointers may be NULL when their rank is 0.
+ */
+typedef struct archead_head {
+  int64_t V, D;
+  int32_t r_c, r_r, g;
+  int32_t reserved;
+  const uint8_t* r_nib;
+  const uint8_t* r_code;
+  const uint16_t* r_super;
+  const int8_t* Ac;
+  const float* sAc;
+  const int8_t* Bc;
+  const float* sBc;
+  const int8_t* Aw;
+  const float* sAw;
+  const int8_t* Bw;
+  const float* sBw;
+} archead_head;
+
+/*
+ * archead_logits -- Y = H W_d^T + (H B_w^T) A_w^T   (ARCHead Sec. 3, logit formula).
+ *   H  bf16 N x D (device), Y float N x V (device, fully overwritten).
+ *   N, V, D, r_c, r_r, g must equal the head's metadata (ARCHEAD_ERR_SHAPE otherwise).
+ *   N <= 64 runs the memory-bound decode kernel (each packed byte read once per call);
+ *   larger N runs the dense-contraction kernel.  Asynchronous on `stream`.
+ *   Precision: residual operands q*c are exact in FP16, H is rounded to FP16, products
+ *   accumulate in FP32; the low-rank terms run in FP32.
+ */
+int archead_logits(const uint16_t* H, const archead_head* head, float* Y, int64_t N,
+                   int64_t V, int64_t D, int r_c, int r_r, int g, void* stream);
+
+/*
+ * archead_nll -- per-token negative log-likelihood in nats (cross-entropy of Sec. 5):
+ *   nll[n] = logsumexp_v Y[n, v] - Y[n, targets[n]], without writing the N x V logits.
+ *   targets int32 N (device), nll_out float N (device).  A target outside [0, V) sets
+ *   ARCHEAD_ERR_TARGET in the device error word and makes that token's nll NaN.
+ */
+int archead_nll(const uint16_t* H, const archead_head* head, const int32_t* targets,
+                float* nll_out, int64_t N, int64_t V, int64_t D, int r_c, int r_r, int g,
+                void* stream);
+
+/*
+ * archead_logits_host -- archead_logits with HOST buffers: copies H_host (bf16 N x D) to
+ * the device, evaluates, copies Y back into Y_host (float N x V), and synchronises
+ * `stream` before returning.  Pinned host memory gives asynchronous copies.  The device
+ * staging buffers come from the library's stream-ordered pool.
+ */
+int archead_logits_host(const uint16_t* H_host, const archead_head* head, float* Y_host,
+                        int64_t N, int64_t V, int64_t D, int r_c, int r_r, int g,
+                        void* stream);
+
+/* archead_nll_host -- archead_nll with host H, targets and nll buffers (synchronous). */
+int archead_nll_host(const uint16_t* H_host, const archead_head* head,
+                     const int32_t* targets_host, float* nll_host, int64_t N, int64_t V,
+                     int64_t D, int r_c, int r_r, int g, void* stream);
+
+/*
+ * archead_repack_residual -- canonical residual nibbles -> device layout (load-time step).
+ *   canon: uint8 V x D/2, byte b of a row holds column 2b in bits 0-3 and column 2b+1 in
+ *          bits 4-7 (two's-complement INT4).
+ *   dev:   uint8 V x D/2, same bytes permuted.  A row is split into 128-column blocks of
+ *          64 bytes (16 32-bit words).  Word slot 4*t + w of a block holds the 8 columns
+ *          32*w + 8*t + {0..7} of the block; inside that word, nibble position p (bits
+ *          4p..4p+3) holds column 2p for p < 4 and column 2(p-4)+1 for p >= 4.
+ *   canon and dev must not overlap.  D % 128 == 0.  Asynchronous on `stream`.
+ */
+int archead_repack_residual(const uint8_t* canon, uint8_t* dev, int64_t V, int64_t D,
+                            void* stream);
+
+/*
+ * archead_dequant -- test and inspection hook: writes dequantised components as FP32.
+ *   R_out  float nrows x D : SC4 residual rows [row0, row0 + nrows): q * c * S (exact)
+ *   Ac_out float nrows x r_c, Aw_out float nrows x r_r : row-wise INT8 factors
+ *   Bc_out float r_c x D, Bw_out float r_r x D : group-wise INT8 factors
+ * Each INT8 entry is the single round-to-nearest-even product of value and scale.  Any
+ * output may be NULL to skip it.  Reads the residual in the device layout.
+ */
+int archead_dequant(const archead_head* head, int64_t row0, int64_t nrows, float* R_out,
+                    float* Ac_out, float* Aw_out, float* Bc_out, float* Bw_out,
+                    void* stream);
+
+/*
+ * archead_check -- synchronises `stream`, then reads and clears this device's error
+ * word.  Returns ARCHEAD_OK, ARCHEAD_ERR_RANGE_H, ARCHEAD_ERR_TARGET, ARCHEAD_ERR_TIMEOUT
+ * or ARCHEAD_ERR_CUDA (a pending CUDA error).
+ */
+int archead_check(void* stream);
+
+/* Human-readable text of a status code (static string, never NULL). */
+const char* archead_strerror(int status);
+
+/* ARCHEAD_ABI_VERSION of the loaded library. */
+int archead_abi_version(void);
+
+/*
+ * archead_last_launches -- number of kernels the library launched during the most recent
+ * successful archead_logits / archead_nll call on this host thread (for launch counting).
+ */
+int archead_last_launches(void);
+
+/*
+ * archead_profile -- measurement hook for timing the main contraction kernel alone.
+ *   archead_profile(1) clears the record and, from then on, each archead_logits /
+ *   archead_nll call on this process records a pair of CUDA events on its stream around
+ *   its residual-contraction kernel (up to 16384 pairs; later launches are not recorded).
+ *   archead_profile(0) stops recording.  archead_profile_read synchronises on the
+ *   recorded events and returns the summed kernel milliseconds and the launch count.
+ *   Both return ARCHEAD_OK or ARCHEAD_ERR_CUDA.  Not thread-safe across devices.
+ */
+int archead_profile(int enable);
+int archead_profile_read(double* total_ms, int* count);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ARCHEAD_H_ */

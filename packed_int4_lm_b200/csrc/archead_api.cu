@@ -1,0 +1,351 @@
+// C ABI of the ARCHead packed LM-head library: argument validation, stream-ordered
+// scratch, the per-device error word and kernel dispatch.  See include/archead.h.
+#include <mutex>
+
+#include "archead_internal.cuh"
+
+namespace archead {
+
+// Device-side error word: one instance per device that loads the library.
+static __device__ unsigned g_error_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool ready = false;
+  unsigned* err = nullptr;       // device address of g_error_word on this device
+  cudaMemPool_t pool = nullptr;  // library-owned stream-ordered pool
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+thread_local int t_last_launches = 0;
+
+// archead_profile: event pairs recorded around the residual kernel
+constexpr int kProfCap = 16384;
+struct Profile {
+  bool on = false;
+  int count = 0;
+  cudaEvent_t* ev = nullptr;  // 2 * kProfCap, created lazily
+} g_prof;
+
+void prof_mark(int which, cudaStream_t st) {
+  if (!g_prof.on || g_prof.count >= kProfCap) return;
+  cudaEventRecord(g_prof.ev[2 * g_prof.count + which], st);
+  if (which == 1) ++g_prof.count;
+}
+
+int current_state(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return ARCHEAD_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState& s = g_dev[dev];
+  if (!s.ready) {
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_error_word) != cudaSuccess) return ARCHEAD_ERR_CUDA;
+    if (cudaMemset(addr, 0, sizeof(unsigned)) != cudaSuccess) return ARCHEAD_ERR_CUDA;
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.handleTypes = cudaMemHandleTypeNone;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool;
+    if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return ARCHEAD_ERR_CUDA;
+    uint64_t keep = ~0ull;  // keep freed blocks cached in the pool between calls
+    cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    if (cudaDeviceSynchronize() != cudaSuccess) return ARCHEAD_ERR_CUDA;
+    s.err = static_cast<unsigned*>(addr);
+    s.pool = pool;
+    s.ready = true;
+  }
+  *out = &s;
+  return ARCHEAD_OK;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int check_head(const archead_head* h, int64_t N, int64_t V, int64_t D, int r_c, int r_r,
+               int g) {
+  if (!h) return ARCHEAD_ERR_NULLPTR;
+  if (h->V != V || h->D != D || h->r_c != r_c || h->r_r != r_r || h->g != g)
+    return ARCHEAD_ERR_SHAPE;
+  // V: the residual kernel's grid.y holds one 128-row vocabulary block each (<= 65535)
+  if (N < 0 || N > 0x7fffffffLL || V < 1 || V > 65535LL * 128 || D < 128 || D % 128 != 0)
+    return ARCHEAD_ERR_SHAPE;
+  if (!(g == 32 || g == 64 || g == 128 || g == 256) || D % g != 0) return ARCHEAD_ERR_SHAPE;
+  if (r_c < 0 || r_c > 128 || r_r < 0 || r_r > 128) return ARCHEAD_ERR_SHAPE;
+  if (!h->r_nib || !h->r_code || !h->r_super) return ARCHEAD_ERR_NULLPTR;
+  if (r_c > 0 && (!h->Ac || !h->sAc || !h->Bc || !h->sBc)) return ARCHEAD_ERR_NULLPTR;
+  if (r_r > 0 && (!h->Aw || !h->sAw || !h->Bw || !h->sBw)) return ARCHEAD_ERR_NULLPTR;
+  if (!aligned(h->r_nib, 16) || !aligned(h->r_code, 16) || !aligned(h->r_super, 16))
+    return ARCHEAD_ERR_ALIGN;
+  const void* f[] = {h->Ac, h->sAc, h->Bc, h->sBc, h->Aw, h->sAw, h->Bw, h->sBw};
+  for (const void* p : f)
+    if (p && !aligned(p, 16)) return ARCHEAD_ERR_ALIGN;
+  return ARCHEAD_OK;
+}
+
+Shapes make_shapes(int64_t N, int64_t V, int64_t D, int r_c, int r_r, int g) {
+  Shapes s;
+  s.N = N;
+  s.V = V;
+  s.D = D;
+  s.r_c = r_c;
+  s.r_r = r_r;
+  s.g = g;
+  return s;
+}
+
+// Stream-ordered scratch: one allocation carved into aligned pieces.
+struct Carve {
+  size_t off = 0;
+  size_t take(size_t bytes) {
+    size_t o = off;
+    off = round_up(off + (bytes ? bytes : 16), 256);
+    return o;
+  }
+};
+
+int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* targets,
+        float* nll, const Shapes& s, cudaStream_t st) {
+  DeviceState* ds;
+  int rc = current_state(&ds);
+  if (rc) return rc;
+  int launches = 0;
+  const int64_t tb = residual_token_block(s.N);
+  const int64_t Npad = (s.N + tb - 1) / tb * tb;
+  const int RR = s.r_c + s.r_r;
+  const bool nll_mode = nll != nullptr;
+  const int nvblk = residual_gemm_vblocks(s);
+  Carve cv;
+  const size_t o_hh = cv.take((size_t)Npad * s.D * 2);
+  const size_t o_t = cv.take((size_t)s.N * RR * 4);
+  const size_t o_part = nll_mode ? cv.take((size_t)s.N * nvblk * 8) : 0;
+  const size_t o_tl = nll_mode ? cv.take((size_t)s.N * 4) : 0;
+  void* base = nullptr;
+  if (cudaMallocFromPoolAsync(&base, cv.off, ds->pool, st) != cudaSuccess) {
+    cudaGetLastError();
+    return ARCHEAD_ERR_NOMEM;
+  }
+  char* b = static_cast<char*>(base);
+  __half* Hh = reinterpret_cast<__half*>(b + o_hh);
+  float* t = reinterpret_cast<float*>(b + o_t);
+  cudaError_t e = launch_prologue(H, head, s, Npad, Hh, t, ds->err, st, &launches);
+  if (e == cudaSuccess) {
+    if (!nll_mode) {
+      prof_mark(0, st);
+      e = launch_residual_gemm(Hh, t, head, s, Y, nullptr, nullptr, nullptr, st, &launches, 0);
+      prof_mark(1, st);
+    } else {
+      float2* part = reinterpret_cast<float2*>(b + o_part);
+      float* tl = reinterpret_cast<float*>(b + o_tl);
+      prof_mark(0, st);
+      e = launch_residual_gemm(Hh, t, head, s, nullptr, targets, part, tl, st, &launches, 1);
+      prof_mark(1, st);
+      if (e == cudaSuccess) e = launch_nll_combine(part, tl, targets, s, nll, ds->err, st, &launches);
+    }
+  }
+  cudaFreeAsync(base, st);
+  if (e != cudaSuccess) return ARCHEAD_ERR_CUDA;
+  t_last_launches = launches;
+  return ARCHEAD_OK;
+}
+
+}  // namespace
+}  // namespace archead
+
+using namespace archead;
+
+extern "C" {
+
+int archead_abi_version(void) { return ARCHEAD_ABI_VERSION; }
+
+int archead_last_launches(void) { return t_last_launches; }
+
+const char* archead_strerror(int status) {
+  switch (status) {
+    case ARCHEAD_OK: return "ok";
+    case ARCHEAD_ERR_NULLPTR: return "a required pointer is NULL";
+    case ARCHEAD_ERR_ALIGN: return "a pointer is not suitably aligned (16 bytes)";
+    case ARCHEAD_ERR_SHAPE: return "sizes disagree with the head or break a limit";
+    case ARCHEAD_ERR_RANGE_H: return "an entry of H is outside the FP16 range or not finite";
+    case ARCHEAD_ERR_TARGET: return "a target id is outside [0, V)";
+    case ARCHEAD_ERR_TIMEOUT: return "a bounded device wait gave up";
+    case ARCHEAD_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
+    case ARCHEAD_ERR_UNSUPPORTED: return "unsupported device or configuration";
+    case ARCHEAD_ERR_NOMEM: return "stream-ordered device allocation failed";
+    default: return "unknown status";
+  }
+}
+
+int archead_logits(const uint16_t* H, const archead_head* head, float* Y, int64_t N,
+                   int64_t V, int64_t D, int r_c, int r_r, int g, void* stream) {
+  int rc = check_head(head, N, V, D, r_c, r_r, g);
+  if (rc) return rc;
+  if (N == 0) {
+    t_last_launches = 0;
+    return ARCHEAD_OK;
+  }
+  if (!H || !Y) return ARCHEAD_ERR_NULLPTR;
+  if (!aligned(H, 16) || !aligned(Y, 4)) return ARCHEAD_ERR_ALIGN;
+  return run(H, head, Y, nullptr, nullptr, make_shapes(N, V, D, r_c, r_r, g),
+             static_cast<cudaStream_t>(stream));
+}
+
+int archead_nll(const uint16_t* H, const archead_head* head, const int32_t* targets,
+                float* nll_out, int64_t N, int64_t V, int64_t D, int r_c, int r_r, int g,
+                void* stream) {
+  int rc = check_head(head, N, V, D, r_c, r_r, g);
+  if (rc) return rc;
+  if (N == 0) {
+    t_last_launches = 0;
+    return ARCHEAD_OK;
+  }
+  if (!H || !targets || !nll_out) return ARCHEAD_ERR_NULLPTR;
+  if (!aligned(H, 16) || !aligned(targets, 4) || !aligned(nll_out, 4)) return ARCHEAD_ERR_ALIGN;
+  return run(H, head, nullptr, targets, nll_out, make_shapes(N, V, D, r_c, r_r, g),
+             static_cast<cudaStream_t>(stream));
+}
+
+int archead_logits_host(const uint16_t* H_host, const archead_head* head, float* Y_host,
+                        int64_t N, int64_t V, int64_t D, int r_c, int r_r, int g,
+                        void* stream) {
+  int rc = check_head(head, N, V, D, r_c, r_r, g);
+  if (rc) return rc;
+  if (N == 0) return ARCHEAD_OK;
+  if (!H_host || !Y_host) return ARCHEAD_ERR_NULLPTR;
+  DeviceState* ds;
+  rc = current_state(&ds);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t hb = (size_t)N * D * 2, yb = (size_t)N * V * 4;
+  void* base = nullptr;
+  const size_t yoff = round_up(hb, 256);
+  if (cudaMallocFromPoolAsync(&base, yoff + yb, ds->pool, st) != cudaSuccess) {
+    cudaGetLastError();
+    return ARCHEAD_ERR_NOMEM;
+  }
+  uint16_t* Hd = static_cast<uint16_t*>(base);
+  float* Yd = reinterpret_cast<float*>(static_cast<char*>(base) + yoff);
+  rc = ARCHEAD_OK;
+  if (cudaMemcpyAsync(Hd, H_host, hb, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    rc = ARCHEAD_ERR_CUDA;
+  if (!rc) rc = archead_logits(Hd, head, Yd, N, V, D, r_c, r_r, g, stream);
+  if (!rc && cudaMemcpyAsync(Y_host, Yd, yb, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    rc = ARCHEAD_ERR_CUDA;
+  cudaFreeAsync(base, st);
+  if (cudaStreamSynchronize(st) != cudaSuccess && !rc) rc = ARCHEAD_ERR_CUDA;
+  return rc;
+}
+
+int archead_nll_host(const uint16_t* H_host, const archead_head* head,
+                     const int32_t* targets_host, float* nll_host, int64_t N, int64_t V,
+                     int64_t D, int r_c, int r_r, int g, void* stream) {
+  int rc = check_head(head, N, V, D, r_c, r_r, g);
+  if (rc) return rc;
+  if (N == 0) return ARCHEAD_OK;
+  if (!H_host || !targets_host || !nll_host) return ARCHEAD_ERR_NULLPTR;
+  DeviceState* ds;
+  rc = current_state(&ds);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t hb = (size_t)N * D * 2, tb = (size_t)N * 4;
+  const size_t toff = round_up(hb, 256), noff = toff + round_up(tb, 256);
+  void* base = nullptr;
+  if (cudaMallocFromPoolAsync(&base, noff + tb, ds->pool, st) != cudaSuccess) {
+    cudaGetLastError();
+    return ARCHEAD_ERR_NOMEM;
+  }
+  char* b = static_cast<char*>(base);
+  uint16_t* Hd = reinterpret_cast<uint16_t*>(b);
+  int32_t* Td = reinterpret_cast<int32_t*>(b + toff);
+  float* Nd = reinterpret_cast<float*>(b + noff);
+  rc = ARCHEAD_OK;
+  if (cudaMemcpyAsync(Hd, H_host, hb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(Td, targets_host, tb, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    rc = ARCHEAD_ERR_CUDA;
+  if (!rc) rc = archead_nll(Hd, head, Td, Nd, N, V, D, r_c, r_r, g, stream);
+  if (!rc && cudaMemcpyAsync(nll_host, Nd, tb, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    rc = ARCHEAD_ERR_CUDA;
+  cudaFreeAsync(base, st);
+  if (cudaStreamSynchronize(st) != cudaSuccess && !rc) rc = ARCHEAD_ERR_CUDA;
+  return rc;
+}
+
+int archead_repack_residual(const uint8_t* canon, uint8_t* dev, int64_t V, int64_t D,
+                            void* stream) {
+  if (!canon || !dev) return ARCHEAD_ERR_NULLPTR;
+  if (V < 1 || V > 0x7fffffffLL || D < 128 || D % 128 != 0) return ARCHEAD_ERR_SHAPE;
+  if (!aligned(canon, 16) || !aligned(dev, 16)) return ARCHEAD_ERR_ALIGN;
+  const char* c0 = reinterpret_cast<const char*>(canon);
+  const char* d0 = reinterpret_cast<const char*>(dev);
+  const size_t n = (size_t)V * D / 2;
+  if (c0 < d0 + n && d0 < c0 + n) return ARCHEAD_ERR_SHAPE;  // overlapping buffers
+  return launch_repack(canon, dev, V, D, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? ARCHEAD_OK
+             : ARCHEAD_ERR_CUDA;
+}
+
+int archead_dequant(const archead_head* head, int64_t row0, int64_t nrows, float* R_out,
+                    float* Ac_out, float* Aw_out, float* Bc_out, float* Bw_out,
+                    void* stream) {
+  if (!head) return ARCHEAD_ERR_NULLPTR;
+  int rc = check_head(head, 0, head->V, head->D, head->r_c, head->r_r, head->g);
+  if (rc) return rc;
+  if (row0 < 0 || nrows < 0 || row0 + nrows > head->V) return ARCHEAD_ERR_SHAPE;
+  return launch_dequant(head, row0, nrows, R_out, Ac_out, Aw_out, Bc_out, Bw_out,
+                        static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? ARCHEAD_OK
+             : ARCHEAD_ERR_CUDA;
+}
+
+int archead_profile(int enable) {
+  if (enable) {
+    if (!g_prof.ev) {
+      g_prof.ev = new cudaEvent_t[2 * kProfCap];
+      for (int i = 0; i < 2 * kProfCap; ++i)
+        if (cudaEventCreate(&g_prof.ev[i]) != cudaSuccess) return ARCHEAD_ERR_CUDA;
+    }
+    g_prof.count = 0;
+  }
+  g_prof.on = enable != 0;
+  return ARCHEAD_OK;
+}
+
+int archead_profile_read(double* total_ms, int* count) {
+  double tot = 0.0;
+  for (int i = 0; i < g_prof.count; ++i) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(g_prof.ev[2 * i + 1]) != cudaSuccess ||
+        cudaEventElapsedTime(&ms, g_prof.ev[2 * i], g_prof.ev[2 * i + 1]) != cudaSuccess)
+      return ARCHEAD_ERR_CUDA;
+    tot += ms;
+  }
+  if (total_ms) *total_ms = tot;
+  if (count) *count = g_prof.count;
+  return ARCHEAD_OK;
+}
+
+int archead_check(void* stream) {
+  DeviceState* ds;
+  int rc = current_state(&ds);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return ARCHEAD_ERR_CUDA;
+  unsigned w = 0;
+  if (cudaMemcpy(&w, ds->err, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return ARCHEAD_ERR_CUDA;
+  if (w && cudaMemset(ds->err, 0, sizeof(unsigned)) != cudaSuccess) return ARCHEAD_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return ARCHEAD_ERR_CUDA;
+  if (w & kErrRangeH) return ARCHEAD_ERR_RANGE_H;
+  if (w & kErrTarget) return ARCHEAD_ERR_TARGET;
+  if (w & kErrTimeout) return ARCHEAD_ERR_TIMEOUT;
+  return ARCHEAD_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,131 @@
+// Prologue of the ARCHead logit path (ARCHead Sec. 3, the bracket (H B_w^T) of the logit
+// formula, and its core analogue H B_c^T):
+//   * Hh = fp16(H), zero-padded to Npad rows -- the B operand of the residual contraction;
+//   * t  = H [Q8(B_c) | Q8(B_w)]^T, N x (r_c + r_r) FP32 -- the rank terms' left products.
+#include "archead_internal.cuh"
+
+namespace archead {
+namespace {
+
+// One thread converts 8 consecutive BF16 values.  Rows n >= N are written as zeros.
+__global__ void __launch_bounds__(256) convert_h_kernel(const uint16_t* __restrict__ H,
+                                                        __half* __restrict__ Hh, int64_t N,
+                                                        int64_t Npad, int64_t D,
+                                                        unsigned* err) {
+  const int64_t total = Npad * D / 8;
+  const int64_t valid = N * D / 8;
+  bool bad = false;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    uint4 out = make_uint4(0, 0, 0, 0);
+    if (i < valid) {
+      uint4 in = *reinterpret_cast<const uint4*>(H + i * 8);
+      uint32_t w[4] = {in.x, in.y, in.z, in.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float lo = __uint_as_float(w[k] << 16);
+        float hi = __uint_as_float(w[k] & 0xFFFF0000u);
+        __half2 h = __floats2half2_rn(lo, hi);
+        o[k] = h2_bits(h);
+        // exponent field all ones: infinite or NaN after rounding to FP16
+        bad |= ((o[k] & 0x7C00u) == 0x7C00u) | ((o[k] & 0x7C000000u) == 0x7C000000u);
+      }
+      out = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    *reinterpret_cast<uint4*>(Hh + i * 8) = out;
+  }
+  if (bad) atomicOr(err, kErrRangeH);
+}
+
+// t[n, j] = sum_d h[n, d] * fl32(B[j, d] * sB[j, d / g]) with j < r_c from B_c and the
+// rest from B_w.  Block (token group of kTN, j); 256 threads stride over D, 8 columns each.
+constexpr int kTN = 8;
+
+__global__ void __launch_bounds__(256) lowrank_t_kernel(
+    const uint16_t* __restrict__ H, const int8_t* __restrict__ Bc,
+    const float* __restrict__ sBc, const int8_t* __restrict__ Bw,
+    const float* __restrict__ sBw, int r_c, int r_r, int64_t N, int64_t D, int g,
+    float* __restrict__ t) {
+  const int j = blockIdx.y;
+  const int RR = r_c + r_r;
+  const int8_t* B;
+  const float* sB;
+  int jj;
+  if (j < r_c) {
+    B = Bc; sB = sBc; jj = j;
+  } else {
+    B = Bw; sB = sBw; jj = j - r_c;
+  }
+  const int64_t G = D / g;
+  const int64_t n0 = (int64_t)blockIdx.x * kTN;
+  const int nv = (N - n0) < kTN ? (int)(N - n0) : kTN;
+  float acc[kTN];
+#pragma unroll
+  for (int n = 0; n < kTN; ++n) acc[n] = 0.f;
+
+  for (int64_t d0 = threadIdx.x * 8; d0 < D; d0 += 256 * 8) {
+    uint2 braw = *reinterpret_cast<const uint2*>(B + jj * D + d0);
+    const float s = sB[jj * G + d0 / g];
+    float b[8];
+    const int8_t* bq = reinterpret_cast<const int8_t*>(&braw);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) b[k] = __fmul_rn((float)bq[k], s);
+#pragma unroll
+    for (int n = 0; n < kTN; ++n) {
+      if (n < nv) {
+        uint4 hv = *reinterpret_cast<const uint4*>(H + (n0 + n) * D + d0);
+        uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
+        float a = acc[n];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          a = fmaf(__uint_as_float(hw[k] << 16), b[2 * k], a);
+          a = fmaf(__uint_as_float(hw[k] & 0xFFFF0000u), b[2 * k + 1], a);
+        }
+        acc[n] = a;
+      }
+    }
+  }
+  // block reduction of the kTN sums
+  __shared__ float red[8][kTN];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int n = 0; n < kTN; ++n) {
+    float v = acc[n];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) red[warp][n] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x < kTN && (int)threadIdx.x < nv) {
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) v += red[w][threadIdx.x];
+    t[(n0 + threadIdx.x) * RR + j] = v;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_prologue(const uint16_t* H, const archead_head* head, const Shapes& s,
+                            int64_t Npad, __half* Hh, float* t, unsigned* err,
+                            cudaStream_t st, int* launches) {
+  {
+    const int64_t chunks = Npad * s.D / 8;
+    int64_t blocks = (chunks + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks < 1) blocks = 1;
+    convert_h_kernel<<<(unsigned)blocks, 256, 0, st>>>(H, Hh, s.N, Npad, s.D, err);
+    ++*launches;
+  }
+  const int RR = s.r_c + s.r_r;
+  if (RR > 0) {
+    dim3 grid((unsigned)((s.N + kTN - 1) / kTN), RR);
+    lowrank_t_kernel<<<grid, 256, 0, st>>>(H, head->Bc, head->sBc, head->Bw, head->sBw,
+                                           s.r_c, s.r_r, s.N, s.D, s.g, t);
+    ++*launches;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace archead

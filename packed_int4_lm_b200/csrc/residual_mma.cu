@@ -1,0 +1,466 @@
+// Residual contraction of the ARCHead logit path with its low-rank epilogue:
+//
+//   Y[n, v] = S_v * sum_d h[n, d] q[v, d] c[v, d / g]                 (SC4 residual, Sec. 3)
+//           + sAc[v] * sum_j Ac[v, j] t[n, j]                         (quantized core)
+//           + sAw[v] * sum_j Aw[v, j] t[n, r_c + j]                   (correction, Sec. 3)
+//
+// (ARCHead Sec. 3: Y = H W_d^T + (H B_w^T) A_w^T with W_d = Q8(A_c) Q8(B_c) + SC4(R).)
+//
+// Warp-level tensor-core path (mma.sync m16n8k16, FP16 operands, FP32 accumulators):
+//  * each warp owns R tiles of 16 vocabulary rows and streams their packed nibbles with
+//    128-bit non-allocating loads, prefetched one 128-column chunk ahead in registers;
+//    every packed byte is read from HBM once per token block;
+//  * nibbles are dequantised in registers to q * c (exact in FP16) straight into the A
+//    fragment; the device nibble layout makes one 32-bit word feed two k16 steps;
+//  * the token block's FP16 hidden states (the B operand) are staged in shared memory by
+//    cp.async in a 3-stage ring, XOR-swizzled so the 128-bit fragment reads are
+//    conflict-free;
+//  * the epilogue applies S_v and adds the rank terms from t staged in shared memory.
+// MODE 0 writes Y.  MODE 1 (fused NLL) writes, per token and vocabulary block, the
+// (max, sum of exp(y - max)) pair and the target's logit, and never writes Y.
+#include "archead_internal.cuh"
+
+namespace archead {
+namespace {
+
+constexpr int kKC = 128;     // columns per pipeline chunk (one 64-byte block of a row)
+constexpr int kStages = 3;   // cp.async ring depth for the hidden-state chunks
+
+struct GemmParams {
+  const __half* Hh;  // Npad x D
+  const float* t;    // N x RR
+  const uint8_t* nib;
+  const uint8_t* code;
+  const uint16_t* sup;
+  const int8_t* Ac;
+  const float* sAc;
+  const int8_t* Aw;
+  const float* sAw;
+  float* Y;
+  const int32_t* targets;
+  float2* part;
+  float* tlogit;
+  int64_t N, V, D;
+  int r_c, r_r, g_shift;
+  int nvblk;
+  int red_off;  // byte offset of the MODE 1 reduction buffer in dynamic shared memory
+};
+
+constexpr int kRows = 128;  // vocabulary rows per block in every configuration
+
+template <int NT, int R, int WARPS>
+struct Cfg {
+  static constexpr int NTOK = NT * 8;
+  static constexpr int ROWS = 16 * R * WARPS;
+  static constexpr int THREADS = WARPS * 32;
+  static constexpr int HS_BYTES = kStages * NTOK * kKC * 2;
+};
+
+// Codes for the 4 windows of chunk kc of one row (CPC codes per chunk, g = 128 / CPC for
+// CPC > 1, g >= 128 otherwise).
+template <int CPC>
+__device__ __forceinline__ void load_codes(const uint8_t* __restrict__ crow, int kc,
+                                           int g_shift, uint32_t out[4]) {
+  if (CPC == 1) {
+    uint32_t c = __ldg(crow + ((kc * kKC) >> g_shift));
+    out[0] = out[1] = out[2] = out[3] = c;
+  } else if (CPC == 2) {
+    uint32_t c0 = __ldg(crow + kc * 2), c1 = __ldg(crow + kc * 2 + 1);
+    out[0] = out[1] = c0;
+    out[2] = out[3] = c1;
+  } else {
+#pragma unroll
+    for (int w = 0; w < 4; ++w) out[w] = __ldg(crow + kc * 4 + w);
+  }
+}
+
+template <int NT, int R, int WARPS, int CPC, int MODE>
+__global__ void __launch_bounds__(WARPS * 32)
+    residual_mma_kernel(const GemmParams p) {
+  using C = Cfg<NT, R, WARPS>;
+  static_assert(C::ROWS == kRows, "block row count");
+  extern __shared__ __align__(128) unsigned char smem[];
+  __half* Hs = reinterpret_cast<__half*>(smem);
+
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int gid = lane >> 2;  // row within the 8-row half tile / token within n8 tile
+  const int tq = lane & 3;    // thread within quad
+  const int64_t D = p.D;
+  const int nchunks = (int)(D / kKC);
+  // grid.x walks token blocks so that blocks sharing vocabulary rows run back to back
+  // and re-read the packed rows from L2 rather than HBM when there are several
+  const int64_t row_block = (int64_t)blockIdx.y * C::ROWS;
+  const int64_t tok0 = (int64_t)blockIdx.x * C::NTOK;
+
+  // rows owned by this thread: tile r -> rows base + gid and base + gid + 8
+  int64_t vrow[R][2];
+  const uint8_t* nib_row[R][2];
+  const uint8_t* code_row[R][2];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      int64_t v = row_block + (int64_t)(warp * R + r) * 16 + gid + 8 * h;
+      vrow[r][h] = v;
+      int64_t vc = v < p.V ? v : p.V - 1;  // clamp loads of tail rows; results discarded
+      nib_row[r][h] = p.nib + vc * (D / 2) + 16 * tq;
+      code_row[r][h] = p.code + vc * (D >> p.g_shift);
+    }
+  }
+
+  // hidden-state chunk loader: NTOK rows x 128 columns -> 16-byte pieces, swizzled
+  auto load_h = [&](int kc, int stage) {
+    __half* dst = Hs + (size_t)stage * C::NTOK * kKC;
+    constexpr int PIECES = C::NTOK * (kKC / 8);
+    for (int i = threadIdx.x; i < PIECES; i += C::THREADS) {
+      int n = i >> 4, c = i & 15;
+      int cs = c ^ ((n & 1) << 2);
+      cp_async16(dst + n * kKC + cs * 8, p.Hh + (tok0 + n) * D + (int64_t)kc * kKC + c * 8);
+    }
+  };
+
+  float acc[R][NT][4];
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[r][j][e] = 0.f;
+
+  // pipeline prologue
+#pragma unroll
+  for (int s = 0; s < kStages - 1; ++s) {
+    if (s < nchunks) load_h(s, s);
+    cp_async_commit();
+  }
+  uint4 cur[R][2];
+  uint32_t ccur[R][2][4];
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      cur[r][h] = ldg_stream(nib_row[r][h]);
+      load_codes<CPC>(code_row[r][h], 0, p.g_shift, ccur[r][h]);
+    }
+
+  for (int kc = 0; kc < nchunks; ++kc) {
+    __syncthreads();  // all warps are done with the stage that is refilled below
+    {
+      int nk = kc + kStages - 1;
+      if (nk < nchunks) load_h(nk, nk % kStages);
+      cp_async_commit();
+    }
+    uint4 nxt[R][2];
+    uint32_t cnxt[R][2][4];
+    const bool more = kc + 1 < nchunks;
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (more) {
+          nxt[r][h] = ldg_stream(nib_row[r][h] + (int64_t)(kc + 1) * 64);
+          load_codes<CPC>(code_row[r][h], kc + 1, p.g_shift, cnxt[r][h]);
+        } else {
+          nxt[r][h] = make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int w = 0; w < 4; ++w) cnxt[r][h][w] = 0;
+        }
+      }
+    cp_async_wait<kStages - 1>();
+    __syncthreads();
+
+    const __half* hs = Hs + (size_t)(kc % kStages) * C::NTOK * kKC;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      uint4 bf[NT];
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        int n = 8 * j + gid;
+        int cs = (4 * w + tq) ^ ((gid & 1) << 2);
+        bf[j] = *reinterpret_cast<const uint4*>(hs + n * kKC + cs * 8);
+      }
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        __half2 pr[2][4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t word = w == 0 ? cur[r][h].x : w == 1 ? cur[r][h].y : w == 2 ? cur[r][h].z
+                                                                               : cur[r][h].w;
+          __half2 c2 = __half2half2(__ushort2half_rn((unsigned short)ccur[r][h][w]));
+          __half2 nc24 = __hmul2(c2, __float2half2_rn(-24.f));
+          dequant_word(word, c2, nc24, pr[h]);
+        }
+        uint32_t a0[4] = {h2_bits(pr[0][0]), h2_bits(pr[1][0]), h2_bits(pr[0][1]),
+                          h2_bits(pr[1][1])};
+        uint32_t a1[4] = {h2_bits(pr[0][2]), h2_bits(pr[1][2]), h2_bits(pr[0][3]),
+                          h2_bits(pr[1][3])};
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+          mma_f16_16816(acc[r][j], a0, bf[j].x, bf[j].y);
+          mma_f16_16816(acc[r][j], a1, bf[j].z, bf[j].w);
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        cur[r][h] = nxt[r][h];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) ccur[r][h][w] = cnxt[r][h][w];
+      }
+  }
+  cp_async_wait<0>();
+  __syncthreads();  // the hidden-state ring is reused for t below
+
+  // ---- epilogue: S_v * acc + rank terms ----
+  const int RR = p.r_c + p.r_r;
+  float* ts = reinterpret_cast<float*>(smem);
+  const int TS = RR + 1;  // padded stride: the 4 token columns of a warp hit 4 banks
+  for (int i = threadIdx.x; i < C::NTOK * RR; i += C::THREADS) {
+    int n = i / RR, j = i - n * RR;
+    int64_t tok = tok0 + n;
+    ts[n * TS + j] = tok < p.N ? p.t[tok * RR + j] : 0.f;
+  }
+  __syncthreads();
+
+  float y[R][NT][4];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int64_t v = vrow[r][h];
+      const int64_t vc = v < p.V ? v : p.V - 1;
+      const float S = bf16_bits_to_float(__ldg(p.sup + vc));
+#pragma unroll
+      for (int j = 0; j < NT; ++j)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) y[r][j][2 * h + e] = S * acc[r][j][2 * h + e];
+      // core and correction rank terms, each with its own row scale
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        const int rank = part == 0 ? p.r_c : p.r_r;
+        if (rank == 0) continue;
+        const int8_t* arow = (part == 0 ? p.Ac : p.Aw) + vc * rank;
+        const float sa = __ldg((part == 0 ? p.sAc : p.sAw) + vc);
+        const int off = part == 0 ? 0 : p.r_c;
+        float lr[NT][2];
+#pragma unroll
+        for (int j = 0; j < NT; ++j) lr[j][0] = lr[j][1] = 0.f;
+        for (int i = 0; i < rank; ++i) {
+          const float a = (float)__ldg(arow + i);
+#pragma unroll
+          for (int j = 0; j < NT; ++j)
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+              lr[j][e] = fmaf(a, ts[(8 * j + 2 * tq + e) * TS + off + i], lr[j][e]);
+        }
+#pragma unroll
+        for (int j = 0; j < NT; ++j)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) y[r][j][2 * h + e] = fmaf(sa, lr[j][e], y[r][j][2 * h + e]);
+      }
+    }
+  }
+
+  if (MODE == 0) {
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int64_t v = vrow[r][h];
+        if (v >= p.V) continue;
+#pragma unroll
+        for (int j = 0; j < NT; ++j)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int64_t tok = tok0 + 8 * j + 2 * tq + e;
+            if (tok < p.N) p.Y[tok * p.V + v] = y[r][j][2 * h + e];
+          }
+      }
+    return;
+  }
+
+  // ---- MODE 1: per-token (max, sum exp) over this block's rows, and the target logit ----
+  float2* red = reinterpret_cast<float2*>(smem + p.red_off);  // [WARPS][NTOK]
+  const float NEG_INF = __int_as_float(0xff800000);
+#pragma unroll
+  for (int j = 0; j < NT; ++j)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      float m = NEG_INF;
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          if (vrow[r][h] < p.V) m = fmaxf(m, y[r][j][2 * h + e]);
+      float sum = 0.f;
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          if (vrow[r][h] < p.V) sum += __expf(y[r][j][2 * h + e] - m);
+      // combine the 8 lanes that share this token (same tq, different gid)
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        const float mo = __shfl_xor_sync(0xffffffffu, m, o);
+        const float so = __shfl_xor_sync(0xffffffffu, sum, o);
+        const float mn = fmaxf(m, mo);
+        const float a = (m == NEG_INF) ? 0.f : sum * __expf(m - mn);
+        const float b = (mo == NEG_INF) ? 0.f : so * __expf(mo - mn);
+        sum = a + b;
+        m = mn;
+      }
+      const int n = 8 * j + 2 * tq + e;
+      if (gid == 0) red[warp * C::NTOK + n] = make_float2(m, sum);
+      const int64_t tok = tok0 + n;
+      if (tok < p.N) {
+        const int64_t tgt = __ldg(p.targets + tok);
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            if (vrow[r][h] == tgt && vrow[r][h] < p.V) p.tlogit[tok] = y[r][j][2 * h + e];
+      }
+    }
+  __syncthreads();
+  for (int n = threadIdx.x; n < C::NTOK; n += C::THREADS) {
+    const int64_t tok = tok0 + n;
+    if (tok >= p.N) continue;
+    float m = NEG_INF, sum = 0.f;
+    for (int w = 0; w < WARPS; ++w) {
+      const float2 q = red[w * C::NTOK + n];
+      const float mn = fmaxf(m, q.x);
+      const float a = (m == NEG_INF) ? 0.f : sum * __expf(m - mn);
+      const float b = (q.x == NEG_INF) ? 0.f : q.y * __expf(q.x - mn);
+      sum = a + b;
+      m = mn;
+    }
+    p.part[tok * p.nvblk + blockIdx.y] = make_float2(m, sum);
+  }
+}
+
+// nll[n] = M + log(sum_b s_b exp(m_b - M)) - y_target, one warp per token, fixed order.
+__global__ void __launch_bounds__(256) nll_combine_kernel(const float2* __restrict__ part,
+                                                          const float* __restrict__ tlogit,
+                                                          const int32_t* __restrict__ targets,
+                                                          int64_t N, int64_t V, int nvblk,
+                                                          float* __restrict__ nll,
+                                                          unsigned* err) {
+  const int lane = threadIdx.x & 31;
+  const int64_t n = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (n >= N) return;
+  const float NEG_INF = __int_as_float(0xff800000);
+  const float2* pr = part + n * nvblk;
+  float m = NEG_INF;
+  for (int b = lane; b < nvblk; b += 32) m = fmaxf(m, pr[b].x);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float s = 0.f;
+  for (int b = lane; b < nvblk; b += 32) {
+    const float2 q = pr[b];
+    if (q.x != NEG_INF) s += q.y * expf(q.x - m);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) {
+    const int32_t tg = targets[n];
+    if (tg < 0 || (int64_t)tg >= V) {
+      nll[n] = __int_as_float(0x7fc00000);
+      atomicOr(err, kErrTarget);
+    } else {
+      nll[n] = m + logf(s) - tlogit[n];
+    }
+  }
+}
+
+template <int NT, int R, int WARPS, int CPC, int MODE>
+cudaError_t launch_cfg(const GemmParams& p0, cudaStream_t st) {
+  using C = Cfg<NT, R, WARPS>;
+  GemmParams p = p0;
+  const int RR = p.r_c + p.r_r;
+  size_t ts = (size_t)C::NTOK * (RR + 1) * 4;
+  size_t base = (size_t)C::HS_BYTES > ts ? (size_t)C::HS_BYTES : ts;
+  base = (base + 15) & ~(size_t)15;
+  p.red_off = (int)base;
+  const size_t smem = base + (size_t)WARPS * C::NTOK * sizeof(float2);
+  auto kern = residual_mma_kernel<NT, R, WARPS, CPC, MODE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)((p.N + C::NTOK - 1) / C::NTOK), (unsigned)p.nvblk);
+  kern<<<grid, C::THREADS, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <int NT, int R, int WARPS, int MODE>
+cudaError_t launch_cpc(const GemmParams& p, int g, cudaStream_t st) {
+  if (g == 32) return launch_cfg<NT, R, WARPS, 4, MODE>(p, st);
+  if (g == 64) return launch_cfg<NT, R, WARPS, 2, MODE>(p, st);
+  return launch_cfg<NT, R, WARPS, 1, MODE>(p, st);
+}
+
+template <int MODE>
+cudaError_t launch_mode(const GemmParams& p, int g, cudaStream_t st) {
+  if (p.N <= 8) return launch_cpc<1, 2, 4, MODE>(p, g, st);
+  if (p.N <= 16) return launch_cpc<2, 2, 4, MODE>(p, g, st);
+  if (p.N <= 32) return launch_cpc<4, 1, 8, MODE>(p, g, st);
+  return launch_cpc<8, 1, 8, MODE>(p, g, st);
+}
+
+}  // namespace
+
+int64_t residual_token_block(int64_t N) {
+  if (N <= 8) return 8;
+  if (N <= 16) return 16;
+  if (N <= 32) return 32;
+  return 64;
+}
+
+int residual_gemm_vblocks(const Shapes& s) { return (int)((s.V + kRows - 1) / kRows); }
+
+cudaError_t launch_residual_gemm(const __half* Hh, const float* t, const archead_head* head,
+                                 const Shapes& s, float* Y, const int32_t* targets,
+                                 float2* part, float* tlogit, cudaStream_t st, int* launches,
+                                 int mode) {
+  GemmParams p;
+  p.Hh = Hh;
+  p.t = t;
+  p.nib = head->r_nib;
+  p.code = head->r_code;
+  p.sup = head->r_super;
+  p.Ac = head->Ac;
+  p.sAc = head->sAc;
+  p.Aw = head->Aw;
+  p.sAw = head->sAw;
+  p.Y = Y;
+  p.targets = targets;
+  p.part = part;
+  p.tlogit = tlogit;
+  p.N = s.N;
+  p.V = s.V;
+  p.D = s.D;
+  p.r_c = s.r_c;
+  p.r_r = s.r_r;
+  int gs = 0;
+  while ((1 << gs) < s.g) ++gs;
+  p.g_shift = gs;
+  p.nvblk = residual_gemm_vblocks(s);
+  p.red_off = 0;
+  cudaError_t e = mode == 0 ? launch_mode<0>(p, s.g, st) : launch_mode<1>(p, s.g, st);
+  ++*launches;
+  return e;
+}
+
+cudaError_t launch_nll_combine(const float2* part, const float* tlogit,
+                               const int32_t* targets, const Shapes& s, float* nll,
+                               unsigned* err, cudaStream_t st, int* launches) {
+  const int nvblk = residual_gemm_vblocks(s);
+  nll_combine_kernel<<<(unsigned)((s.N + 7) / 8), 256, 0, st>>>(part, tlogit, targets, s.N,
+                                                                 s.V, nvblk, nll, err);
+  ++*launches;
+  return cudaGetLastError();
+}
+
+}  // namespace archead

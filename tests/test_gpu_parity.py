@@ -1,0 +1,257 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 CPU oracle.
+
+Acceptance (the logit path's stated tolerances):
+  * dequantised components bit-exact;
+  * logits: max |Y - Y_ref| <= 1e-2 * rms(Y_ref);
+  * per-token NLL: |nll - nll_ref| <= 1e-3 nats.
+Shapes span several 128-row vocabulary blocks with a ragged tail, token counts on both
+sides of every token-block size (8, 16, 32, 64) and a multi-block prefill, and all
+supported group sizes.  The five synthetic heads run at full size on sampled tokens.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import packed_int4_lm_b200 as ah
+from workloads import (WORKLOADS, bf16_bits, make_channel_scales, make_hidden,
+                       make_targets, make_weight, random_canonical_head)
+
+pytestmark = pytest.mark.gpu
+
+LOGIT_TOL = 1e-2   # relative to rms(Y_ref)
+NLL_TOL = 1e-3     # nats
+
+
+def _rand_H(N, D, seed, sigma_s=0.5, n_out=4, mult=20.0):
+    s = make_channel_scales(D, sigma_s, n_out, mult, seed)
+    return make_hidden(N, s, seed + 1)
+
+
+def _assert_logits(Y, Yref, what=""):
+    Y = np.asarray(Y, dtype=np.float64)
+    rms = np.sqrt(np.mean(Yref ** 2))
+    err = np.max(np.abs(Y - Yref))
+    assert np.all(np.isfinite(Y)), what
+    assert err <= LOGIT_TOL * rms, f"{what}: max err {err:.3e} > {LOGIT_TOL} * rms {rms:.3e}"
+    return err / rms
+
+
+@pytest.fixture(scope="module")
+def dev(cuda_ok):
+    return torch.device("cuda:0")
+
+
+# ----------------------------------------------------------------------------------------
+# bit-exact dequantisation (repack + device layout + dequant hook)
+# ----------------------------------------------------------------------------------------
+@pytest.mark.parametrize("g", [32, 64, 128, 256])
+def test_dequant_bit_exact(dev, g):
+    head = random_canonical_head(300, 512, 5, 3, g, seed=g, zero_rows=4, zero_groups=20)
+    dh = ah.DeviceHead.from_canonical(head, dev)
+    out = ah.dequant(dh)
+    torch.cuda.synchronize()
+    assert np.array_equal(out["R"].cpu().double().numpy(), oracle.unpack_residual(head))
+    assert np.array_equal(out["Ac"].cpu().double().numpy(),
+                          oracle.dequant_int8_rowwise(head["Ac"], head["sAc"]))
+    assert np.array_equal(out["Aw"].cpu().double().numpy(),
+                          oracle.dequant_int8_rowwise(head["Aw"], head["sAw"]))
+    assert np.array_equal(out["Bc"].cpu().double().numpy(),
+                          oracle.dequant_int8_groupwise(head["Bc"], head["sBc"], g))
+    assert np.array_equal(out["Bw"].cpu().double().numpy(),
+                          oracle.dequant_int8_groupwise(head["Bw"], head["sBw"], g))
+    part = ah.dequant(dh, 17, 40)
+    assert np.array_equal(part["R"].cpu().double().numpy(),
+                          oracle.unpack_residual(head, slice(17, 57)))
+
+
+# ----------------------------------------------------------------------------------------
+# logits and NLL on arbitrary packed bytes
+# ----------------------------------------------------------------------------------------
+@pytest.fixture(scope="module")
+def rhead(dev):
+    head = random_canonical_head(1000, 512, 8, 8, 64, seed=11, zero_rows=3, zero_groups=50)
+    return head, ah.DeviceHead.from_canonical(head, dev)
+
+
+@pytest.mark.parametrize("N", [1, 3, 8, 9, 16, 17, 31, 33, 64, 65, 130, 200])
+def test_logits_random_head(dev, rhead, N):
+    head, dh = rhead
+    H = _rand_H(N, 512, 100 + N)
+    Y = ah.logits(H.to(dev), dh)
+    ah.check()
+    Yref = oracle.logits(head, bf16_bits(H))
+    _assert_logits(Y.cpu().numpy(), Yref, f"N={N}")
+
+
+@pytest.mark.parametrize("g,r_c,r_r,V,D", [(32, 3, 0, 257, 256), (64, 0, 0, 129, 128),
+                                           (128, 16, 16, 515, 1024), (256, 1, 7, 300, 512),
+                                           (128, 0, 32, 700, 640)])
+def test_logits_shapes_groups_ranks(dev, g, r_c, r_r, V, D):
+    head = random_canonical_head(V, D, r_c, r_r, g, seed=V + D)
+    dh = ah.DeviceHead.from_canonical(head, dev)
+    for N in (5, 40):
+        H = _rand_H(N, D, N + g)
+        Y = ah.logits(H.to(dev), dh)
+        ah.check()
+        _assert_logits(Y.cpu().numpy(), oracle.logits(head, bf16_bits(H)), f"{g} {N}")
+
+
+@pytest.mark.parametrize("N", [1, 7, 64, 100])
+def test_nll_random_head(dev, rhead, N):
+    head, dh = rhead
+    H = _rand_H(N, 512, 300 + N)
+    tg = make_targets(N, head["V"], 7 + N)
+    out = ah.nll(H.to(dev), dh, tg.to(dev))
+    ah.check()
+    ref = oracle.nll(head, bf16_bits(H), tg.numpy())
+    err = np.max(np.abs(out.cpu().double().numpy() - ref))
+    assert err <= NLL_TOL, err
+
+
+def test_host_entry_points_match_device(dev, rhead):
+    head, dh = rhead
+    H = _rand_H(20, 512, 5)
+    Yd = ah.logits(H.to(dev), dh).cpu()
+    Yh = ah.logits_host(H.pin_memory(), dh)
+    assert torch.equal(Yd, Yh)
+    tg = make_targets(20, head["V"], 3)
+    nd = ah.nll(H.to(dev), dh, tg.to(dev)).cpu()
+    nh = ah.nll_host(H, dh, tg)
+    assert torch.equal(nd, nh)
+
+
+def test_launch_counts(dev, rhead):
+    head, dh = rhead
+    H = _rand_H(4, 512, 1).to(dev)
+    ah.logits(H, dh)
+    assert ah.last_launches() == 3
+    ah.nll(H, dh, make_targets(4, head["V"], 1).to(dev))
+    assert ah.last_launches() == 4
+    torch.cuda.synchronize()
+
+
+def test_empty_batch_is_noop(dev, rhead):
+    _, dh = rhead
+    H = torch.empty(0, 512, dtype=torch.bfloat16, device=dev)
+    Y = ah.logits(H, dh)
+    assert Y.shape == (0, 1000)
+    ah.check()
+
+
+def test_fp16_overflow_in_H_is_reported(dev, rhead):
+    _, dh = rhead
+    H = _rand_H(3, 512, 9)
+    H[1, 17] = 1.0e5
+    Y = ah.logits(H.to(dev), dh)
+    with pytest.raises(ah.ArcheadError) as ei:
+        ah.check()
+    assert ei.value.status == -4
+    assert not torch.isfinite(Y[1]).all()
+    ah.check()  # the error word was cleared
+
+
+def test_bad_target_is_reported(dev, rhead):
+    head, dh = rhead
+    H = _rand_H(4, 512, 10).to(dev)
+    tg = torch.tensor([0, head["V"], 5, -1], dtype=torch.int32, device=dev)
+    out = ah.nll(H, dh, tg)
+    with pytest.raises(ah.ArcheadError) as ei:
+        ah.check()
+    assert ei.value.status == -5
+    o = out.cpu()
+    assert torch.isnan(o[1]) and torch.isnan(o[3]) and torch.isfinite(o[0]) and torch.isfinite(o[2])
+
+
+def test_shape_mismatch_rejected(dev, rhead):
+    _, dh = rhead
+    H = _rand_H(2, 512, 11).to(dev)
+    Y = torch.empty(2, 1000, device=dev)
+    import ctypes
+    rc = ah._lib.lib().archead_logits(H.data_ptr(), ctypes.byref(dh.struct), Y.data_ptr(), 2,
+                                      999, 512, 8, 8, 64, None)
+    assert rc == -3
+
+
+# ----------------------------------------------------------------------------------------
+# the five synthetic heads (full size; oracle on sampled tokens where N is large)
+# ----------------------------------------------------------------------------------------
+def _build(w, device):
+    W = make_weight(w.V, w.D, w.rank, w.sigma0, w.noise, w.seed_w, device=device)
+    s = make_channel_scales(w.D, w.sigma_s, w.n_outliers, w.outlier_mult, w.seed_scales)
+    Hc = make_hidden(w.n_cal, s, w.seed_hcal)
+    head = ah.pack.build_head(W, Hc.to(device), w.r_c, w.r_r, w.g, w.p, w.lam,
+                              seed=w.seed_rsvd)
+    del W
+    torch.cuda.empty_cache()
+    return head, s
+
+
+_HEADS = {}
+
+
+def _workload_head(name, dev):
+    w = WORKLOADS[name]
+    key = (w.index,)
+    if key not in _HEADS:
+        head, s = _build(w, dev)
+        _HEADS[key] = (head, s, ah.DeviceHead.from_canonical(head, dev))
+    return w, _HEADS[key]
+
+
+def test_workload_tiny(dev):
+    w, (head, s, dh) = _workload_head("tiny", dev)
+    N = w.Ns[0]
+    H = make_hidden(N, s, w.seed_heval)
+    Y = ah.logits(H.to(dev), dh)
+    ah.check()
+    Yref = oracle.logits(head, bf16_bits(H))
+    _assert_logits(Y.cpu().numpy(), Yref, "tiny")
+    tg = make_targets(N, w.V, w.seed_targets)
+    n = ah.nll(H.to(dev), dh, tg.to(dev))
+    ah.check()
+    assert np.max(np.abs(n.cpu().double().numpy() - oracle.nll_from_logits(Yref, tg.numpy()))) <= NLL_TOL
+
+
+@pytest.mark.slow
+def test_workload_qwen_decode_and_prefill(dev):
+    w, (head, s, dh) = _workload_head("qwen_decode", dev)
+    Hfull = make_hidden(4096, s, w.seed_heval)           # prefill batch; decode uses its prefix
+    sample = np.array([0, 1, 2, 3, 15, 63, 64, 1000, 2047, 4095])
+    Yref = oracle.logits(head, bf16_bits(Hfull[sample]))
+    for N in w.Ns:
+        Y = ah.logits(Hfull[:N].to(dev), dh)
+        ah.check()
+        rows = [i for i, r in enumerate(sample) if r < N]
+        _assert_logits(Y.cpu().numpy()[sample[rows]], Yref[rows], f"decode N={N}")
+    Y = ah.logits(Hfull.to(dev), dh)
+    ah.check()
+    _assert_logits(Y[torch.from_numpy(sample).to(dev)].cpu().numpy(), Yref, "prefill N=4096")
+
+
+@pytest.mark.slow
+def test_workload_llama_batched(dev):
+    w, (head, s, dh) = _workload_head("llama_batched", dev)
+    H = make_hidden(max(w.Ns), s, w.seed_heval)
+    sample = np.array([0, 5, 31, 32, 100, 127, 128, 255])
+    Yref = oracle.logits(head, bf16_bits(H[sample]))
+    for N in w.Ns:
+        Y = ah.logits(H[:N].to(dev), dh)
+        ah.check()
+        rows = [i for i, r in enumerate(sample) if r < N]
+        _assert_logits(Y.cpu().numpy()[sample[rows]], Yref[rows], f"llama N={N}")
+
+
+@pytest.mark.slow
+def test_workload_wide_nll(dev):
+    w, (head, s, dh) = _workload_head("wide_nll", dev)
+    N = w.Ns[0]
+    H = make_hidden(N, s, w.seed_heval)
+    tg = make_targets(N, w.V, w.seed_targets)
+    out = ah.nll(H.to(dev), dh, tg.to(dev))
+    ah.check()
+    sample = np.array([0, 1, 511, 4096, 8191])
+    ref = oracle.nll(head, bf16_bits(H[sample]), tg.numpy()[sample])
+    got = out.cpu().double().numpy()[sample]
+    assert np.max(np.abs(got - ref)) <= NLL_TOL, (got, ref)
+    assert np.all(np.isfinite(out.cpu().numpy()))
