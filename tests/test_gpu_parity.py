@@ -97,9 +97,26 @@ def test_logits_shapes_groups_ranks(dev, g, r_c, r_r, V, D):
         _assert_logits(Y.cpu().numpy(), oracle.logits(head, bf16_bits(H)), f"{g} {N}")
 
 
+@pytest.fixture(scope="module")
+def nhead(dev):
+    """Random packed bytes scaled so that rms(Y) is a few units, the regime of language-model
+    logits.  The absolute NLL error of any FP32 evaluation grows with the logit magnitude
+    (rounding of sums of size |Y|), so an absolute bound in nats is meaningful only there."""
+    head = random_canonical_head(1000, 512, 8, 8, 64, seed=12, zero_rows=3, zero_groups=50,
+                                 super_exp_range=(-17, -13), factor_exp_range=(-13, -10))
+    return head, ah.DeviceHead.from_canonical(head, dev)
+
+
+def test_nll_head_is_in_logit_regime(nhead):
+    head, _ = nhead
+    Y = oracle.logits(head, bf16_bits(_rand_H(8, 512, 1)))
+    rms = np.sqrt(np.mean(Y ** 2))
+    assert 0.5 < rms < 20, rms
+
+
 @pytest.mark.parametrize("N", [1, 7, 64, 100])
-def test_nll_random_head(dev, rhead, N):
-    head, dh = rhead
+def test_nll_random_head(dev, nhead, N):
+    head, dh = nhead
     H = _rand_H(N, 512, 300 + N)
     tg = make_targets(N, head["V"], 7 + N)
     out = ah.nll(H.to(dev), dh, tg.to(dev))

@@ -159,7 +159,7 @@ def bf16_bits(x: torch.Tensor) -> np.ndarray:
 
 def random_canonical_head(V: int, D: int, r_c: int, r_r: int, g: int, seed: int,
                           zero_rows: int = 0, zero_groups: int = 0,
-                          super_exp_range=(-14, -4)) -> dict:
+                          super_exp_range=(-14, -4), factor_exp_range=(-9, -5)) -> dict:
     """Arbitrary packed-head bytes in the canonical layout (random, not constructed).
 
     Layout (per row v, little-endian bytes):
@@ -170,7 +170,9 @@ def random_canonical_head(V: int, D: int, r_c: int, r_r: int, g: int, seed: int,
       Ac int8 V x r_c, sAc f32 V ;  Bc int8 r_c x D, sBc f32 r_c x D/g
       Aw int8 V x r_r, sAw f32 V ;  Bw int8 r_r x D, sBw f32 r_r x D/g
     zero_rows rows get an all-zero residual (super-scale 0, codes 0); zero_groups random
-    groups get code 0.  INT8 values are drawn from [-127, 127].
+    groups get code 0.  INT8 values are drawn from [-127, 127].  Super-scales are
+    2^e (1 + m/128) with e uniform in super_exp_range; INT8 scales are 2^u with u uniform in
+    factor_exp_range (these two ranges set the logit magnitude).
     """
     rng = np.random.default_rng(seed)
     G = D // g
@@ -188,7 +190,7 @@ def random_canonical_head(V: int, D: int, r_c: int, r_r: int, g: int, seed: int,
     def i8(shape):
         return rng.integers(-127, 128, size=shape, dtype=np.int64).astype(np.int8)
 
-    def pos_f32(shape, lo=-9, hi=-5):
+    def pos_f32(shape, lo=factor_exp_range[0], hi=factor_exp_range[1]):
         return (2.0 ** rng.uniform(lo, hi, size=shape)).astype(np.float32)
 
     head["Ac"] = i8((V, r_c))
