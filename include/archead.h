@@ -171,6 +171,27 @@ int archead_abi_version(void);
 int archead_last_launches(void);
 
 /*
+ * archead_logits_noalloc -- archead_logits that allocates no device memory.
+ *   The paper has no counterpart to this entry point: it exists for callers that cannot
+ *   let a library allocate, such as serving engines that reserve nearly all GPU memory up
+ *   front for their own pool and account for every byte, or decode loops that must not
+ *   enter an allocator between kernels.
+ *   Same arguments, layouts, results and error codes as archead_logits.  Its temporary
+ *   buffers (the FP16 copy of H, Npad x D with Npad = N rounded up to 8, 16, 32 or a
+ *   multiple of 64, plus the N x (r_c + r_r) FP32 rank products, each rounded up to 256
+ *   bytes) live in one fixed 2 MiB device array that every GPU loading the library holds
+ *   until the process exits; larger requests return ARCHEAD_ERR_SHAPE before anything is
+ *   enqueued (e.g. D = 4096 allows N <= 192 with r_c + r_r = 64).
+ *   The first call on a device looks up that array's device address (cudaGetSymbolAddress)
+ *   with the device current; make that first call before any stream capture.
+ *   All calls share the one array: calls whose kernels overlap on the GPU (different
+ *   streams, or several host threads) race on it and must be serialised by the caller.
+ *   Each call writes every scratch byte before reading it, so no clearing is needed.
+ */
+int archead_logits_noalloc(const uint16_t* H, const archead_head* head, float* Y, int64_t N,
+                           int64_t V, int64_t D, int r_c, int r_r, int g, void* stream);
+
+/*
  * archead_profile -- measurement hook for timing the main contraction kernel alone.
  *   archead_profile(1) clears the record and, from then on, each archead_logits /
  *   archead_nll call on this process records a pair of CUDA events on its stream around

@@ -157,6 +157,20 @@ int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* ta
 }
 
 }  // namespace
+
+// Argument validation shared with other entry points (same checks as archead_logits).
+int validate_head_args(const archead_head* head, int64_t N, int64_t V, int64_t D, int r_c,
+                       int r_r, int g) {
+  return check_head(head, N, V, D, r_c, r_r, g);
+}
+
+// Device address of this device's error word (the device must be current).
+unsigned* error_word_address() {
+  void* addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, g_error_word) != cudaSuccess) return nullptr;
+  return static_cast<unsigned*>(addr);
+}
+
 }  // namespace archead
 
 using namespace archead;

@@ -122,6 +122,11 @@ cudaError_t launch_nll_combine(const float2* part, const float* tlogit,
 
 cudaError_t launch_repack(const uint8_t* canon, uint8_t* dev, int64_t V, int64_t D,
                           cudaStream_t st);
+
+// Host helpers defined in archead_api.cu.
+int validate_head_args(const archead_head* head, int64_t N, int64_t V, int64_t D, int r_c,
+                       int r_r, int g);
+unsigned* error_word_address();
 cudaError_t launch_dequant(const archead_head* head, int64_t row0, int64_t nrows,
                            float* R_out, float* Ac_out, float* Aw_out, float* Bc_out,
                            float* Bw_out, cudaStream_t st);
