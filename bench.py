@@ -76,16 +76,20 @@ def kernel_source_sha():
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload):
-    """DRAM bytes per launch of the main kernel from the committed ncu summary, or None
-    when the kernel source changed since those counters were taken."""
+def profiled_traffic(workload, Ns):
+    """Mean DRAM bytes per launch of the main kernel over the step's batches, from the
+    committed ncu summary; None when the kernel source changed since those counters were
+    taken or a batch size was not captured."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p)).get(workload)
     if not d or d.get("source_sha") != kernel_source_sha():
         return None
-    return d.get("bytes_per_launch")
+    by_n = d.get("bytes_per_launch_by_N", {})
+    if not all(str(N) in by_n for N in Ns):
+        return None
+    return sum(by_n[str(N)] for N in Ns) / len(Ns)
 
 
 class ClockSampler:
@@ -313,7 +317,7 @@ def main():
                 "unit": "TFLOP/s", "frac": achieved / peaks["bf16_sustained"]}
     roof["peak_source"] = peaks["source"]
     roof["kernel"] = "residual_mma_kernel"
-    roof["traffic"] = profiled_traffic(w.name)
+    roof["traffic"] = profiled_traffic(w.name, Ns)
     roof["main_kernel_share"] = main_ms / max(elapsed_ms, 1e-9)
 
     # per-N detail (not part of the headline)
