@@ -117,10 +117,12 @@ int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* ta
   int rc = current_state(&ds);
   if (rc) return rc;
   int launches = 0;
-  const int64_t tb = residual_token_block(s.N);
-  const int64_t Npad = (s.N + tb - 1) / tb * tb;
   const int RR = s.r_c + s.r_r;
   const bool nll_mode = nll != nullptr;
+  // logits for N >= 16: tensor-memory (tcgen05) kernel; otherwise the warp-MMA kernel
+  const bool use_tc = !nll_mode && s.N >= 16;
+  const int64_t tb = use_tc ? tc_token_tile(s.N, RR) : residual_token_block(s.N);
+  const int64_t Npad = (s.N + tb - 1) / tb * tb;
   const int nvblk = residual_gemm_vblocks(s);
   Carve cv;
   const size_t o_hh = cv.take((size_t)Npad * s.D * 2);
@@ -135,9 +137,15 @@ int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* ta
   char* b = static_cast<char*>(base);
   __half* Hh = reinterpret_cast<__half*>(b + o_hh);
   float* t = reinterpret_cast<float*>(b + o_t);
-  cudaError_t e = launch_prologue(H, head, s, Npad, Hh, t, ds->err, st, &launches);
+  cudaError_t e = use_tc ? launch_prologue_blocked(H, head, s, (int)tb, Hh, t, ds->err, st,
+                                                   &launches)
+                         : launch_prologue(H, head, s, Npad, Hh, t, ds->err, st, &launches);
   if (e == cudaSuccess) {
-    if (!nll_mode) {
+    if (use_tc) {
+      prof_mark(0, st);
+      e = launch_residual_tc(Hh, t, head, s, Y, ds->err, st, &launches);
+      prof_mark(1, st);
+    } else if (!nll_mode) {
       prof_mark(0, st);
       e = launch_residual_gemm(Hh, t, head, s, Y, nullptr, nullptr, nullptr, st, &launches, 0);
       prof_mark(1, st);

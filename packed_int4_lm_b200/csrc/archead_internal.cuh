@@ -105,6 +105,20 @@ cudaError_t launch_prologue(const uint16_t* H, const archead_head* head, const S
                             int64_t Npad, __half* Hh, float* t, unsigned* err,
                             cudaStream_t st, int* launches);
 
+// t = H [Q8(B_c) | Q8(B_w)]^T alone (N x (r_c + r_r) FP32).
+cudaError_t launch_lowrank_t(const uint16_t* H, const archead_head* head, const Shapes& s,
+                             float* t, cudaStream_t st, int* launches);
+
+// tcgen05 path: token tile (16, 32, 64 or 128) for N tokens and r_c + r_r = RR; the
+// blocked FP16 copy of H (Npad = N rounded up to the tile) and t; the contraction.
+int tc_token_tile(int64_t N, int RR);
+cudaError_t launch_prologue_blocked(const uint16_t* H, const archead_head* head,
+                                    const Shapes& s, int nt, __half* Hb, float* t,
+                                    unsigned* err, cudaStream_t st, int* launches);
+cudaError_t launch_residual_tc(const __half* Hb, const float* t, const archead_head* head,
+                               const Shapes& s, float* Y, unsigned* err, cudaStream_t st,
+                               int* launches);
+
 // Residual dequant-contraction over token blocks of up to 64 (mma.sync path).
 // mode 0: write logits Y.  mode 1: write NLL partials (max, sum exp) per (token, vocabulary
 // block) into part[N x residual_gemm_vblocks] and the target logit into tlogit[N].

@@ -118,6 +118,13 @@ cudaError_t launch_prologue(const uint16_t* H, const archead_head* head, const S
     convert_h_kernel<<<(unsigned)blocks, 256, 0, st>>>(H, Hh, s.N, Npad, s.D, err);
     ++*launches;
   }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_lowrank_t(H, head, s, t, st, launches);
+}
+
+cudaError_t launch_lowrank_t(const uint16_t* H, const archead_head* head, const Shapes& s,
+                             float* t, cudaStream_t st, int* launches) {
   const int RR = s.r_c + s.r_r;
   if (RR > 0) {
     dim3 grid((unsigned)((s.N + kTN - 1) / kTN), RR);

@@ -86,11 +86,11 @@ def test_logits_random_head(dev, rhead, N):
 
 @pytest.mark.parametrize("g,r_c,r_r,V,D", [(32, 3, 0, 257, 256), (64, 0, 0, 129, 128),
                                            (128, 16, 16, 515, 1024), (256, 1, 7, 300, 512),
-                                           (128, 0, 32, 700, 640)])
+                                           (128, 0, 32, 700, 640), (128, 80, 80, 300, 256)])
 def test_logits_shapes_groups_ranks(dev, g, r_c, r_r, V, D):
     head = random_canonical_head(V, D, r_c, r_r, g, seed=V + D)
     dh = ah.DeviceHead.from_canonical(head, dev)
-    for N in (5, 40):
+    for N in (5, 40, 150):
         H = _rand_H(N, D, N + g)
         Y = ah.logits(H.to(dev), dh)
         ah.check()
