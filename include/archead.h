@@ -61,9 +61,10 @@ enum archead_status {
  * quantized core factors, the quantized correction factors and the shape metadata; no
  * dense head).  Every pointer is a device pointer, 16-byte aligned, owned by the caller.
  *
- *   r_nib   uint8  V x D/2  signed INT4 residual nibbles in the DEVICE layout written by
- *                           archead_repack_residual (see there)
- *   r_code  uint8  V x D/g  UINT8 code c of each residual group (g columns)
+ *   r_nib   uint8  ceil(V/128)*128 x D/2  signed INT4 residual nibbles in the DEVICE
+ *                           layout written by archead_repack_residual (see there)
+ *   r_code  uint8  ceil(V/128)*128 x D/g  UINT8 code c of each residual group (g
+ *                           columns), row-major; rows >= V are padding (any value)
  *   r_super bf16   V        per-row BF16 super-scale S; residual entry = q * c * S
  *   Ac int8 V x r_c, sAc f32 V         core left factor, one FP32 scale per row
  *   Bc int8 r_c x D, sBc f32 r_c x D/g core right factor, one FP32 scale per g columns
@@ -130,10 +131,13 @@ int archead_nll_host(const uint16_t* H_host, const archead_head* head,
  * archead_repack_residual -- canonical residual nibbles -> device layout (load-time step).
  *   canon: uint8 V x D/2, byte b of a row holds column 2b in bits 0-3 and column 2b+1 in
  *          bits 4-7 (two's-complement INT4).
- *   dev:   uint8 V x D/2, same bytes permuted.  A row is split into 128-column blocks of
- *          64 bytes (16 32-bit words).  Word slot 4*t + w of a block holds the 8 columns
- *          32*w + 8*t + {0..7} of the block; inside that word, nibble position p (bits
- *          4p..4p+3) holds column 2p for p < 4 and column 2(p-4)+1 for p >= 4.
+ *   dev:   uint8 Vpad x D/2 with Vpad = ceil(V/128)*128 (rows >= V are written as zeros),
+ *          the same nibbles tiled for sequential streaming: the 128-column block kb of the
+ *          128-row tile T is the contiguous 8 KB region starting at (T*(D/128) + kb)*8192;
+ *          in it, the 16-byte chunk i (0..3) of tile row s starts at (i*128 + s)*16.  Chunk
+ *          i of a row's block holds four 32-bit words, word w for the 8 columns
+ *          32*w + 8*i + {0..7}; inside a word, nibble position p (bits 4p..4p+3) holds
+ *          column 2p for p < 4 and column 2(p-4)+1 for p >= 4.
  *   canon and dev must not overlap.  D % 128 == 0.  Asynchronous on `stream`.
  */
 int archead_repack_residual(const uint8_t* canon, uint8_t* dev, int64_t V, int64_t D,

@@ -62,15 +62,21 @@ class DeviceHead:
     def from_canonical(cls, head: dict, device="cuda", stream=None) -> "DeviceHead":
         dev = torch.device(device)
         up = {}
+        Vpad = (int(head["V"]) + 127) // 128 * 128
         for k in _KEYS:
             a = np.ascontiguousarray(head[k])
+            if k == "r_code" and a.shape[0] != Vpad:
+                # the device code array holds whole 128-row tiles (rows >= V are zero)
+                a = np.concatenate([a, np.zeros((Vpad - a.shape[0], a.shape[1]), a.dtype)])
             if a.dtype == np.uint16:
                 t = torch.from_numpy(a.view(np.int16))
             else:
                 t = torch.from_numpy(a)
             up[k] = t.to(dev, non_blocking=False)
         canon = up["r_nib"]
-        devnib = torch.empty_like(canon)
+        V, D = int(head["V"]), int(head["D"])
+        # device layout: rows padded to a multiple of 128 (see archead_repack_residual)
+        devnib = torch.empty((V + 127) // 128 * 128, D // 2, dtype=torch.uint8, device=dev)
         st = _stream_handle(stream)
         _lib.check(_lib.lib().archead_repack_residual(canon.data_ptr(), devnib.data_ptr(),
                                                       int(head["V"]), int(head["D"]), st),

@@ -119,14 +119,17 @@ int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* ta
   int launches = 0;
   const int RR = s.r_c + s.r_r;
   const bool nll_mode = nll != nullptr;
-  // logits for N >= 16: tensor-memory (tcgen05) kernel; otherwise the warp-MMA kernel
-  const bool use_tc = !nll_mode && s.N >= 16;
+  // logits: N <= 16 small-batch decode kernel; larger N the tensor-memory (tcgen05) kernel;
+  // the fused NLL runs on the warp-MMA kernel with its split-vocabulary epilogue
+  const bool use_dec = !nll_mode && s.N <= 16;
+  const bool use_tc = !nll_mode && !use_dec;
   const int64_t tb = use_tc ? tc_token_tile(s.N, RR) : residual_token_block(s.N);
   const int64_t Npad = (s.N + tb - 1) / tb * tb;
   const int nvblk = residual_gemm_vblocks(s);
   Carve cv;
   const size_t o_hh = cv.take((size_t)Npad * s.D * 2);
   const size_t o_t = cv.take((size_t)s.N * RR * 4);
+  const size_t o_hsum = use_dec ? cv.take((size_t)s.N * (s.D / s.g) * 4) : 0;
   const size_t o_part = nll_mode ? cv.take((size_t)s.N * nvblk * 8) : 0;
   const size_t o_tl = nll_mode ? cv.take((size_t)s.N * 4) : 0;
   void* base = nullptr;
@@ -144,6 +147,11 @@ int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* ta
     if (use_tc) {
       prof_mark(0, st);
       e = launch_residual_tc(Hh, t, head, s, Y, ds->err, st, &launches);
+      prof_mark(1, st);
+    } else if (use_dec) {
+      prof_mark(0, st);
+      e = launch_decode_mma(H, Hh, t, reinterpret_cast<float*>(b + o_hsum), head, s, Y, st,
+                            &launches);
       prof_mark(1, st);
     } else if (!nll_mode) {
       prof_mark(0, st);
@@ -306,8 +314,8 @@ int archead_repack_residual(const uint8_t* canon, uint8_t* dev, int64_t V, int64
   if (!aligned(canon, 16) || !aligned(dev, 16)) return ARCHEAD_ERR_ALIGN;
   const char* c0 = reinterpret_cast<const char*>(canon);
   const char* d0 = reinterpret_cast<const char*>(dev);
-  const size_t n = (size_t)V * D / 2;
-  if (c0 < d0 + n && d0 < c0 + n) return ARCHEAD_ERR_SHAPE;  // overlapping buffers
+  const size_t nc = (size_t)V * D / 2, nd = (size_t)((V + 127) / 128 * 128) * D / 2;
+  if (c0 < d0 + nd && d0 < c0 + nc) return ARCHEAD_ERR_SHAPE;  // overlapping buffers
   return launch_repack(canon, dev, V, D, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? ARCHEAD_OK
              : ARCHEAD_ERR_CUDA;

@@ -59,6 +59,47 @@ __device__ __forceinline__ void dequant_word(uint32_t w, __half2 c2, __half2 nc2
   out[3] = __hfma2(*reinterpret_cast<__half2*>(&p3), c2, nc24);
 }
 
+// Same result as dequant_word with fewer integer-pipe instructions (one shift, four
+// LOP3) and more FP16 ones.  A nibble in bits 0-3 of a half under exponent 1024 (pattern
+// 0x6400, unit 1) reads 1024 + n; in bits 4-7 it reads 1024 + 16n.  With the top bit
+// flipped (offset binary n = q + 8), x - 1032 and x / 16 - 72 both give q exactly, and
+// q * c is exact in FP16 (|q * c| <= 2040).
+__device__ __forceinline__ void dequant_word_lite(uint32_t w, __half2 c2, __half2 out[4]) {
+  const uint32_t w2 = w >> 8;
+  uint32_t x0 = and_xor(w, 0x000F000Fu, 0x64086408u);
+  uint32_t x1 = and_xor(w, 0x00F000F0u, 0x64806480u);
+  uint32_t x2 = and_xor(w2, 0x000F000Fu, 0x64086408u);
+  uint32_t x3 = and_xor(w2, 0x00F000F0u, 0x64806480u);
+  const __half2 k1032 = __float2half2_rn(1032.f);
+  const __half2 k16 = __float2half2_rn(0.0625f);
+  const __half2 k72 = __float2half2_rn(-72.f);
+  out[0] = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&x0), k1032), c2);
+  out[1] = __hmul2(__hfma2(*reinterpret_cast<__half2*>(&x1), k16, k72), c2);
+  out[2] = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&x2), k1032), c2);
+  out[3] = __hmul2(__hfma2(*reinterpret_cast<__half2*>(&x3), k16, k72), c2);
+}
+
+// The four FP16 pairs of one device-layout word as 1032 + q (offset-binary nibble under
+// the exponent of 1024, unit 1): three shifts and four LOP3, no FP16 arithmetic.  A
+// contraction over these values equals the contraction over q plus 1032 times the sum of
+// the other operand, which the caller removes.  Pair i holds (column 2i, column 2i + 1).
+__device__ __forceinline__ void magic_word(uint32_t w, uint32_t out[4]) {
+  out[0] = and_xor(w, 0x000F000Fu, 0x64086408u);
+  out[1] = and_xor(w >> 4, 0x000F000Fu, 0x64086408u);
+  out[2] = and_xor(w >> 8, 0x000F000Fu, 0x64086408u);
+  out[3] = and_xor(w >> 12, 0x000F000Fu, 0x64086408u);
+}
+
+// Device nibble layout, tiled: rows are padded to a multiple of 128 and every 128-row
+// tile's 128-column block (64 bytes per row) is one contiguous 8 KB region, so each tile
+// streams sequentially from HBM.  Inside the region, 16-byte chunk i (i = 0..3) of row s
+// of the tile sits at (i * 128 + s) * 16.  Chunk i of a row block holds the 32-bit words of
+// the 32-column windows w = 0..3 for the eight columns 32w + 8i + {0..7}, and inside a word
+// nibble p holds column 2p (p < 4) or 2(p - 4) + 1 (p >= 4).
+__device__ __forceinline__ int64_t nib_chunk_offset(int64_t v, int64_t kb, int64_t nkb, int i) {
+  return (((v >> 7) * nkb + kb) << 13) + (((int64_t)i << 7) + (v & 127)) * 16;
+}
+
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
@@ -76,6 +117,12 @@ __device__ __forceinline__ void mma_f16_16816(float d[4], const uint32_t a[4],
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem));
+}
+// 16-byte copy that reads src_bytes (0 or 16) from global memory and zero-fills the rest.
+__device__ __forceinline__ void cp_async16_zfill(void* smem, const void* gmem, uint32_t src_bytes) {
+  uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem),
+               "r"(src_bytes));
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n"); }
 template <int N>
@@ -118,6 +165,13 @@ cudaError_t launch_prologue_blocked(const uint16_t* H, const archead_head* head,
 cudaError_t launch_residual_tc(const __half* Hb, const float* t, const archead_head* head,
                                const Shapes& s, float* Y, unsigned* err, cudaStream_t st,
                                int* launches);
+
+// Small-batch decode (N <= 16): independent warps, per-warp cp.async rings, warp MMAs;
+// Hh is the row-major FP16 copy of H padded to residual_token_block(N) rows; hsum
+// (N x D/g FP32 scratch) receives 1032 times each token's sum of H over each group.
+cudaError_t launch_decode_mma(const uint16_t* H, const __half* Hh, const float* t,
+                              float* hsum, const archead_head* head, const Shapes& s,
+                              float* Y, cudaStream_t st, int* launches);
 
 // Residual dequant-contraction over token blocks of up to 64 (mma.sync path).
 // mode 0: write logits Y.  mode 1: write NLL partials (max, sum exp) per (token, vocabulary

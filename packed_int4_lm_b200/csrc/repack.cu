@@ -1,11 +1,13 @@
 // Load-time layout step and the dequantisation inspection hook.
 //
-// Device nibble layout (see archead_repack_residual in archead.h): a row is cut into
-// 128-column blocks of 16 32-bit words; word slot 4t + w of a block carries the columns
-// 32w + 8t + {0..7}; inside the word, nibble p carries column 2p (p < 4) or
-// 2(p - 4) + 1 (p >= 4).  One warp-quad 128-bit load then brings each thread the eight
-// columns it dequantises into an m16n8k16 A fragment for each of four 32-column windows,
-// and the nibble pairs (p, p + 4) land in the two halves of one FP16x2 register.
+// Device nibble layout (see archead_repack_residual in archead.h and nib_chunk_offset):
+// rows padded to a multiple of 128; each 128-row tile's 128-column block is a contiguous
+// 8 KB region of 16-byte chunks, chunk i of tile row s at (i * 128 + s) * 16.  Chunk i of a
+// row block holds, for the four 32-column windows w, the word of columns 32w + 8i + {0..7};
+// inside a word nibble p holds column 2p (p < 4) or 2(p - 4) + 1 (p >= 4).  So a warp-quad
+// thread's 16-byte chunk feeds its m16n8k16 A fragments for all four windows, a thread that
+// owns a whole row reads its four chunks conflict-free, and the nibble pairs (p, p + 4)
+// land in the two halves of one FP16x2 register.
 #include "archead_internal.cuh"
 
 namespace archead {
@@ -15,37 +17,44 @@ __device__ __forceinline__ int nibble_pos_of_column(int i8) {
   return (i8 & 1) ? 4 + (i8 >> 1) : (i8 >> 1);
 }
 
+// One thread per 16-byte device chunk (row v, block kb, chunk i): its four words are the
+// windows w = 0..3 of columns 32w + 8i + {0..7}.  Padding rows (v >= V) are zeros.
 __global__ void __launch_bounds__(256) repack_kernel(const uint8_t* __restrict__ canon,
                                                      uint8_t* __restrict__ dev, int64_t V,
                                                      int64_t D) {
-  const int64_t words_per_row = D / 8;
-  const int64_t total = V * words_per_row;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t v = i / words_per_row;
-    const int64_t widx = i - v * words_per_row;  // device word index within the row
-    const int64_t blk = widx >> 4;
-    const int slot = (int)(widx & 15);
-    const int t = slot >> 2, w = slot & 3;
-    const int64_t col0 = blk * 128 + 32 * w + 8 * t;
-    // canonical: 8 consecutive columns = 4 bytes starting at byte col0 / 2 (4-aligned)
-    const uint32_t cw = *reinterpret_cast<const uint32_t*>(canon + v * (D / 2) + col0 / 2);
-    uint32_t out = 0;
+  const int64_t nkb = D / 128;
+  const int64_t Vpad = (V + 127) / 128 * 128;
+  const int64_t total = Vpad * nkb * 4;
+  for (int64_t q = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; q < total;
+       q += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t v = q / (nkb * 4);
+    const int64_t rem = q - v * nkb * 4;
+    const int64_t kb = rem >> 2;
+    const int i = (int)(rem & 3);
+    uint32_t out[4] = {0u, 0u, 0u, 0u};
+    if (v < V) {
 #pragma unroll
-    for (int i8 = 0; i8 < 8; ++i8) {
-      const uint32_t nib = (cw >> (4 * i8)) & 0xFu;
-      out |= nib << (4 * nibble_pos_of_column(i8));
+      for (int w = 0; w < 4; ++w) {
+        const int64_t col0 = kb * 128 + 32 * w + 8 * i;
+        // canonical: 8 consecutive columns = 4 bytes starting at byte col0 / 2 (4-aligned)
+        const uint32_t cw = *reinterpret_cast<const uint32_t*>(canon + v * (D / 2) + col0 / 2);
+#pragma unroll
+        for (int i8 = 0; i8 < 8; ++i8)
+          out[w] |= ((cw >> (4 * i8)) & 0xFu) << (4 * nibble_pos_of_column(i8));
+      }
     }
-    reinterpret_cast<uint32_t*>(dev + v * (D / 2))[widx] = out;
+    *reinterpret_cast<uint4*>(dev + nib_chunk_offset(v, kb, nkb, i)) =
+        make_uint4(out[0], out[1], out[2], out[3]);
   }
 }
 
-__device__ __forceinline__ int residual_q(const uint8_t* __restrict__ dev_row, int64_t d) {
-  const int64_t blk = d >> 7;
+__device__ __forceinline__ int residual_q(const uint8_t* __restrict__ dev, int64_t v, int64_t d,
+                                          int64_t nkb) {
+  const int64_t kb = d >> 7;
   const int within = (int)(d & 127);
-  const int w = within >> 5, t = (within & 31) >> 3, i8 = within & 7;
+  const int w = within >> 5, i = (within & 31) >> 3, i8 = within & 7;
   const uint32_t word =
-      reinterpret_cast<const uint32_t*>(dev_row)[blk * 16 + 4 * t + w];
+      reinterpret_cast<const uint32_t*>(dev + nib_chunk_offset(v, kb, nkb, i))[w];
   const int nib = (int)((word >> (4 * nibble_pos_of_column(i8))) & 0xFu);
   return nib >= 8 ? nib - 16 : nib;
 }
@@ -60,7 +69,7 @@ __global__ void __launch_bounds__(256) dequant_residual_kernel(
        i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t r = i / D, d = i - r * D;
     const int64_t v = row0 + r;
-    const int q = residual_q(nib + v * (D / 2), d);
+    const int q = residual_q(nib, v, d, D / 128);
     const float c = (float)code[v * G + d / g];
     const float S = bf16_bits_to_float(sup[v]);
     // q * c * S has at most 20 significant bits: exact in either order
@@ -104,7 +113,7 @@ unsigned grid_for(int64_t n) {
 
 cudaError_t launch_repack(const uint8_t* canon, uint8_t* dev, int64_t V, int64_t D,
                           cudaStream_t st) {
-  repack_kernel<<<grid_for(V * D / 8), 256, 0, st>>>(canon, dev, V, D);
+  repack_kernel<<<grid_for((V + 127) / 128 * 128 * (D / 32)), 256, 0, st>>>(canon, dev, V, D);
   return cudaGetLastError();
 }
 

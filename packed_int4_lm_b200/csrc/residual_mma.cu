@@ -8,7 +8,8 @@
 //
 // Warp-level tensor-core path (mma.sync m16n8k16, FP16 operands, FP32 accumulators):
 //  * each warp owns R tiles of 16 vocabulary rows and streams their packed nibbles with
-//    128-bit non-allocating loads, prefetched one 128-column chunk ahead in registers;
+//    128-bit non-allocating loads (one 16-byte chunk per thread and row from the tiled
+//    device layout), prefetched one 128-column chunk ahead in registers;
 //    every packed byte is read from HBM once per token block;
 //  * nibbles are dequantised in registers to q * c (exact in FP16) straight into the A
 //    fragment; the device nibble layout makes one 32-bit word feed two k16 steps;
@@ -104,7 +105,7 @@ __global__ void __launch_bounds__(WARPS * 32)
       int64_t v = row_block + (int64_t)(warp * R + r) * 16 + gid + 8 * h;
       vrow[r][h] = v;
       int64_t vc = v < p.V ? v : p.V - 1;  // clamp loads of tail rows; results discarded
-      nib_row[r][h] = p.nib + vc * (D / 2) + 16 * tq;
+      nib_row[r][h] = p.nib + nib_chunk_offset(vc, 0, D / 128, tq);  // block 0
       code_row[r][h] = p.code + vc * (D >> p.g_shift);
     }
   }
@@ -159,7 +160,7 @@ __global__ void __launch_bounds__(WARPS * 32)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         if (more) {
-          nxt[r][h] = ldg_stream(nib_row[r][h] + (int64_t)(kc + 1) * 64);
+          nxt[r][h] = ldg_stream(nib_row[r][h] + ((int64_t)(kc + 1) << 13));
           load_codes<CPC>(code_row[r][h], kc + 1, p.g_shift, cnxt[r][h]);
         } else {
           nxt[r][h] = make_uint4(0, 0, 0, 0);

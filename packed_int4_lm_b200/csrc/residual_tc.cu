@@ -2,19 +2,26 @@
 //
 //   Y[n, v] = S_v * sum_d h[n, d] q[v, d] c[v, d / g]  +  rank terms        (ARCHead Sec. 3)
 //
-// One CTA computes a 128-row vocabulary tile for a tile of NT tokens (NT = 16..128):
-//  * warps 0-3 own one vocabulary row per thread (= one TMEM lane).  They stream the row's
-//    packed nibbles (64 bytes per 128-column block, prefetched one block ahead),
-//    dequantise them to exact FP16 q*c in registers and store them with tcgen05.st into a
-//    two-stage A ring in tensor memory (a 128 x 128 FP16 block = 64 TMEM columns);
-//  * warp 4, one thread: bulk-copies (TMA engine, no tensor map) the token tile's FP16 H
-//    block -- pre-arranged by the prologue as the 8 x 16-byte core-matrix image the MMA
-//    reads -- into a shared-memory ring;
-//  * warp 5, one thread: issues tcgen05.mma kind::f16 with A from tensor memory and B from
-//    shared memory, eight K=16 steps per block, into an M=128 x N=NT FP32 accumulator in
-//    tensor memory, and commits each stage back to its producers;
-//  * epilogue (warps 0-3): tcgen05.ld of the accumulator row, times S_v, plus the core and
+// Persistent, warp-specialised kernel.  A work item is one 128-row vocabulary tile for one
+// tile of NT tokens (NT = 16..128):
+//  * warp 8 (one thread) feeds three shared-memory rings with bulk copies (TMA engine, no
+//    tensor map, no multicast): the tile's 8 KB packed-nibble block per 128 columns (the
+//    tiled device layout makes it one contiguous region), the tile's group-scale codes once
+//    per item, and the token tile's FP16 H block (pre-arranged by the prologue as the
+//    128-byte-swizzled K-major image the MMA reads);
+//  * warps 0-3 (dequant): one vocabulary row per thread (= one TMEM lane).  A thread reads
+//    its row's four 16-byte chunks of the block (conflict free: chunk i of row s sits at
+//    (i * 128 + s) * 16), dequantises them to exact FP16 q*c and stores them with
+//    tcgen05.st into an A ring of 2-4 stages in tensor memory (128 x 128 FP16 = 64
+//    columns per stage); the dequant warps issue no global loads;
+//  * warp 9 (one thread): issues tcgen05.mma kind::f16, A from tensor memory, B from
+//    shared memory, eight K=16 steps per block, into one of two M=128 x N=NT FP32
+//    accumulators, so the next item's MMAs overlap the previous item's epilogue;
+//  * warps 4-7 (epilogue): tcgen05.ld of an accumulator row, times S_v, plus the core and
 //    correction rank terms from t staged in shared memory, stored coalesced into Y.
+// Scheduling: with a single token tile (decode) every CTA owns a contiguous run of tiles;
+// otherwise items are dealt round-robin with the token tile varying fastest, so CTAs
+// working on the same rows run together and re-read them from L2.
 // Every mbarrier wait is bounded (about a second of SM cycles); a wait that gives up sets
 // the device error word, the CTA drains what it issued and frees its tensor memory.
 #include "tc_common.cuh"
@@ -22,14 +29,14 @@
 namespace archead {
 namespace {
 
-constexpr int kTcThreads = 192;  // warps 0-3 dequant + epilogue, 4 H producer, 5 MMA issuer
-constexpr int kASt = 2;          // A-ring stages in tensor memory (64 columns each)
+constexpr int kTcThreads = 320;  // warps 0-3 dequant, 4-7 epilogue, 8 producer, 9 MMA
+constexpr int kPkBytes = 8192;   // packed block of one 128-row tile (128 columns)
 
 struct TcParams {
   const __half* Hb;  // blocked FP16 H: [token tile][128-column block][NT x 128 image]
   const float* t;    // N x RR
   const uint8_t* nib;
-  const uint8_t* code;
+  const uint8_t* code;  // Vpad x G
   const uint16_t* sup;
   const int8_t* Ac;
   const float* sAc;
@@ -38,206 +45,311 @@ struct TcParams {
   float* Y;
   int64_t N, V, D;
   int r_c, r_r, g_shift;
+  int n_tok_tiles;
+  int64_t n_vtiles;
   unsigned* err;
 };
 
 template <int NT>
 struct TcCfg {
-  static constexpr int SB = NT <= 64 ? 4 : 3;  // H ring stages
-  static constexpr int HSTAGE = NT * 256;      // bytes of one 128-column H block
-  static constexpr int TMEM_COLS = 256;        // NT accumulator columns + 2 x 64 A columns
-  static_assert(NT + 64 * kASt <= TMEM_COLS, "tensor memory budget");
+  static constexpr int SB = NT <= 16 ? 8 : (NT <= 32 ? 4 : 3);  // H ring stages
+  static constexpr int SP = NT <= 32 ? 6 : 4;                   // packed ring stages
+  static constexpr int HSTAGE = NT * 256;  // bytes of one 128-column H block
+  static constexpr int TMEM_COLS = NT <= 64 ? 256 : 512;
+  // A-ring stages (64 columns each) in what the two accumulators leave, at most 4
+  static constexpr int SA = (TMEM_COLS - 2 * NT) / 64 < 4 ? (TMEM_COLS - 2 * NT) / 64 : 4;
+  static_assert(SA >= 2 && 2 * NT + 64 * SA <= TMEM_COLS, "tensor memory budget");
   static_assert(NT % 16 == 0 && NT >= 16 && NT <= 256, "M=128 MMA needs N in 16..256");
 };
 
+__host__ __device__ inline size_t round16(size_t x) { return (x + 15) & ~(size_t)15; }
+
 template <int NT>
-size_t tc_smem_bytes(int RR) {
+size_t tc_smem_bytes(int RR, int G) {
   using C = TcCfg<NT>;
-  return (size_t)C::SB * C::HSTAGE + (size_t)RR * NT * 4 + 256;
+  return (size_t)C::SB * C::HSTAGE + (size_t)C::SP * kPkBytes + 2 * round16((size_t)128 * G) +
+         round16((size_t)RR * NT * 4) + 512;
 }
 
-// codes of the four 32-column windows of block kb (see residual_mma.cu: load_codes)
-template <int CPC>
-__device__ __forceinline__ void block_codes(const uint8_t* __restrict__ crow, int kb,
-                                            int g_shift, uint32_t out[4]) {
-  if (CPC == 1) {
-    uint32_t c = __ldg(crow + ((kb * 128) >> g_shift));
-    out[0] = out[1] = out[2] = out[3] = c;
-  } else if (CPC == 2) {
-    uint32_t c0 = __ldg(crow + kb * 2), c1 = __ldg(crow + kb * 2 + 1);
-    out[0] = out[1] = c0;
-    out[2] = out[3] = c1;
+// The k-th work item of this CTA: its tile's first row, its row limit, its token tile.
+struct Item {
+  int64_t vt, row0, row_end;
+  int tt;
+};
+
+__device__ __forceinline__ bool get_item(const TcParams& p, int k, Item& it) {
+  if (p.n_tok_tiles == 1) {
+    const int64_t t0 = p.n_vtiles * blockIdx.x / gridDim.x;
+    const int64_t t1 = p.n_vtiles * (blockIdx.x + 1) / gridDim.x;
+    it.vt = t0 + k;
+    if (it.vt >= t1) return false;
+    it.tt = 0;
   } else {
-#pragma unroll
-    for (int w = 0; w < 4; ++w) out[w] = __ldg(crow + kb * 4 + w);
+    const int64_t gi = blockIdx.x + (int64_t)k * gridDim.x;
+    if (gi >= p.n_vtiles * p.n_tok_tiles) return false;
+    it.vt = gi / p.n_tok_tiles;
+    it.tt = (int)(gi - it.vt * p.n_tok_tiles);
   }
+  it.row0 = it.vt * 128;
+  it.row_end = it.row0 + 128 < p.V ? it.row0 + 128 : p.V;
+  return true;
 }
 
-template <int NT, int CPC>
-__global__ void __launch_bounds__(kTcThreads, 1) residual_tc_kernel(const TcParams p) {
+template <int NT, int CPC, int DQ>
+__global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcParams p) {
   using C = TcCfg<NT>;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int RR = p.r_c + p.r_r;
-  unsigned char* Hs = smem;
-  float* ts = reinterpret_cast<float*>(smem + C::SB * C::HSTAGE);  // ts[j * NT + n]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SB * C::HSTAGE +
-                                               (((size_t)RR * NT * 4 + 15) & ~(size_t)15));
-  uint64_t* b_full = bars;
-  uint64_t* b_empty = bars + C::SB;
-  uint64_t* a_full = bars + 2 * C::SB;
-  uint64_t* a_empty = a_full + kASt;
-  uint64_t* acc_full = a_empty + kASt;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t D = p.D;
   const int nkb = (int)(D / 128);
-  const int64_t row0 = (int64_t)blockIdx.y * 128;
-  const int64_t tok0 = (int64_t)blockIdx.x * NT;
+  const int G = (int)(D >> p.g_shift);
+  const int code_bytes = 128 * G;
+  unsigned char* Hs = smem;
+  unsigned char* pk = Hs + C::SB * C::HSTAGE;
+  unsigned char* cds = pk + C::SP * kPkBytes;  // [2][128 x G]
+  float* ts = reinterpret_cast<float*>(cds + 2 * round16(code_bytes));  // ts[j * NT + n]
+  uint64_t* bars =
+      reinterpret_cast<uint64_t*>(reinterpret_cast<unsigned char*>(ts) + round16((size_t)RR * NT * 4));
+  uint64_t* b_full = bars;
+  uint64_t* b_empty = b_full + C::SB;
+  uint64_t* p_full = b_empty + C::SB;
+  uint64_t* p_empty = p_full + C::SP;
+  uint64_t* c_full = p_empty + C::SP;   // [2]
+  uint64_t* c_empty = c_full + 2;       // [2]
+  uint64_t* a_full = c_empty + 2;
+  uint64_t* a_empty = a_full + C::SA;
+  uint64_t* acc_full = a_empty + C::SA;  // [2]
+  uint64_t* acc_empty = acc_full + 2;    // [2]
+  uint64_t* mma_done = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::SB; ++s) {
       tc::mbar_init(&b_full[s], 1);
       tc::mbar_init(&b_empty[s], 1);
     }
-    for (int s = 0; s < kASt; ++s) {
+    for (int s = 0; s < C::SP; ++s) {
+      tc::mbar_init(&p_full[s], 1);
+      tc::mbar_init(&p_empty[s], 4);  // one arrival per dequant warp
+    }
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&c_full[s], 1);
+      tc::mbar_init(&c_empty[s], 4);
+      tc::mbar_init(&acc_full[s], 1);
+      tc::mbar_init(&acc_empty[s], 128);
+    }
+    for (int s = 0; s < C::SA; ++s) {
       tc::mbar_init(&a_full[s], 128);
       tc::mbar_init(&a_empty[s], 1);
     }
-    tc::mbar_init(acc_full, 1);
+    tc::mbar_init(mma_done, 1);
     tc::mbar_fence_init();
   }
-  if (warp == 5) tc::tmem_alloc(tmem_slot, C::TMEM_COLS);
-  for (int i = threadIdx.x; i < NT * RR; i += kTcThreads) {
-    const int j = i / NT, n = i - j * NT;
-    const int64_t tok = tok0 + n;
-    ts[i] = tok < p.N ? p.t[tok * RR + j] : 0.f;
-  }
+  if (warp == 9) tc::tmem_alloc(tmem_slot, C::TMEM_COLS);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tbase = *tmem_slot;
-  const uint32_t acol = tbase + NT;  // A ring: columns NT .. NT + 128 (lane field 0)
+  const uint32_t acol = tbase + 2 * NT;  // A ring after the two accumulators (lane 0)
 
-  if (warp == 4) {
-    // ---------------- H producer ----------------
+  if (warp == 8) {
+    // ---------------- producer: codes, packed blocks, H blocks ----------------
     if (lane == 0) {
-      const unsigned char* src =
-          reinterpret_cast<const unsigned char*>(p.Hb) + (int64_t)blockIdx.x * nkb * C::HSTAGE;
-      int issued = 0;
+      int k = 0;
       bool ok = true;
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % C::SB;
-        if (kb >= C::SB && !tc::mbar_wait(&b_empty[s], ((kb / C::SB) - 1) & 1, p.err)) {
+      int nb_issued = 0, np_issued = 0, nc_issued = 0;
+      Item it;
+      for (int i = 0; ok && get_item(p, i, it); ++i) {
+        const int cs = i & 1;
+        if (i >= 2 && !tc::mbar_wait(&c_empty[cs], ((i >> 1) - 1) & 1, p.err)) {
           ok = false;
           break;
         }
-        tc::mbar_arrive_expect_tx(&b_full[s], C::HSTAGE);
-        tc::bulk_g2s(Hs + s * C::HSTAGE, src + (int64_t)kb * C::HSTAGE, C::HSTAGE, &b_full[s]);
-        ++issued;
+        tc::mbar_arrive_expect_tx(&c_full[cs], (uint32_t)code_bytes);
+        tc::bulk_g2s(cds + cs * round16(code_bytes), p.code + it.row0 * G, (uint32_t)code_bytes,
+                     &c_full[cs]);
+        ++nc_issued;
+        const uint8_t* psrc = p.nib + ((it.vt * nkb) << 13);
+        const unsigned char* hsrc =
+            reinterpret_cast<const unsigned char*>(p.Hb) + (int64_t)it.tt * nkb * C::HSTAGE;
+        for (int kb = 0; kb < nkb; ++kb, ++k) {
+          const int sp = k % C::SP, sb = k % C::SB;
+          if (k >= C::SP && !tc::mbar_wait(&p_empty[sp], ((k / C::SP) - 1) & 1, p.err)) {
+            ok = false;
+            break;
+          }
+          tc::mbar_arrive_expect_tx(&p_full[sp], kPkBytes);
+          tc::bulk_g2s(pk + sp * kPkBytes, psrc + ((int64_t)kb << 13), kPkBytes, &p_full[sp]);
+          ++np_issued;
+          if (k >= C::SB && !tc::mbar_wait(&b_empty[sb], ((k / C::SB) - 1) & 1, p.err)) {
+            ok = false;
+            break;
+          }
+          tc::mbar_arrive_expect_tx(&b_full[sb], C::HSTAGE);
+          tc::bulk_g2s(Hs + sb * C::HSTAGE, hsrc + (int64_t)kb * C::HSTAGE, C::HSTAGE, &b_full[sb]);
+          ++nb_issued;
+        }
       }
       if (!ok) {  // drain copies that may still be in flight before the CTA exits
-        for (int kb = issued - C::SB < 0 ? 0 : issued - C::SB; kb < issued; ++kb)
-          tc::mbar_wait(&b_full[kb % C::SB], (kb / C::SB) & 1, p.err);
+        for (int q = nb_issued - C::SB < 0 ? 0 : nb_issued - C::SB; q < nb_issued; ++q)
+          tc::mbar_wait(&b_full[q % C::SB], (q / C::SB) & 1, p.err);
+        for (int q = np_issued - C::SP < 0 ? 0 : np_issued - C::SP; q < np_issued; ++q)
+          tc::mbar_wait(&p_full[q % C::SP], (q / C::SP) & 1, p.err);
+        for (int q = nc_issued - 2 < 0 ? 0 : nc_issued - 2; q < nc_issued; ++q)
+          tc::mbar_wait(&c_full[q & 1], (q >> 1) & 1, p.err);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_f16_m128(NT);
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int sa = kb % kASt, sb = kb % C::SB;
-        if (!tc::mbar_wait(&a_full[sa], (kb / kASt) & 1, p.err)) break;
-        if (!tc::mbar_wait(&b_full[sb], (kb / C::SB) & 1, p.err)) break;
+      int k = 0;
+      bool ok = true;
+      Item it;
+      for (int i = 0; ok && get_item(p, i, it); ++i) {
+        const int ab = i & 1;
+        if (i >= 2 && !tc::mbar_wait(&acc_empty[ab], ((i >> 1) - 1) & 1, p.err)) break;
         tc::fence_after_sync();
-        const uint32_t hb = tc::smem_u32(Hs + sb * C::HSTAGE);
+        const uint32_t dcol = tbase + ab * NT;
+        for (int kb = 0; kb < nkb; ++kb, ++k) {
+          const int sa = k % C::SA, sb = k % C::SB;
+          if (!tc::mbar_wait(&a_full[sa], (k / C::SA) & 1, p.err) ||
+              !tc::mbar_wait(&b_full[sb], (k / C::SB) & 1, p.err)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          const uint32_t hb = tc::smem_u32(Hs + sb * C::HSTAGE);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint64_t bd = tc::smem_desc_kmajor(hb + 256 * j, 128, 2048);
-          tc::mma_f16_ts(tbase, acol + 64 * sa + 8 * j, bd, idesc, (kb | j) != 0);
+          for (int j = 0; j < 8; ++j) {
+            // K step j: 64-column half j / 4 (NT x 128 bytes each), 32-byte offset j % 4
+            const uint64_t bd =
+                tc::smem_desc_kmajor_sw128(hb + (j >> 2) * NT * 128 + (j & 3) * 32);
+            tc::mma_f16_ts(dcol, acol + 64 * sa + 8 * j, bd, idesc, (kb | j) != 0);
+          }
+          tc::mma_commit(&a_empty[sa]);
+          tc::mma_commit(&b_empty[sb]);
         }
-        tc::mma_commit(&a_empty[sa]);
-        tc::mma_commit(&b_empty[sb]);
+        if (ok) tc::mma_commit(&acc_full[ab]);
       }
-      tc::mma_commit(acc_full);
+      tc::mma_commit(mma_done);
+      tc::mbar_wait(mma_done, 0, p.err);  // every MMA issued here has retired
     }
-  } else {
-    // ---------------- dequant + epilogue: thread = vocabulary row = TMEM lane ----------------
-    const int tid = threadIdx.x;  // 0..127
-    const int64_t v = row0 + tid;
-    const int64_t vc = v < p.V ? v : p.V - 1;  // tail rows load a valid row; results dropped
-    const uint8_t* nrow = p.nib + vc * (D / 2);
-    const uint8_t* crow = p.code + vc * (D >> p.g_shift);
+  } else if (warp < 4) {
+    // ---------------- dequant: thread = tile row = TMEM lane ----------------
+    const int tid = threadIdx.x;
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+    int k = 0;
     bool ok = true;
-
-    uint4 cur[4], nxt[4];
-    uint32_t cc[4], cn[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) cur[i] = ldg_stream(nrow + 16 * i);
-    block_codes<CPC>(crow, 0, p.g_shift, cc);
-
-    for (int kb = 0; kb < nkb; ++kb) {
-      const int sa = kb % kASt;
-      if (kb + 1 < nkb) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) nxt[i] = ldg_stream(nrow + (int64_t)(kb + 1) * 64 + 16 * i);
-        block_codes<CPC>(crow, kb + 1, p.g_shift, cn);
+    Item it;
+    for (int i = 0; ok && get_item(p, i, it); ++i) {
+      const int cs = i & 1;
+      // warp-uniform outcomes: the tcgen05 stores below are whole-warp instructions
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(&c_full[cs], (i >> 1) & 1, p.err))) {
+        ok = false;
+        break;
       }
-      // 16 words: slot 4t + w holds block columns 32w + 8t + {0..7}; its pair i is
-      // A columns (32w + 8t + 2i, +1) = TMEM column 16w + 4t + i of this stage
-      uint32_t a[64];
-      const uint32_t wds[16] = {cur[0].x, cur[0].y, cur[0].z, cur[0].w, cur[1].x, cur[1].y,
-                                cur[1].z, cur[1].w, cur[2].x, cur[2].y, cur[2].z, cur[2].w,
-                                cur[3].x, cur[3].y, cur[3].z, cur[3].w};
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const __half2 c2 = __half2half2(__ushort2half_rn((unsigned short)cc[w]));
-        const __half2 nc24 = __hmul2(c2, __float2half2_rn(-24.f));
-#pragma unroll
-        for (int t4 = 0; t4 < 4; ++t4) {
-          __half2 pr[4];
-          dequant_word(wds[4 * t4 + w], c2, nc24, pr);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) a[16 * w + 4 * t4 + i] = h2_bits(pr[i]);
-        }
-      }
-      if (kb >= kASt) {
-        // warp-uniform outcome: the tcgen05 stores below are whole-warp instructions
-        if (!__all_sync(0xffffffffu, tc::mbar_wait(&a_empty[sa], ((kb / kASt) - 1) & 1, p.err))) {
+      const unsigned char* crow = cds + cs * round16(code_bytes) + tid * G;
+      for (int kb = 0; kb < nkb; ++kb, ++k) {
+        const int sp = k % C::SP, sa = k % C::SA;
+        if (!__all_sync(0xffffffffu, tc::mbar_wait(&p_full[sp], (k / C::SP) & 1, p.err))) {
           ok = false;
           break;
         }
-        tc::fence_after_sync();
-      }
-      const uint32_t ta = acol + 64 * sa + lane_off;
-      tc::tmem_st16(ta, a);
-      tc::tmem_st16(ta + 16, a + 16);
-      tc::tmem_st16(ta + 32, a + 32);
-      tc::tmem_st16(ta + 48, a + 48);
-      tc::tmem_wait_st();
-      tc::fence_before_sync();
-      tc::mbar_arrive(&a_full[sa]);
+        const unsigned char* src = pk + sp * kPkBytes + tid * 16;
+        uint32_t wd[16];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        cur[i] = nxt[i];
-        cc[i] = cn[i];
+        for (int c = 0; c < 4; ++c) {
+          const uint4 u = *reinterpret_cast<const uint4*>(src + c * 128 * 16);
+          wd[4 * c + 0] = u.x;
+          wd[4 * c + 1] = u.y;
+          wd[4 * c + 2] = u.z;
+          wd[4 * c + 3] = u.w;
+        }
+        uint32_t cw[4];
+        if (CPC == 1) {
+          cw[0] = cw[1] = cw[2] = cw[3] = crow[(kb * 128) >> p.g_shift];
+        } else if (CPC == 2) {
+          cw[0] = cw[1] = crow[kb * 2];
+          cw[2] = cw[3] = crow[kb * 2 + 1];
+        } else {
+#pragma unroll
+          for (int w = 0; w < 4; ++w) cw[w] = crow[kb * 4 + w];
+        }
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&p_empty[sp]);
+        if (k >= C::SA) {
+          if (!__all_sync(0xffffffffu,
+                          tc::mbar_wait(&a_empty[sa], ((k / C::SA) - 1) & 1, p.err))) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+        }
+        const uint32_t ta = acol + 64 * sa + lane_off;
+        // window w (32 block columns) = TMEM columns 16w..16w+15: words w, 4+w, 8+w, 12+w
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const __half2 c2 = __half2half2(__ushort2half_rn((unsigned short)cw[w]));
+          uint32_t a16[16];
+#pragma unroll
+          for (int t4 = 0; t4 < 4; ++t4) {
+            __half2 pr[4];
+            if (DQ == 0) {
+              dequant_word(wd[4 * t4 + w], c2, __hmul2(c2, __float2half2_rn(-24.f)), pr);
+            } else {
+              dequant_word_lite(wd[4 * t4 + w], c2, pr);
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) a16[4 * t4 + q] = h2_bits(pr[q]);
+          }
+          tc::tmem_st16(ta + 16 * w, a16);
+        }
+        tc::tmem_wait_st();
+        tc::fence_before_sync();
+        tc::mbar_arrive(&a_full[sa]);
       }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&c_empty[cs]);
     }
-
-    if (ok && __all_sync(0xffffffffu, tc::mbar_wait(acc_full, 0, p.err))) {
+  } else if (warp < 8) {
+    // ---------------- epilogue: thread = accumulator row = TMEM lane ----------------
+    const int e = threadIdx.x - 128;
+    const uint32_t lane_off = (uint32_t)(32 * (warp - 4)) << 16;
+    int cur_tt = -1;
+    Item it;
+    for (int i = 0; get_item(p, i, it); ++i) {
+      const int ab = i & 1;
+      if (it.tt != cur_tt) {  // stage t of this token tile (transposed: ts[j * NT + n])
+        asm volatile("bar.sync 1, 128;\n" ::: "memory");
+        const int64_t tok0 = (int64_t)it.tt * NT;
+        for (int q = e; q < NT * RR; q += 128) {
+          const int j = q / NT, n = q - j * NT;
+          const int64_t tok = tok0 + n;
+          ts[q] = tok < p.N ? __ldg(p.t + tok * RR + j) : 0.f;
+        }
+        asm volatile("bar.sync 1, 128;\n" ::: "memory");
+        cur_tt = it.tt;
+      }
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(&acc_full[ab], (i >> 1) & 1, p.err))) break;
       tc::fence_after_sync();
+      const int64_t v = it.row0 + e;
+      const bool live = v < it.row_end;
+      const int64_t vc = live ? v : it.row0;
       const float S = bf16_bits_to_float(__ldg(p.sup + vc));
       const float sac = p.r_c ? __ldg(p.sAc + vc) : 0.f;
       const float saw = p.r_r ? __ldg(p.sAw + vc) : 0.f;
       const int8_t* arow_c = p.Ac + vc * p.r_c;
       const int8_t* arow_w = p.Aw + vc * p.r_r;
+      const int64_t tok0 = (int64_t)it.tt * NT;
 #pragma unroll 1
       for (int c = 0; c < NT / 16; ++c) {
         float y[16];
-        tc::tmem_ld16(tbase + lane_off + 16 * c, y);
+        tc::tmem_ld16(tbase + ab * NT + lane_off + 16 * c, y);
 #pragma unroll
-        for (int k = 0; k < 16; ++k) y[k] *= S;
+        for (int q = 0; q < 16; ++q) y[q] *= S;
 #pragma unroll 1
         for (int part = 0; part < 2; ++part) {
           const int rank = part == 0 ? p.r_c : p.r_r;
@@ -246,9 +358,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) residual_tc_kernel(const TcPara
           const float* tcol = ts + (part == 0 ? 0 : p.r_c) * NT + 16 * c;
           float lr[16];
 #pragma unroll
-          for (int k = 0; k < 16; ++k) lr[k] = 0.f;
-          for (int j = 0; j < rank; ++j) {
-            const float aj = (float)__ldg(arow + j);
+          for (int q = 0; q < 16; ++q) lr[q] = 0.f;
+          auto acc_j = [&](float aj, int j) {
             const float4* tp = reinterpret_cast<const float4*>(tcol + j * NT);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -258,35 +369,51 @@ __global__ void __launch_bounds__(kTcThreads, 1) residual_tc_kernel(const TcPara
               lr[4 * q + 2] = fmaf(aj, tv.z, lr[4 * q + 2]);
               lr[4 * q + 3] = fmaf(aj, tv.w, lr[4 * q + 3]);
             }
+          };
+          int j = 0;
+          if ((rank & 3) == 0 && ((reinterpret_cast<uintptr_t>(arow) & 3) == 0)) {
+            // four INT8 factor entries per 32-bit load
+            const uint32_t* aw4 = reinterpret_cast<const uint32_t*>(arow);
+#pragma unroll 2
+            for (; j < rank; j += 4) {
+              const uint32_t wv = __ldg(aw4 + (j >> 2));
+              acc_j((float)(int8_t)(wv & 0xFF), j);
+              acc_j((float)(int8_t)((wv >> 8) & 0xFF), j + 1);
+              acc_j((float)(int8_t)((wv >> 16) & 0xFF), j + 2);
+              acc_j((float)(int8_t)(wv >> 24), j + 3);
+            }
           }
+          for (; j < rank; ++j) acc_j((float)__ldg(arow + j), j);
           const float sc = part == 0 ? sac : saw;
 #pragma unroll
-          for (int k = 0; k < 16; ++k) y[k] = fmaf(sc, lr[k], y[k]);
+          for (int q = 0; q < 16; ++q) y[q] = fmaf(sc, lr[q], y[q]);
         }
-        if (v < p.V) {
+        if (live) {
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const int64_t tok = tok0 + 16 * c + k;
-            if (tok < p.N) p.Y[tok * p.V + v] = y[k];
+          for (int q = 0; q < 16; ++q) {
+            const int64_t tok = tok0 + 16 * c + q;
+            if (tok < p.N) p.Y[tok * p.V + v] = y[q];
           }
         }
       }
+      tc::fence_before_sync();
+      tc::mbar_arrive(&acc_empty[ab]);
     }
   }
 
-  if (warp == 5 && lane == 0) tc::mbar_wait(acc_full, 0, p.err);  // all MMAs retired
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tbase, C::TMEM_COLS);
   }
 }
 
-// FP16 copy of H in the blocked image the MMA's B operand reads: for token tile tt of NT
-// rows and 128-column block kb, a contiguous NT x 128 block whose 16-byte piece (token n,
-// columns 8c..8c+7) sits at ((n / 8) * 16 + c) * 128 + (n % 8) * 16 bytes.  Rows >= N are
-// zero.  Non-finite or out-of-range FP16 values set kErrRangeH.
+// FP16 copy of H in the image the MMA's B operand reads: for token tile tt of NT rows and
+// 128-column block kb, a contiguous NT x 128 block made of two 64-column halves; in half h
+// the 16-byte piece (token n, columns 64h + 8c .. +7) sits at h * NT * 128 + n * 128 +
+// (c ^ (n % 8)) * 16 bytes (K-major, 128-byte swizzle).  Rows >= N are zero.  Non-finite
+// or out-of-range FP16 values set kErrRangeH.
 __global__ void __launch_bounds__(256) convert_h_blocked_kernel(const uint16_t* __restrict__ H,
                                                                 __half* __restrict__ Hb,
                                                                 int64_t N, int64_t Npad,
@@ -315,31 +442,54 @@ __global__ void __launch_bounds__(256) convert_h_blocked_kernel(const uint16_t* 
       out = make_uint4(o[0], o[1], o[2], o[3]);
     }
     const int64_t tt = n / nt, nn = n - tt * nt;
-    const int64_t kb = kc >> 4, c = kc & 15;
-    const int64_t off = (tt * nkb + kb) * (int64_t)nt * 128 + ((nn >> 3) * 16 + c) * 64 + (nn & 7) * 8;
+    const int64_t kb = kc >> 4, half = (kc >> 3) & 1, c = kc & 7;
+    const int64_t off = (tt * nkb + kb) * (int64_t)nt * 128 + half * (int64_t)nt * 64 + nn * 64 +
+                        ((c ^ (nn & 7)) * 8);
     *reinterpret_cast<uint4*>(Hb + off) = out;
   }
   if (bad) atomicOr(err, kErrRangeH);
 }
 
-template <int NT, int CPC>
+template <int NT, int CPC, int DQ>
 cudaError_t launch_tc_cfg(const TcParams& p, cudaStream_t st) {
   const int RR = p.r_c + p.r_r;
-  const size_t smem = tc_smem_bytes<NT>(RR);
-  auto kern = residual_tc_kernel<NT, CPC>;
+  const size_t smem = tc_smem_bytes<NT>(RR, (int)(p.D >> p.g_shift));
+  auto kern = residual_tc_kernel<NT, CPC, DQ>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)((p.N + NT - 1) / NT), (unsigned)((p.V + 127) / 128));
-  kern<<<grid, kTcThreads, smem, st>>>(p);
+  int dev = 0, sms = 0, smem_sm = 0, regs_sm = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) !=
+          cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev)) !=
+          cudaSuccess)
+    return e;
+  cudaFuncAttributes fa;
+  if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
+  // resident CTAs per SM: registers (allocated per warp in units of 256), shared memory
+  // (plus the 1 KB the driver reserves per CTA), warps, and tensor-memory columns
+  const int warps = kTcThreads / 32;
+  const int regs_warp = (fa.numRegs * 32 + 255) / 256 * 256;
+  int occ = regs_sm / (regs_warp * warps);
+  const int by_smem = smem_sm / (int)(smem + fa.sharedSizeBytes + 1024);
+  if (by_smem < occ) occ = by_smem;
+  if (64 / warps < occ) occ = 64 / warps;
+  if (512 / TcCfg<NT>::TMEM_COLS < occ) occ = 512 / TcCfg<NT>::TMEM_COLS;
+  if (occ < 1) occ = 1;
+  int64_t items = p.n_vtiles * p.n_tok_tiles;
+  int64_t grid = (int64_t)sms * occ;
+  if (grid > items) grid = items;
+  kern<<<(unsigned)grid, kTcThreads, smem, st>>>(p);
   return cudaGetLastError();
 }
 
 template <int NT>
 cudaError_t launch_tc_nt(const TcParams& p, int g, cudaStream_t st) {
-  if (g == 32) return launch_tc_cfg<NT, 4>(p, st);
-  if (g == 64) return launch_tc_cfg<NT, 2>(p, st);
-  return launch_tc_cfg<NT, 1>(p, st);
+  if (g == 32) return launch_tc_cfg<NT, 4, 1>(p, st);
+  if (g == 64) return launch_tc_cfg<NT, 2, 1>(p, st);
+  return launch_tc_cfg<NT, 1, 1>(p, st);
 }
 
 }  // namespace
@@ -389,6 +539,8 @@ cudaError_t launch_residual_tc(const __half* Hb, const float* t, const archead_h
   p.g_shift = gs;
   p.err = err;
   const int nt = tc_token_tile(s.N, s.r_c + s.r_r);
+  p.n_tok_tiles = (int)((s.N + nt - 1) / nt);
+  p.n_vtiles = (s.V + 127) / 128;
   cudaError_t e;
   switch (nt) {
     case 16: e = launch_tc_nt<16>(p, s.g, st); break;

@@ -134,6 +134,21 @@ __device__ __forceinline__ uint64_t smem_desc_kmajor(uint32_t saddr, uint32_t lb
   return d;                // base offset 0, layout type 0 (no swizzle)
 }
 
+// Shared-memory matrix descriptor, K-major with the 128-byte swizzle: rows of 128 bytes
+// (64 FP16) in 8-row atoms of 1024 bytes, 16-byte chunk c of row r stored at chunk
+// position c ^ (r % 8) (the hardware XORs address bits 4-6 with bits 7-9).  sbo = 1024,
+// the distance between 8-row atoms; the K offset inside an atom is added to the start
+// address.  The atoms must be 1024-byte aligned.
+__device__ __forceinline__ uint64_t smem_desc_kmajor_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1 << 16;                    // leading byte offset (unused here): 16 bytes
+  d |= (uint64_t)(1024 >> 4) << 32;          // stride byte offset: 1024
+  d |= (uint64_t)1 << 46;                    // descriptor version for sm_100
+  d |= (uint64_t)2 << 61;                    // layout type: 128-byte swizzle
+  return d;
+}
+
 // D[tmem] (+)= A[tmem] * B[smem]^T, one M=128 x N x K=16 step, issued by one thread.
 __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                            uint32_t idesc, uint32_t accumulate) {

@@ -139,9 +139,13 @@ def test_host_entry_points_match_device(dev, rhead):
 
 
 def test_launch_counts(dev, rhead):
+    """Kernels per call: small-batch logits = FP16 H, t, H group sums, contraction;
+    larger batches = blocked FP16 H, t, contraction; NLL = FP16 H, t, contraction, combine."""
     head, dh = rhead
     H = _rand_H(4, 512, 1).to(dev)
     ah.logits(H, dh)
+    assert ah.last_launches() == 4
+    ah.logits(_rand_H(40, 512, 2).to(dev), dh)
     assert ah.last_launches() == 3
     ah.nll(H, dh, make_targets(4, head["V"], 1).to(dev))
     assert ah.last_launches() == 4
