@@ -119,17 +119,15 @@ int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* ta
   int launches = 0;
   const int RR = s.r_c + s.r_r;
   const bool nll_mode = nll != nullptr;
-  // logits: N <= 16 small-batch decode kernel; larger N the tensor-memory (tcgen05) kernel;
-  // the fused NLL runs on the warp-MMA kernel with its split-vocabulary epilogue
-  const bool use_dec = !nll_mode && s.N <= 16;
-  const bool use_tc = !nll_mode && !use_dec;
+  // N <= 8 on the warp-MMA kernel (one token block), larger N on the tensor-memory
+  // (tcgen05) kernel; both have a fused split-vocabulary NLL epilogue
+  const bool use_tc = s.N > 8;
   const int64_t tb = use_tc ? tc_token_tile(s.N, RR) : residual_token_block(s.N);
   const int64_t Npad = (s.N + tb - 1) / tb * tb;
   const int nvblk = residual_gemm_vblocks(s);
   Carve cv;
   const size_t o_hh = cv.take((size_t)Npad * s.D * 2);
   const size_t o_t = cv.take((size_t)s.N * RR * 4);
-  const size_t o_hsum = use_dec ? cv.take((size_t)s.N * (s.D / s.g) * 4) : 0;
   const size_t o_part = nll_mode ? cv.take((size_t)s.N * nvblk * 8) : 0;
   const size_t o_tl = nll_mode ? cv.take((size_t)s.N * 4) : 0;
   void* base = nullptr;
@@ -145,14 +143,14 @@ int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* ta
                          : launch_prologue(H, head, s, Npad, Hh, t, ds->err, st, &launches);
   if (e == cudaSuccess) {
     if (use_tc) {
+      float2* part = nll_mode ? reinterpret_cast<float2*>(b + o_part) : nullptr;
+      float* tl = nll_mode ? reinterpret_cast<float*>(b + o_tl) : nullptr;
       prof_mark(0, st);
-      e = launch_residual_tc(Hh, t, head, s, Y, ds->err, st, &launches);
+      e = launch_residual_tc(Hh, t, head, s, nll_mode ? nullptr : Y, targets, part, tl, ds->err,
+                             st, &launches);
       prof_mark(1, st);
-    } else if (use_dec) {
-      prof_mark(0, st);
-      e = launch_decode_mma(H, Hh, t, reinterpret_cast<float*>(b + o_hsum), head, s, Y, st,
-                            &launches);
-      prof_mark(1, st);
+      if (e == cudaSuccess && nll_mode)
+        e = launch_nll_combine(part, tl, targets, s, nll, ds->err, st, &launches);
     } else if (!nll_mode) {
       prof_mark(0, st);
       e = launch_residual_gemm(Hh, t, head, s, Y, nullptr, nullptr, nullptr, st, &launches, 0);

@@ -79,17 +79,6 @@ __device__ __forceinline__ void dequant_word_lite(uint32_t w, __half2 c2, __half
   out[3] = __hmul2(__hfma2(*reinterpret_cast<__half2*>(&x3), k16, k72), c2);
 }
 
-// The four FP16 pairs of one device-layout word as 1032 + q (offset-binary nibble under
-// the exponent of 1024, unit 1): three shifts and four LOP3, no FP16 arithmetic.  A
-// contraction over these values equals the contraction over q plus 1032 times the sum of
-// the other operand, which the caller removes.  Pair i holds (column 2i, column 2i + 1).
-__device__ __forceinline__ void magic_word(uint32_t w, uint32_t out[4]) {
-  out[0] = and_xor(w, 0x000F000Fu, 0x64086408u);
-  out[1] = and_xor(w >> 4, 0x000F000Fu, 0x64086408u);
-  out[2] = and_xor(w >> 8, 0x000F000Fu, 0x64086408u);
-  out[3] = and_xor(w >> 12, 0x000F000Fu, 0x64086408u);
-}
-
 // Device nibble layout, tiled: rows are padded to a multiple of 128 and every 128-row
 // tile's 128-column block (64 bytes per row) is one contiguous 8 KB region, so each tile
 // streams sequentially from HBM.  Inside the region, 16-byte chunk i (i = 0..3) of row s
@@ -162,16 +151,11 @@ int tc_token_tile(int64_t N, int RR);
 cudaError_t launch_prologue_blocked(const uint16_t* H, const archead_head* head,
                                     const Shapes& s, int nt, __half* Hb, float* t,
                                     unsigned* err, cudaStream_t st, int* launches);
+// Y != nullptr: write logits.  Y == nullptr: fused NLL, writing (max, sum exp) partials
+// into part[N x ceil(V/128)] and target logits into tlogit[N] (see launch_nll_combine).
 cudaError_t launch_residual_tc(const __half* Hb, const float* t, const archead_head* head,
-                               const Shapes& s, float* Y, unsigned* err, cudaStream_t st,
-                               int* launches);
-
-// Small-batch decode (N <= 16): independent warps, per-warp cp.async rings, warp MMAs;
-// Hh is the row-major FP16 copy of H padded to residual_token_block(N) rows; hsum
-// (N x D/g FP32 scratch) receives 1032 times each token's sum of H over each group.
-cudaError_t launch_decode_mma(const uint16_t* H, const __half* Hh, const float* t,
-                              float* hsum, const archead_head* head, const Shapes& s,
-                              float* Y, cudaStream_t st, int* launches);
+                               const Shapes& s, float* Y, const int32_t* targets, float2* part,
+                               float* tlogit, unsigned* err, cudaStream_t st, int* launches);
 
 // Residual dequant-contraction over token blocks of up to 64 (mma.sync path).
 // mode 0: write logits Y.  mode 1: write NLL partials (max, sum exp) per (token, vocabulary

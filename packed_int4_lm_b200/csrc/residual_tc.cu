@@ -4,8 +4,9 @@
 //
 // Persistent, warp-specialised kernel.  A work item is one 128-row vocabulary tile for one
 // tile of NT tokens (NT = 16..128):
-//  * warp 8 (one thread) feeds three shared-memory rings with bulk copies (TMA engine, no
-//    tensor map, no multicast): the tile's 8 KB packed-nibble block per 128 columns (the
+//  * warp 8 (two threads, independent streams) feeds three shared-memory rings with bulk
+//    copies (TMA engine, no tensor map, no multicast): the tile's 8 KB packed-nibble block
+//    per 128 columns (the
 //    tiled device layout makes it one contiguous region), the tile's group-scale codes once
 //    per item, and the token tile's FP16 H block (pre-arranged by the prologue as the
 //    128-byte-swizzled K-major image the MMA reads);
@@ -43,6 +44,9 @@ struct TcParams {
   const int8_t* Aw;
   const float* sAw;
   float* Y;
+  const int32_t* targets;  // fused NLL: target ids (N)
+  float2* part;            // fused NLL: (max, sum exp) per (token, vocabulary tile)
+  float* tlogit;           // fused NLL: the target's logit per token
   int64_t N, V, D;
   int r_c, r_r, g_shift;
   int n_tok_tiles;
@@ -64,11 +68,17 @@ struct TcCfg {
 
 __host__ __device__ inline size_t round16(size_t x) { return (x + 15) & ~(size_t)15; }
 
+// fused-NLL scratch: a 16-token x 128-row transposed logit chunk plus the tile's targets
 template <int NT>
+constexpr size_t nll_scratch_bytes() {
+  return (size_t)16 * 128 * 4 + (size_t)NT * 4;
+}
+
+template <int NT, int MODE>
 size_t tc_smem_bytes(int RR, int G) {
   using C = TcCfg<NT>;
   return (size_t)C::SB * C::HSTAGE + (size_t)C::SP * kPkBytes + 2 * round16((size_t)128 * G) +
-         round16((size_t)RR * NT * 4) + 512;
+         round16((size_t)RR * NT * 4) + (MODE ? nll_scratch_bytes<NT>() : 0) + 512;
 }
 
 // The k-th work item of this CTA: its tile's first row, its row limit, its token tile.
@@ -95,7 +105,7 @@ __device__ __forceinline__ bool get_item(const TcParams& p, int k, Item& it) {
   return true;
 }
 
-template <int NT, int CPC, int DQ>
+template <int NT, int CPC, int DQ, int MODE>
 __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcParams p) {
   using C = TcCfg<NT>;
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -108,8 +118,12 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
   unsigned char* pk = Hs + C::SB * C::HSTAGE;
   unsigned char* cds = pk + C::SP * kPkBytes;  // [2][128 x G]
   float* ts = reinterpret_cast<float*>(cds + 2 * round16(code_bytes));  // ts[j * NT + n]
-  uint64_t* bars =
-      reinterpret_cast<uint64_t*>(reinterpret_cast<unsigned char*>(ts) + round16((size_t)RR * NT * 4));
+  float* nll_y = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(ts) +
+                                          round16((size_t)RR * NT * 4));  // [16][128]
+  int32_t* tgt_s = reinterpret_cast<int32_t*>(nll_y + 16 * 128);          // [NT]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<unsigned char*>(ts) +
+                                               round16((size_t)RR * NT * 4) +
+                                               (MODE ? nll_scratch_bytes<NT>() : 0));
   uint64_t* b_full = bars;
   uint64_t* b_empty = b_full + C::SB;
   uint64_t* p_full = b_empty + C::SB;
@@ -155,11 +169,12 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
   const uint32_t acol = tbase + 2 * NT;  // A ring after the two accumulators (lane 0)
 
   if (warp == 8) {
-    // ---------------- producer: codes, packed blocks, H blocks ----------------
+    // ---------------- producers: lane 0 codes + packed blocks, lane 1 H blocks ----------
+    // Two independent streams, so the packed prefetch is not held back by the H ring
+    // (whose stages free up only as MMAs retire).
     if (lane == 0) {
-      int k = 0;
+      int k = 0, np = 0, nc = 0;
       bool ok = true;
-      int nb_issued = 0, np_issued = 0, nc_issued = 0;
       Item it;
       for (int i = 0; ok && get_item(p, i, it); ++i) {
         const int cs = i & 1;
@@ -167,38 +182,51 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
           ok = false;
           break;
         }
+        tc::fence_proxy_async_smem();  // the stage was read with generic loads
         tc::mbar_arrive_expect_tx(&c_full[cs], (uint32_t)code_bytes);
         tc::bulk_g2s(cds + cs * round16(code_bytes), p.code + it.row0 * G, (uint32_t)code_bytes,
                      &c_full[cs]);
-        ++nc_issued;
+        ++nc;
         const uint8_t* psrc = p.nib + ((it.vt * nkb) << 13);
-        const unsigned char* hsrc =
-            reinterpret_cast<const unsigned char*>(p.Hb) + (int64_t)it.tt * nkb * C::HSTAGE;
         for (int kb = 0; kb < nkb; ++kb, ++k) {
-          const int sp = k % C::SP, sb = k % C::SB;
+          const int sp = k % C::SP;
           if (k >= C::SP && !tc::mbar_wait(&p_empty[sp], ((k / C::SP) - 1) & 1, p.err)) {
             ok = false;
             break;
           }
+          tc::fence_proxy_async_smem();  // the stage was read with generic loads
           tc::mbar_arrive_expect_tx(&p_full[sp], kPkBytes);
           tc::bulk_g2s(pk + sp * kPkBytes, psrc + ((int64_t)kb << 13), kPkBytes, &p_full[sp]);
-          ++np_issued;
+          ++np;
+        }
+      }
+      if (!ok) {  // drain copies still in flight before the CTA exits
+        for (int q = np - C::SP < 0 ? 0 : np - C::SP; q < np; ++q)
+          tc::mbar_wait(&p_full[q % C::SP], (q / C::SP) & 1, p.err);
+        for (int q = nc - 2 < 0 ? 0 : nc - 2; q < nc; ++q)
+          tc::mbar_wait(&c_full[q & 1], (q >> 1) & 1, p.err);
+      }
+    } else if (lane == 1) {
+      int k = 0, nb = 0;
+      bool ok = true;
+      Item it;
+      for (int i = 0; ok && get_item(p, i, it); ++i) {
+        const unsigned char* hsrc =
+            reinterpret_cast<const unsigned char*>(p.Hb) + (int64_t)it.tt * nkb * C::HSTAGE;
+        for (int kb = 0; kb < nkb; ++kb, ++k) {
+          const int sb = k % C::SB;
           if (k >= C::SB && !tc::mbar_wait(&b_empty[sb], ((k / C::SB) - 1) & 1, p.err)) {
             ok = false;
             break;
           }
           tc::mbar_arrive_expect_tx(&b_full[sb], C::HSTAGE);
           tc::bulk_g2s(Hs + sb * C::HSTAGE, hsrc + (int64_t)kb * C::HSTAGE, C::HSTAGE, &b_full[sb]);
-          ++nb_issued;
+          ++nb;
         }
       }
-      if (!ok) {  // drain copies that may still be in flight before the CTA exits
-        for (int q = nb_issued - C::SB < 0 ? 0 : nb_issued - C::SB; q < nb_issued; ++q)
+      if (!ok) {
+        for (int q = nb - C::SB < 0 ? 0 : nb - C::SB; q < nb; ++q)
           tc::mbar_wait(&b_full[q % C::SB], (q / C::SB) & 1, p.err);
-        for (int q = np_issued - C::SP < 0 ? 0 : np_issued - C::SP; q < np_issued; ++q)
-          tc::mbar_wait(&p_full[q % C::SP], (q / C::SP) & 1, p.err);
-        for (int q = nc_issued - 2 < 0 ? 0 : nc_issued - 2; q < nc_issued; ++q)
-          tc::mbar_wait(&c_full[q & 1], (q >> 1) & 1, p.err);
       }
     }
   } else if (warp == 9) {
@@ -330,10 +358,13 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
           const int64_t tok = tok0 + n;
           ts[q] = tok < p.N ? __ldg(p.t + tok * RR + j) : 0.f;
         }
+        if (MODE == 1)
+          for (int q = e; q < NT; q += 128) tgt_s[q] = tok0 + q < p.N ? __ldg(p.targets + tok0 + q) : -1;
         asm volatile("bar.sync 1, 128;\n" ::: "memory");
         cur_tt = it.tt;
       }
-      if (!__all_sync(0xffffffffu, tc::mbar_wait(&acc_full[ab], (i >> 1) & 1, p.err))) break;
+      // one outcome for all four epilogue warps: they share named barriers below
+      if (!tc::bar_and(1, 128, tc::mbar_wait(&acc_full[ab], (i >> 1) & 1, p.err))) break;
       tc::fence_after_sync();
       const int64_t v = it.row0 + e;
       const bool live = v < it.row_end;
@@ -388,12 +419,46 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
 #pragma unroll
           for (int q = 0; q < 16; ++q) y[q] = fmaf(sc, lr[q], y[q]);
         }
-        if (live) {
+        if (MODE == 0) {
+          if (live) {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+              const int64_t tok = tok0 + 16 * c + q;
+              if (tok < p.N) p.Y[tok * p.V + v] = y[q];
+            }
+          }
+        } else {
+          // ---- fused NLL: per token of the chunk, (max, sum exp) over the tile's rows ----
+          const float NEG_INF = __int_as_float(0xff800000);
 #pragma unroll
           for (int q = 0; q < 16; ++q) {
-            const int64_t tok = tok0 + 16 * c + q;
-            if (tok < p.N) p.Y[tok * p.V + v] = y[q];
+            nll_y[q * 128 + e] = live ? y[q] : NEG_INF;
+            const int tg = tgt_s[16 * c + q];
+            if (live && tg == v) p.tlogit[tok0 + 16 * c + q] = y[q];
           }
+          asm volatile("bar.sync 1, 128;\n" ::: "memory");
+          // thread e: token q = e / 8 of the chunk, rows 16 * (e % 8) .. +15
+          const int q = e >> 3, seg = e & 7;
+          const float* yr = nll_y + q * 128 + 16 * seg;
+          float m = NEG_INF;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) m = fmaxf(m, yr[i]);
+          float sm = 0.f;
+          if (m != NEG_INF) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) sm += __expf(yr[i] - m);
+          }
+#pragma unroll
+          for (int o = 1; o < 8; o <<= 1) {  // combine the 8 segments of the token
+            const float mo = __shfl_xor_sync(0xffffffffu, m, o);
+            const float so = __shfl_xor_sync(0xffffffffu, sm, o);
+            const float mn = fmaxf(m, mo);
+            sm = (m == NEG_INF ? 0.f : sm * __expf(m - mn)) + (mo == NEG_INF ? 0.f : so * __expf(mo - mn));
+            m = mn;
+          }
+          const int64_t tok = tok0 + 16 * c + q;
+          if (seg == 0 && tok < p.N) p.part[tok * p.n_vtiles + it.vt] = make_float2(m, sm);
+          asm volatile("bar.sync 1, 128;\n" ::: "memory");
         }
       }
       tc::fence_before_sync();
@@ -450,11 +515,11 @@ __global__ void __launch_bounds__(256) convert_h_blocked_kernel(const uint16_t* 
   if (bad) atomicOr(err, kErrRangeH);
 }
 
-template <int NT, int CPC, int DQ>
+template <int NT, int CPC, int DQ, int MODE>
 cudaError_t launch_tc_cfg(const TcParams& p, cudaStream_t st) {
   const int RR = p.r_c + p.r_r;
-  const size_t smem = tc_smem_bytes<NT>(RR, (int)(p.D >> p.g_shift));
-  auto kern = residual_tc_kernel<NT, CPC, DQ>;
+  const size_t smem = tc_smem_bytes<NT, MODE>(RR, (int)(p.D >> p.g_shift));
+  auto kern = residual_tc_kernel<NT, CPC, DQ, MODE>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -485,11 +550,21 @@ cudaError_t launch_tc_cfg(const TcParams& p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <int NT>
+template <int NT, int MODE>
 cudaError_t launch_tc_nt(const TcParams& p, int g, cudaStream_t st) {
-  if (g == 32) return launch_tc_cfg<NT, 4, 1>(p, st);
-  if (g == 64) return launch_tc_cfg<NT, 2, 1>(p, st);
-  return launch_tc_cfg<NT, 1, 1>(p, st);
+  if (g == 32) return launch_tc_cfg<NT, 4, 1, MODE>(p, st);
+  if (g == 64) return launch_tc_cfg<NT, 2, 1, MODE>(p, st);
+  return launch_tc_cfg<NT, 1, 1, MODE>(p, st);
+}
+
+template <int MODE>
+cudaError_t launch_tc_mode(const TcParams& p, int nt, int g, cudaStream_t st) {
+  switch (nt) {
+    case 16: return launch_tc_nt<16, MODE>(p, g, st);
+    case 32: return launch_tc_nt<32, MODE>(p, g, st);
+    case 64: return launch_tc_nt<64, MODE>(p, g, st);
+    default: return launch_tc_nt<128, MODE>(p, g, st);
+  }
 }
 
 }  // namespace
@@ -516,8 +591,8 @@ cudaError_t launch_prologue_blocked(const uint16_t* H, const archead_head* head,
 }
 
 cudaError_t launch_residual_tc(const __half* Hb, const float* t, const archead_head* head,
-                               const Shapes& s, float* Y, unsigned* err, cudaStream_t st,
-                               int* launches) {
+                               const Shapes& s, float* Y, const int32_t* targets, float2* part,
+                               float* tlogit, unsigned* err, cudaStream_t st, int* launches) {
   TcParams p;
   p.Hb = Hb;
   p.t = t;
@@ -529,6 +604,9 @@ cudaError_t launch_residual_tc(const __half* Hb, const float* t, const archead_h
   p.Aw = head->Aw;
   p.sAw = head->sAw;
   p.Y = Y;
+  p.targets = targets;
+  p.part = part;
+  p.tlogit = tlogit;
   p.N = s.N;
   p.V = s.V;
   p.D = s.D;
@@ -541,13 +619,7 @@ cudaError_t launch_residual_tc(const __half* Hb, const float* t, const archead_h
   const int nt = tc_token_tile(s.N, s.r_c + s.r_r);
   p.n_tok_tiles = (int)((s.N + nt - 1) / nt);
   p.n_vtiles = (s.V + 127) / 128;
-  cudaError_t e;
-  switch (nt) {
-    case 16: e = launch_tc_nt<16>(p, s.g, st); break;
-    case 32: e = launch_tc_nt<32>(p, s.g, st); break;
-    case 64: e = launch_tc_nt<64>(p, s.g, st); break;
-    default: e = launch_tc_nt<128>(p, s.g, st); break;
-  }
+  cudaError_t e = Y ? launch_tc_mode<0>(p, nt, s.g, st) : launch_tc_mode<1>(p, nt, s.g, st);
   ++*launches;
   return e;
 }

@@ -52,6 +52,30 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
   return true;
 }
 
+// Named barrier `id` over `count` threads that also returns the AND of their predicates,
+// so a group of warps agrees on one outcome (e.g. whether a bounded wait succeeded).
+__device__ __forceinline__ bool bar_and(uint32_t id, uint32_t count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
+// Orders this thread's view of prior generic-proxy shared-memory accesses (made visible to
+// it through an mbarrier wait) before its subsequent async-proxy operations.  A producer
+// issues it after waiting for consumers that READ a stage with ordinary loads and before
+// the bulk copy that overwrites the stage: without it that write-after-read is not ordered
+// across the two proxies, and a refill can race with the last reads.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+
 // ---- bulk copy global -> shared (TMA engine, no tensor map, no multicast) ---------------
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
                                          uint64_t* bar) {

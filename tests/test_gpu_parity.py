@@ -114,7 +114,7 @@ def test_nll_head_is_in_logit_regime(nhead):
     assert 0.5 < rms < 20, rms
 
 
-@pytest.mark.parametrize("N", [1, 7, 64, 100])
+@pytest.mark.parametrize("N", [1, 7, 8, 9, 64, 100, 130, 300])
 def test_nll_random_head(dev, nhead, N):
     head, dh = nhead
     H = _rand_H(N, 512, 300 + N)
@@ -124,6 +124,32 @@ def test_nll_random_head(dev, nhead, N):
     ref = oracle.nll(head, bf16_bits(H), tg.numpy())
     err = np.max(np.abs(out.cpu().double().numpy() - ref))
     assert err <= NLL_TOL, err
+
+
+def test_many_items_per_cta_consistent(dev):
+    """A vocabulary large enough that every persistent CTA of the tensor-memory kernel runs
+    several 128-row tiles, repeated: the first 16 tokens of N = 64 and N = 32 calls must
+    match the N = 16 call tile for tile, and sampled rows must match the oracle.  Races
+    between the producer's bulk copies and the consumers' reads of a ring stage show up
+    here as a few corrupted tiles."""
+    V, D = 151936, 4096
+    head = random_canonical_head(V, D, 32, 32, 128, seed=40, super_exp_range=(-17, -13),
+                                 factor_exp_range=(-13, -10))
+    dh = ah.DeviceHead.from_canonical(head, dev)
+    H = _rand_H(64, D, 41)
+    Hd = H.to(dev)
+    Y16 = ah.logits(Hd[:16].contiguous(), dh)
+    ah.check()
+    rows = np.arange(0, V, 97)
+    Yref = oracle.logits(head, bf16_bits(H[:16]), rows=rows)
+    _assert_logits(Y16.cpu().numpy()[:, rows], Yref, "N=16 sampled rows")
+    tol = 1e-4 * float(Y16.abs().max())
+    for rep in range(4):
+        for N in (64, 32):
+            Yn = ah.logits(Hd[:N].contiguous(), dh)
+            ah.check()
+            diff = float((Yn[:16] - Y16).abs().max())
+            assert diff <= tol, (rep, N, diff, tol)
 
 
 def test_host_entry_points_match_device(dev, rhead):
@@ -139,12 +165,12 @@ def test_host_entry_points_match_device(dev, rhead):
 
 
 def test_launch_counts(dev, rhead):
-    """Kernels per call: small-batch logits = FP16 H, t, H group sums, contraction;
-    larger batches = blocked FP16 H, t, contraction; NLL = FP16 H, t, contraction, combine."""
+    """Kernels per call: logits = FP16 H (row-major or blocked), t, contraction;
+    NLL = FP16 H, t, contraction, combine."""
     head, dh = rhead
     H = _rand_H(4, 512, 1).to(dev)
     ah.logits(H, dh)
-    assert ah.last_launches() == 4
+    assert ah.last_launches() == 3
     ah.logits(_rand_H(40, 512, 2).to(dev), dh)
     assert ah.last_launches() == 3
     ah.nll(H, dh, make_targets(4, head["V"], 1).to(dev))
