@@ -120,14 +120,17 @@ int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* ta
   const int RR = s.r_c + s.r_r;
   const bool nll_mode = nll != nullptr;
   // N <= 8 on the warp-MMA kernel (one token block), larger N on the tensor-memory
-  // (tcgen05) kernel; both have a fused split-vocabulary NLL epilogue
-  const bool use_tc = s.N > 8;
-  const int64_t tb = use_tc ? tc_token_tile(s.N, RR) : residual_token_block(s.N);
+  // (tcgen05) kernel when its shared-memory rings fit the shape; both have a fused
+  // split-vocabulary NLL epilogue
+  const TcPlan plan = s.N > 8 ? tc_plan(s, nll_mode) : TcPlan{0, 0, 0};
+  const bool use_tc = plan.nt > 0;
+  const int64_t tb = use_tc ? plan.nt : residual_token_block(s.N);
   const int64_t Npad = (s.N + tb - 1) / tb * tb;
   const int nvblk = residual_gemm_vblocks(s);
   Carve cv;
-  const size_t o_hh = cv.take((size_t)Npad * s.D * 2);
-  const size_t o_t = cv.take((size_t)s.N * RR * 4);
+  // tcgen05: the B image holds H and the rank blocks; warp MMAs: FP16 H plus FP32 t
+  const size_t o_hh = cv.take((size_t)Npad * (s.D + (use_tc ? 128 * plan.nrb : 0)) * 2);
+  const size_t o_t = cv.take(use_tc ? 0 : (size_t)s.N * RR * 4);
   const size_t o_part = nll_mode ? cv.take((size_t)s.N * nvblk * 8) : 0;
   const size_t o_tl = nll_mode ? cv.take((size_t)s.N * 4) : 0;
   void* base = nullptr;
@@ -138,16 +141,15 @@ int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* ta
   char* b = static_cast<char*>(base);
   __half* Hh = reinterpret_cast<__half*>(b + o_hh);
   float* t = reinterpret_cast<float*>(b + o_t);
-  cudaError_t e = use_tc ? launch_prologue_blocked(H, head, s, (int)tb, Hh, t, ds->err, st,
-                                                   &launches)
+  cudaError_t e = use_tc ? launch_prologue_blocked(H, head, s, plan, Hh, ds->err, st, &launches)
                          : launch_prologue(H, head, s, Npad, Hh, t, ds->err, st, &launches);
   if (e == cudaSuccess) {
     if (use_tc) {
       float2* part = nll_mode ? reinterpret_cast<float2*>(b + o_part) : nullptr;
       float* tl = nll_mode ? reinterpret_cast<float*>(b + o_tl) : nullptr;
       prof_mark(0, st);
-      e = launch_residual_tc(Hh, t, head, s, nll_mode ? nullptr : Y, targets, part, tl, ds->err,
-                             st, &launches);
+      e = launch_residual_tc(Hh, head, s, plan, nll_mode ? nullptr : Y, targets, part, tl,
+                             ds->err, st, &launches);
       prof_mark(1, st);
       if (e == cudaSuccess && nll_mode)
         e = launch_nll_combine(part, tl, targets, s, nll, ds->err, st, &launches);

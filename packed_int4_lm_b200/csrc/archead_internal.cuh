@@ -141,21 +141,44 @@ cudaError_t launch_prologue(const uint16_t* H, const archead_head* head, const S
                             int64_t Npad, __half* Hh, float* t, unsigned* err,
                             cudaStream_t st, int* launches);
 
-// t = H [Q8(B_c) | Q8(B_w)]^T alone (N x (r_c + r_r) FP32).
+// t = H [Q8(B_c) | Q8(B_w)]^T (N x (r_c + r_r) FP32).  With img != nullptr the products
+// go instead, split into FP16 pieces, into the rank blocks of the tcgen05 B image (token
+// tile nt, nkbt blocks per tile); a piece outside the FP16 range sets kErrRangeH.
 cudaError_t launch_lowrank_t(const uint16_t* H, const archead_head* head, const Shapes& s,
-                             float* t, cudaStream_t st, int* launches);
+                             float* t, __half* img, int nt, int64_t nkbt, unsigned* err,
+                             cudaStream_t st, int* launches);
 
-// tcgen05 path: token tile (16, 32, 64 or 128) for N tokens and r_c + r_r = RR; the
-// blocked FP16 copy of H (Npad = N rounded up to the tile) and t; the contraction.
-int tc_token_tile(int64_t N, int RR);
+// tcgen05 path.  The MMA's B operand is a blocked FP16 image of the tokens: per token tile
+// of nt rows, nkb = D / 128 blocks of H followed by nrb = ceil((r_c + r_r) / 32) rank
+// blocks, each nt x 128 FP16 (see tc_image_offset).  Rank block b holds, for the factor
+// index j = 32 b + i (i < 32), columns 4i..4i+3 = (t1, t2, t1, t2), where t1 = fp16(t_j)
+// and t2 = fp16(t_j - t1) split the FP32 left product t = H [Q8(B_c) | Q8(B_w)]^T.
+struct TcPlan {
+  int nt;   // token tile: 16, 32, 64 or 128 (0: the shape does not fit this kernel)
+  int sb;   // stages of the shared-memory ring of B blocks
+  int nrb;  // rank blocks after the nkb blocks of H
+};
+TcPlan tc_plan(const Shapes& s, bool nll);
+// FP16 element offset of (token nn of token tile tt, column kk < 128 of block kb) in the
+// blocked image with nkbt blocks per token tile: two 64-column halves of nt rows x 128
+// bytes, the 16-byte chunk c of row nn stored at chunk c ^ (nn % 8) (the K-major 128-byte
+// swizzle the MMA's shared-memory descriptor names).
+__host__ __device__ __forceinline__ int64_t tc_image_offset(int64_t tt, int64_t kb,
+                                                            int64_t nkbt, int nt, int64_t nn,
+                                                            int kk) {
+  return (tt * nkbt + kb) * (int64_t)nt * 128 + (int64_t)(kk >> 6) * nt * 64 + nn * 64 +
+         ((((kk >> 3) & 7) ^ (int)(nn & 7)) << 3) + (kk & 7);
+}
+// Blocked image of H (zero rows up to the token tile) and its rank blocks.
 cudaError_t launch_prologue_blocked(const uint16_t* H, const archead_head* head,
-                                    const Shapes& s, int nt, __half* Hb, float* t,
+                                    const Shapes& s, const TcPlan& plan, __half* Hb,
                                     unsigned* err, cudaStream_t st, int* launches);
 // Y != nullptr: write logits.  Y == nullptr: fused NLL, writing (max, sum exp) partials
 // into part[N x ceil(V/128)] and target logits into tlogit[N] (see launch_nll_combine).
-cudaError_t launch_residual_tc(const __half* Hb, const float* t, const archead_head* head,
-                               const Shapes& s, float* Y, const int32_t* targets, float2* part,
-                               float* tlogit, unsigned* err, cudaStream_t st, int* launches);
+cudaError_t launch_residual_tc(const __half* Hb, const archead_head* head, const Shapes& s,
+                               const TcPlan& plan, float* Y, const int32_t* targets,
+                               float2* part, float* tlogit, unsigned* err, cudaStream_t st,
+                               int* launches);
 
 // Residual dequant-contraction over token blocks of up to 64 (mma.sync path).
 // mode 0: write logits Y.  mode 1: write NLL partials (max, sum exp) per (token, vocabulary

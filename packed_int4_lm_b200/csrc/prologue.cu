@@ -1,7 +1,8 @@
 // Prologue of the ARCHead logit path (ARCHead Sec. 3, the bracket (H B_w^T) of the logit
 // formula, and its core analogue H B_c^T):
 //   * Hh = fp16(H), zero-padded to Npad rows -- the B operand of the residual contraction;
-//   * t  = H [Q8(B_c) | Q8(B_w)]^T, N x (r_c + r_r) FP32 -- the rank terms' left products.
+//   * t  = H [Q8(B_c) | Q8(B_w)]^T, N x (r_c + r_r) FP32 -- the rank terms' left products
+//     (for the tcgen05 path, split into FP16 pieces inside the MMA's B image instead).
 #include "archead_internal.cuh"
 
 namespace archead {
@@ -46,7 +47,8 @@ __global__ void __launch_bounds__(256) lowrank_t_kernel(
     const uint16_t* __restrict__ H, const int8_t* __restrict__ Bc,
     const float* __restrict__ sBc, const int8_t* __restrict__ Bw,
     const float* __restrict__ sBw, int r_c, int r_r, int64_t N, int64_t D, int g,
-    float* __restrict__ t) {
+    float* __restrict__ t, __half* __restrict__ img, int nt, int64_t nkbt,
+    unsigned* err) {
   const int j = blockIdx.y;
   const int RR = r_c + r_r;
   const int8_t* B;
@@ -101,7 +103,20 @@ __global__ void __launch_bounds__(256) lowrank_t_kernel(
     float v = 0.f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) v += red[w][threadIdx.x];
-    t[(n0 + threadIdx.x) * RR + j] = v;
+    const int64_t n = n0 + threadIdx.x;
+    if (!img) {
+      t[n * RR + j] = v;
+    } else {
+      // hi / lo FP16 pieces: t1 + t2 carries 22 significant bits of v
+      const __half t1 = __float2half_rn(v);
+      const __half t2 = __float2half_rn(v - __half2float(t1));
+      if (!(fabsf(v) < 65504.f)) atomicOr(err, kErrRangeH);
+      const uint32_t w = (uint32_t)__half_as_ushort(t1) | ((uint32_t)__half_as_ushort(t2) << 16);
+      const int64_t tt = n / nt, nn = n - tt * nt;
+      const int64_t kb = D / 128 + j / 32;
+      *reinterpret_cast<uint2*>(img + tc_image_offset(tt, kb, nkbt, nt, nn, 4 * (j & 31))) =
+          make_uint2(w, w);
+    }
   }
 }
 
@@ -120,16 +135,18 @@ cudaError_t launch_prologue(const uint16_t* H, const archead_head* head, const S
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_lowrank_t(H, head, s, t, st, launches);
+  return launch_lowrank_t(H, head, s, t, nullptr, 0, 0, err, st, launches);
 }
 
 cudaError_t launch_lowrank_t(const uint16_t* H, const archead_head* head, const Shapes& s,
-                             float* t, cudaStream_t st, int* launches) {
+                             float* t, __half* img, int nt, int64_t nkbt, unsigned* err,
+                             cudaStream_t st, int* launches) {
   const int RR = s.r_c + s.r_r;
   if (RR > 0) {
     dim3 grid((unsigned)((s.N + kTN - 1) / kTN), RR);
     lowrank_t_kernel<<<grid, 256, 0, st>>>(H, head->Bc, head->sBc, head->Bw, head->sBw,
-                                           s.r_c, s.r_r, s.N, s.D, s.g, t);
+                                           s.r_c, s.r_r, s.N, s.D, s.g, t, img, nt, nkbt,
+                                           err);
     ++*launches;
   }
   return cudaGetLastError();

@@ -1,25 +1,36 @@
-// Residual contraction on the 5th-generation tensor cores (tcgen05, TMEM accumulators).
+// Logit contraction on the 5th-generation tensor cores (tcgen05, TMEM accumulators).
 //
-//   Y[n, v] = S_v * sum_d h[n, d] q[v, d] c[v, d / g]  +  rank terms        (ARCHead Sec. 3)
+//   Y[n, v] = S_v sum_d h[n, d] q[v, d] c[v, d / g]  +  sum_j a[v, j] t[n, j]   (ARCHead Sec. 3)
+//
+// with a = [Q8(A_c) | Q8(A_w)] (row-scaled INT8) and t = H [Q8(B_c) | Q8(B_w)]^T.  Both sums
+// run on the tensor cores into ONE FP32 accumulator per (row, token), scaled by a per-row
+// S'_v = S_v 2^k_v:
+//   * residual K columns: A = q c 2^-k (exact in FP16 for k <= 24), B = fp16(h);
+//   * rank K columns (4 per factor index j): A = (x1, x1, x2, x2), B = (t1, t2, t1, t2),
+//     where x = a / S' and t are each split into an FP16 hi piece and an FP16 remainder, so
+//     x1 t1 + x1 t2 + x2 t1 + x2 t2 carries about 22 significant bits of a t / S';
+//   * the epilogue writes S'_v times the accumulator.
+// k_v is chosen from the row's scales alone: every factor entry obeys |a| <= 128 max(sAc,
+// sAw), and k puts that bound between 2^12 and 2^14 after division by S', far inside FP16.
 //
 // Persistent, warp-specialised kernel.  A work item is one 128-row vocabulary tile for one
 // tile of NT tokens (NT = 16..128):
 //  * warp 8 (two threads, independent streams) feeds three shared-memory rings with bulk
 //    copies (TMA engine, no tensor map, no multicast): the tile's 8 KB packed-nibble block
-//    per 128 columns (the
-//    tiled device layout makes it one contiguous region), the tile's group-scale codes once
-//    per item, and the token tile's FP16 H block (pre-arranged by the prologue as the
-//    128-byte-swizzled K-major image the MMA reads);
+//    per 128 columns (one contiguous region in the tiled device layout), the tile's
+//    group-scale codes once per item, and the token tile's FP16 B blocks (pre-arranged by
+//    the prologue as the 128-byte-swizzled K-major image the MMA reads);
 //  * warps 0-3 (dequant): one vocabulary row per thread (= one TMEM lane).  A thread reads
-//    its row's four 16-byte chunks of the block (conflict free: chunk i of row s sits at
-//    (i * 128 + s) * 16), dequantises them to exact FP16 q*c and stores them with
+//    its row's four 16-byte chunks of a block (conflict free: chunk i of row s sits at
+//    (i * 128 + s) * 16), dequantises them to exact FP16 q c 2^-k, and after the residual
+//    blocks converts its row's factor entries into the rank blocks; it stores both with
 //    tcgen05.st into an A ring of 2-4 stages in tensor memory (128 x 128 FP16 = 64
-//    columns per stage); the dequant warps issue no global loads;
+//    columns per stage);
 //  * warp 9 (one thread): issues tcgen05.mma kind::f16, A from tensor memory, B from
-//    shared memory, eight K=16 steps per block, into one of two M=128 x N=NT FP32
-//    accumulators, so the next item's MMAs overlap the previous item's epilogue;
-//  * warps 4-7 (epilogue): tcgen05.ld of an accumulator row, times S_v, plus the core and
-//    correction rank terms from t staged in shared memory, stored coalesced into Y.
+//    shared memory, K=16 steps, into one of two M=128 x N=NT FP32 accumulators, so the
+//    next item's MMAs overlap the previous item's epilogue;
+//  * warps 4-7 (epilogue): tcgen05.ld of an accumulator row, times S'_v, stored coalesced
+//    into Y, or reduced on chip into split-vocabulary log-sum-exp partials (fused NLL).
 // Scheduling: with a single token tile (decode) every CTA owns a contiguous run of tiles;
 // otherwise items are dealt round-robin with the token tile varying fastest, so CTAs
 // working on the same rows run together and re-read them from L2.
@@ -32,10 +43,10 @@ namespace {
 
 constexpr int kTcThreads = 320;  // warps 0-3 dequant, 4-7 epilogue, 8 producer, 9 MMA
 constexpr int kPkBytes = 8192;   // packed block of one 128-row tile (128 columns)
+constexpr int kMaxSB = 8;        // deepest B ring
 
 struct TcParams {
-  const __half* Hb;  // blocked FP16 H: [token tile][128-column block][NT x 128 image]
-  const float* t;    // N x RR
+  const __half* Hb;  // B image: [token tile][nkb + nrb blocks][NT x 128]
   const uint8_t* nib;
   const uint8_t* code;  // Vpad x G
   const uint16_t* sup;
@@ -49,6 +60,10 @@ struct TcParams {
   float* tlogit;           // fused NLL: the target's logit per token
   int64_t N, V, D;
   int r_c, r_r, g_shift;
+  int nrb;         // rank blocks after the residual blocks
+  int rank_steps;  // K=16 steps holding rank columns: ceil(4 (r_c + r_r) / 16)
+  int a_words;     // factor rows readable as aligned 32-bit words
+  int sb;          // B ring stages (<= kMaxSB)
   int n_tok_tiles;
   int64_t n_vtiles;
   unsigned* err;
@@ -56,9 +71,8 @@ struct TcParams {
 
 template <int NT>
 struct TcCfg {
-  static constexpr int SB = NT <= 16 ? 8 : (NT <= 32 ? 4 : 3);  // H ring stages
-  static constexpr int SP = NT <= 32 ? 6 : 4;                   // packed ring stages
-  static constexpr int HSTAGE = NT * 256;  // bytes of one 128-column H block
+  static constexpr int SP = NT <= 32 ? 6 : 4;  // packed ring stages
+  static constexpr int HSTAGE = NT * 256;      // bytes of one 128-column B block
   static constexpr int TMEM_COLS = NT <= 64 ? 256 : 512;
   // A-ring stages (64 columns each) in what the two accumulators leave, at most 4
   static constexpr int SA = (TMEM_COLS - 2 * NT) / 64 < 4 ? (TMEM_COLS - 2 * NT) / 64 : 4;
@@ -74,11 +88,11 @@ constexpr size_t nll_scratch_bytes() {
   return (size_t)16 * 128 * 4 + (size_t)NT * 4;
 }
 
-template <int NT, int MODE>
-size_t tc_smem_bytes(int RR, int G) {
+template <int NT>
+size_t tc_smem_bytes(int sb, int G, bool nll) {
   using C = TcCfg<NT>;
-  return (size_t)C::SB * C::HSTAGE + (size_t)C::SP * kPkBytes + 2 * round16((size_t)128 * G) +
-         round16((size_t)RR * NT * 4) + (MODE ? nll_scratch_bytes<NT>() : 0) + 512;
+  return (size_t)sb * C::HSTAGE + (size_t)C::SP * kPkBytes + 2 * round16((size_t)128 * G) +
+         (nll ? nll_scratch_bytes<NT>() : 0) + 512;
 }
 
 // The k-th work item of this CTA: its tile's first row, its row limit, its token tile.
@@ -105,28 +119,91 @@ __device__ __forceinline__ bool get_item(const TcParams& p, int k, Item& it) {
   return true;
 }
 
+// The row scales of vocabulary row v (clamped into range; rows past V only pad a tile).
+struct RowIn {
+  float S, sac, saw;
+};
+__device__ __forceinline__ RowIn load_row(const TcParams& p, int64_t v) {
+  const int64_t vc = v < p.V ? v : p.V - 1;
+  RowIn r;
+  r.S = bf16_bits_to_float(__ldg(p.sup + vc));
+  r.sac = p.r_c ? __ldg(p.sAc + vc) : 0.f;
+  r.saw = p.r_r ? __ldg(p.sAw + vc) : 0.f;
+  return r;
+}
+
+// Accumulator scale S' = S 2^k of a row and the factor 2^-k applied to its group codes
+// (0 when S = 0: the residual row is zero and is dropped).  With M = 128 max(|sAc|, |sAw|)
+// bounding every factor entry, k = ilogb(M) - ilogb(S) - 13 puts M / S' in (2^12, 2^14);
+// k is clamped to [-5, 40] (q c 2^5 <= 65280 stays finite in FP16; q c 2^-k is exact for
+// k <= 24 and below that the residual is under 2^-30 of the factor terms).
+struct RowScale {
+  float sp, cs;
+};
+__device__ __forceinline__ RowScale row_scale(const RowIn& in) {
+  const float M = 128.f * fmaxf(fabsf(in.sac), fabsf(in.saw));
+  RowScale r;
+  if (in.S != 0.f) {
+    int k = 0;
+    if (M > 0.f) {
+      k = ilogbf(M) - ilogbf(in.S) - 13;
+      k = k < -5 ? -5 : (k > 40 ? 40 : k);
+    }
+    r.sp = ldexpf(in.S, k);
+    r.cs = ldexpf(1.f, -k);
+  } else {
+    r.sp = M > 0.f ? ldexpf(1.f, ilogbf(M) - 13) : 1.f;
+    r.cs = 0.f;
+  }
+  return r;
+}
+
+// Four INT8 factor entries j .. j+3 of row v in the concatenation [A_c | A_w] (zeros past
+// r_c + r_r).  With a_words the four never straddle the two factors (r_c % 4 == 0).
+__device__ __forceinline__ uint32_t factor_word(const TcParams& p, int64_t v, int j) {
+  const int RR = p.r_c + p.r_r;
+  if (p.a_words) {
+    if (j < p.r_c) return __ldg(reinterpret_cast<const uint32_t*>(p.Ac + v * p.r_c + j));
+    if (j < RR) return __ldg(reinterpret_cast<const uint32_t*>(p.Aw + v * p.r_r + (j - p.r_c)));
+    return 0u;
+  }
+  uint32_t w = 0;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int jj = j + u;
+    int8_t b = 0;
+    if (jj < p.r_c) b = __ldg(p.Ac + v * p.r_c + jj);
+    else if (jj < RR) b = __ldg(p.Aw + v * p.r_r + (jj - p.r_c));
+    w |= (uint32_t)(uint8_t)b << (8 * u);
+  }
+  return w;
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* ptr) {
+  asm volatile("prefetch.global.L2 [%0];\n" ::"l"(ptr));
+}
+
 template <int NT, int CPC, int DQ, int MODE>
 __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcParams p) {
   using C = TcCfg<NT>;
   extern __shared__ __align__(1024) unsigned char smem[];
-  const int RR = p.r_c + p.r_r;
   const int64_t D = p.D;
   const int nkb = (int)(D / 128);
+  const int nkbt = nkb + p.nrb;  // B blocks per item
   const int G = (int)(D >> p.g_shift);
   const int code_bytes = 128 * G;
+  const int SB = p.sb;
   unsigned char* Hs = smem;
-  unsigned char* pk = Hs + C::SB * C::HSTAGE;
+  unsigned char* pk = Hs + SB * C::HSTAGE;
   unsigned char* cds = pk + C::SP * kPkBytes;  // [2][128 x G]
-  float* ts = reinterpret_cast<float*>(cds + 2 * round16(code_bytes));  // ts[j * NT + n]
-  float* nll_y = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(ts) +
-                                          round16((size_t)RR * NT * 4));  // [16][128]
-  int32_t* tgt_s = reinterpret_cast<int32_t*>(nll_y + 16 * 128);          // [NT]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<unsigned char*>(ts) +
-                                               round16((size_t)RR * NT * 4) +
-                                               (MODE ? nll_scratch_bytes<NT>() : 0));
+  unsigned char* after_codes = cds + 2 * round16(code_bytes);
+  float* nll_y = reinterpret_cast<float*>(after_codes);  // [16][128]
+  int32_t* tgt_s = reinterpret_cast<int32_t*>(nll_y + 16 * 128);  // [NT]
+  uint64_t* bars =
+      reinterpret_cast<uint64_t*>(after_codes + (MODE ? nll_scratch_bytes<NT>() : 0));
   uint64_t* b_full = bars;
-  uint64_t* b_empty = b_full + C::SB;
-  uint64_t* p_full = b_empty + C::SB;
+  uint64_t* b_empty = b_full + kMaxSB;
+  uint64_t* p_full = b_empty + kMaxSB;
   uint64_t* p_empty = p_full + C::SP;
   uint64_t* c_full = p_empty + C::SP;   // [2]
   uint64_t* c_empty = c_full + 2;       // [2]
@@ -140,7 +217,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::SB; ++s) {
+    for (int s = 0; s < SB; ++s) {
       tc::mbar_init(&b_full[s], 1);
       tc::mbar_init(&b_empty[s], 1);
     }
@@ -169,8 +246,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
   const uint32_t acol = tbase + 2 * NT;  // A ring after the two accumulators (lane 0)
 
   if (warp == 8) {
-    // ---------------- producers: lane 0 codes + packed blocks, lane 1 H blocks ----------
-    // Two independent streams, so the packed prefetch is not held back by the H ring
+    // ---------------- producers: lane 0 codes + packed blocks, lane 1 B blocks ----------
+    // Two independent streams, so the packed prefetch is not held back by the B ring
     // (whose stages free up only as MMAs retire).
     if (lane == 0) {
       int k = 0, np = 0, nc = 0;
@@ -212,10 +289,10 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
       Item it;
       for (int i = 0; ok && get_item(p, i, it); ++i) {
         const unsigned char* hsrc =
-            reinterpret_cast<const unsigned char*>(p.Hb) + (int64_t)it.tt * nkb * C::HSTAGE;
-        for (int kb = 0; kb < nkb; ++kb, ++k) {
-          const int sb = k % C::SB;
-          if (k >= C::SB && !tc::mbar_wait(&b_empty[sb], ((k / C::SB) - 1) & 1, p.err)) {
+            reinterpret_cast<const unsigned char*>(p.Hb) + (int64_t)it.tt * nkbt * C::HSTAGE;
+        for (int kb = 0; kb < nkbt; ++kb, ++k) {
+          const int sb = k % SB;
+          if (k >= SB && !tc::mbar_wait(&b_empty[sb], ((k / SB) - 1) & 1, p.err)) {
             ok = false;
             break;
           }
@@ -225,8 +302,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
         }
       }
       if (!ok) {
-        for (int q = nb - C::SB < 0 ? 0 : nb - C::SB; q < nb; ++q)
-          tc::mbar_wait(&b_full[q % C::SB], (q / C::SB) & 1, p.err);
+        for (int q = nb - SB < 0 ? 0 : nb - SB; q < nb; ++q)
+          tc::mbar_wait(&b_full[q % SB], (q / SB) & 1, p.err);
       }
     }
   } else if (warp == 9) {
@@ -241,10 +318,12 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
         if (i >= 2 && !tc::mbar_wait(&acc_empty[ab], ((i >> 1) - 1) & 1, p.err)) break;
         tc::fence_after_sync();
         const uint32_t dcol = tbase + ab * NT;
-        for (int kb = 0; kb < nkb; ++kb, ++k) {
-          const int sa = k % C::SA, sb = k % C::SB;
+        for (int kb = 0; kb < nkbt; ++kb, ++k) {
+          const int sa = k % C::SA, sb = k % SB;
+          // residual blocks: 8 K steps; rank blocks: the steps that hold factor columns
+          const int steps = kb < nkb ? 8 : min(8, p.rank_steps - 8 * (kb - nkb));
           if (!tc::mbar_wait(&a_full[sa], (k / C::SA) & 1, p.err) ||
-              !tc::mbar_wait(&b_full[sb], (k / C::SB) & 1, p.err)) {
+              !tc::mbar_wait(&b_full[sb], (k / SB) & 1, p.err)) {
             ok = false;
             break;
           }
@@ -252,10 +331,12 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
           const uint32_t hb = tc::smem_u32(Hs + sb * C::HSTAGE);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            // K step j: 64-column half j / 4 (NT x 128 bytes each), 32-byte offset j % 4
-            const uint64_t bd =
-                tc::smem_desc_kmajor_sw128(hb + (j >> 2) * NT * 128 + (j & 3) * 32);
-            tc::mma_f16_ts(dcol, acol + 64 * sa + 8 * j, bd, idesc, (kb | j) != 0);
+            if (j < steps) {
+              // K step j: 64-column half j / 4 (NT x 128 bytes each), 32-byte offset j % 4
+              const uint64_t bd =
+                  tc::smem_desc_kmajor_sw128(hb + (j >> 2) * NT * 128 + (j & 3) * 32);
+              tc::mma_f16_ts(dcol, acol + 64 * sa + 8 * j, bd, idesc, (kb | j) != 0);
+            }
           }
           tc::mma_commit(&a_empty[sa]);
           tc::mma_commit(&b_empty[sb]);
@@ -269,10 +350,26 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
     // ---------------- dequant: thread = tile row = TMEM lane ----------------
     const int tid = threadIdx.x;
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
-    int k = 0;
+    int k = 0;   // A-ring sequence: residual and rank blocks
+    int kp = 0;  // packed-ring sequence: residual blocks only
     bool ok = true;
     Item it;
-    for (int i = 0; ok && get_item(p, i, it); ++i) {
+    bool have = get_item(p, 0, it);
+    RowIn rin = {0.f, 0.f, 0.f};
+    if (have) rin = load_row(p, it.row0 + tid);
+    for (int i = 0; ok && have; ++i) {
+      // the next item's row scales load while this one runs
+      Item nx;
+      const bool have_nx = get_item(p, i + 1, nx);
+      RowIn rnx = rin;
+      if (have_nx) rnx = load_row(p, nx.row0 + tid);
+      const int64_t v = it.row0 + tid;
+      const bool live = v < it.row_end;
+      const RowScale rs = row_scale(rin);
+      if (live && p.nrb) {  // the factor rows are read after the residual blocks
+        if (p.r_c) prefetch_l2(p.Ac + v * p.r_c);
+        if (p.r_r) prefetch_l2(p.Aw + v * p.r_r);
+      }
       const int cs = i & 1;
       // warp-uniform outcomes: the tcgen05 stores below are whole-warp instructions
       if (!__all_sync(0xffffffffu, tc::mbar_wait(&c_full[cs], (i >> 1) & 1, p.err))) {
@@ -280,9 +377,9 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
         break;
       }
       const unsigned char* crow = cds + cs * round16(code_bytes) + tid * G;
-      for (int kb = 0; kb < nkb; ++kb, ++k) {
-        const int sp = k % C::SP, sa = k % C::SA;
-        if (!__all_sync(0xffffffffu, tc::mbar_wait(&p_full[sp], (k / C::SP) & 1, p.err))) {
+      for (int kb = 0; kb < nkb; ++kb, ++k, ++kp) {
+        const int sp = kp % C::SP, sa = k % C::SA;
+        if (!__all_sync(0xffffffffu, tc::mbar_wait(&p_full[sp], (kp / C::SP) & 1, p.err))) {
           ok = false;
           break;
         }
@@ -320,7 +417,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
         // window w (32 block columns) = TMEM columns 16w..16w+15: words w, 4+w, 8+w, 12+w
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-          const __half2 c2 = __half2half2(__ushort2half_rn((unsigned short)cw[w]));
+          // c 2^-k is exact in FP16 (8 significant bits, k <= 24)
+          const __half2 c2 = __float2half2_rn((float)cw[w] * rs.cs);
           uint32_t a16[16];
 #pragma unroll
           for (int t4 = 0; t4 < 4; ++t4) {
@@ -341,6 +439,45 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
       }
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&c_empty[cs]);
+      // rank blocks: factor index j = 32 rb + i takes TMEM columns 2i (x1, x1) and
+      // 2i + 1 (x2, x2), x = fl32(A[v, j] s_v) / S' split into FP16 hi and remainder
+      const float rcp = 1.f / rs.sp;
+      for (int rb = 0; ok && rb < p.nrb; ++rb, ++k) {
+        const int sa = k % C::SA;
+        uint32_t fw[8];
+#pragma unroll
+        for (int w = 0; w < 8; ++w) fw[w] = live ? factor_word(p, v, 32 * rb + 4 * w) : 0u;
+        if (k >= C::SA) {
+          if (!__all_sync(0xffffffffu,
+                          tc::mbar_wait(&a_empty[sa], ((k / C::SA) - 1) & 1, p.err))) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+        }
+        const uint32_t ta = acol + 64 * sa + lane_off;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t a16[16];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int j = 32 * rb + 8 * q4 + u;
+            const int8_t e = (int8_t)((fw[2 * q4 + (u >> 2)] >> (8 * (u & 3))) & 0xFFu);
+            const float x = __fmul_rn((float)e, j < p.r_c ? rin.sac : rin.saw) * rcp;
+            const __half x1 = __float2half_rn(x);
+            const __half x2 = __float2half_rn(x - __half2float(x1));
+            a16[2 * u] = h2_bits(__half2half2(x1));
+            a16[2 * u + 1] = h2_bits(__half2half2(x2));
+          }
+          tc::tmem_st16(ta + 16 * q4, a16);
+        }
+        tc::tmem_wait_st();
+        tc::fence_before_sync();
+        tc::mbar_arrive(&a_full[sa]);
+      }
+      it = nx;
+      have = have_nx;
+      rin = rnx;
     }
   } else if (warp < 8) {
     // ---------------- epilogue: thread = accumulator row = TMEM lane ----------------
@@ -350,75 +487,26 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
     Item it;
     for (int i = 0; get_item(p, i, it); ++i) {
       const int ab = i & 1;
-      if (it.tt != cur_tt) {  // stage t of this token tile (transposed: ts[j * NT + n])
+      const int64_t tok0 = (int64_t)it.tt * NT;
+      if (MODE == 1 && it.tt != cur_tt) {  // the token tile's targets
         asm volatile("bar.sync 1, 128;\n" ::: "memory");
-        const int64_t tok0 = (int64_t)it.tt * NT;
-        for (int q = e; q < NT * RR; q += 128) {
-          const int j = q / NT, n = q - j * NT;
-          const int64_t tok = tok0 + n;
-          ts[q] = tok < p.N ? __ldg(p.t + tok * RR + j) : 0.f;
-        }
-        if (MODE == 1)
-          for (int q = e; q < NT; q += 128) tgt_s[q] = tok0 + q < p.N ? __ldg(p.targets + tok0 + q) : -1;
+        for (int q = e; q < NT; q += 128)
+          tgt_s[q] = tok0 + q < p.N ? __ldg(p.targets + tok0 + q) : -1;
         asm volatile("bar.sync 1, 128;\n" ::: "memory");
         cur_tt = it.tt;
       }
+      const int64_t v = it.row0 + e;
+      const bool live = v < it.row_end;
+      const float sp = row_scale(load_row(p, v)).sp;  // loads overlap the wait below
       // one outcome for all four epilogue warps: they share named barriers below
       if (!tc::bar_and(1, 128, tc::mbar_wait(&acc_full[ab], (i >> 1) & 1, p.err))) break;
       tc::fence_after_sync();
-      const int64_t v = it.row0 + e;
-      const bool live = v < it.row_end;
-      const int64_t vc = live ? v : it.row0;
-      const float S = bf16_bits_to_float(__ldg(p.sup + vc));
-      const float sac = p.r_c ? __ldg(p.sAc + vc) : 0.f;
-      const float saw = p.r_r ? __ldg(p.sAw + vc) : 0.f;
-      const int8_t* arow_c = p.Ac + vc * p.r_c;
-      const int8_t* arow_w = p.Aw + vc * p.r_r;
-      const int64_t tok0 = (int64_t)it.tt * NT;
 #pragma unroll 1
       for (int c = 0; c < NT / 16; ++c) {
         float y[16];
         tc::tmem_ld16(tbase + ab * NT + lane_off + 16 * c, y);
 #pragma unroll
-        for (int q = 0; q < 16; ++q) y[q] *= S;
-#pragma unroll 1
-        for (int part = 0; part < 2; ++part) {
-          const int rank = part == 0 ? p.r_c : p.r_r;
-          if (rank == 0) continue;
-          const int8_t* arow = part == 0 ? arow_c : arow_w;
-          const float* tcol = ts + (part == 0 ? 0 : p.r_c) * NT + 16 * c;
-          float lr[16];
-#pragma unroll
-          for (int q = 0; q < 16; ++q) lr[q] = 0.f;
-          auto acc_j = [&](float aj, int j) {
-            const float4* tp = reinterpret_cast<const float4*>(tcol + j * NT);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const float4 tv = tp[q];
-              lr[4 * q + 0] = fmaf(aj, tv.x, lr[4 * q + 0]);
-              lr[4 * q + 1] = fmaf(aj, tv.y, lr[4 * q + 1]);
-              lr[4 * q + 2] = fmaf(aj, tv.z, lr[4 * q + 2]);
-              lr[4 * q + 3] = fmaf(aj, tv.w, lr[4 * q + 3]);
-            }
-          };
-          int j = 0;
-          if ((rank & 3) == 0 && ((reinterpret_cast<uintptr_t>(arow) & 3) == 0)) {
-            // four INT8 factor entries per 32-bit load
-            const uint32_t* aw4 = reinterpret_cast<const uint32_t*>(arow);
-#pragma unroll 2
-            for (; j < rank; j += 4) {
-              const uint32_t wv = __ldg(aw4 + (j >> 2));
-              acc_j((float)(int8_t)(wv & 0xFF), j);
-              acc_j((float)(int8_t)((wv >> 8) & 0xFF), j + 1);
-              acc_j((float)(int8_t)((wv >> 16) & 0xFF), j + 2);
-              acc_j((float)(int8_t)(wv >> 24), j + 3);
-            }
-          }
-          for (; j < rank; ++j) acc_j((float)__ldg(arow + j), j);
-          const float sc = part == 0 ? sac : saw;
-#pragma unroll
-          for (int q = 0; q < 16; ++q) y[q] = fmaf(sc, lr[q], y[q]);
-        }
+        for (int q = 0; q < 16; ++q) y[q] *= sp;
         if (MODE == 0) {
           if (live) {
 #pragma unroll
@@ -474,26 +562,26 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
   }
 }
 
-// FP16 copy of H in the image the MMA's B operand reads: for token tile tt of NT rows and
-// 128-column block kb, a contiguous NT x 128 block made of two 64-column halves; in half h
-// the 16-byte piece (token n, columns 64h + 8c .. +7) sits at h * NT * 128 + n * 128 +
-// (c ^ (n % 8)) * 16 bytes (K-major, 128-byte swizzle).  Rows >= N are zero.  Non-finite
-// or out-of-range FP16 values set kErrRangeH.
+// The B image of the residual blocks: FP16 copy of H, for token tile tt of nt rows and
+// 128-column block kb a contiguous nt x 128 block at tc_image_offset (K-major, 128-byte
+// swizzle).  Rows >= N are zero, and so are the nrb rank blocks after the nkb blocks of H,
+// which the low-rank prologue then fills.  Non-finite or out-of-range FP16 values set
+// kErrRangeH.
 __global__ void __launch_bounds__(256) convert_h_blocked_kernel(const uint16_t* __restrict__ H,
                                                                 __half* __restrict__ Hb,
                                                                 int64_t N, int64_t Npad,
-                                                                int64_t D, int nt,
+                                                                int64_t D, int64_t nkbt, int nt,
                                                                 unsigned* err) {
-  const int64_t chunks_per_row = D / 8;
+  const int64_t chunks_per_row = nkbt * 16;  // 8 FP16 per chunk
   const int64_t total = Npad * chunks_per_row;
-  const int64_t nkb = D / 128;
+  const int64_t hchunks = D / 8;
   bool bad = false;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
        i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t n = i / chunks_per_row;
     const int64_t kc = i - n * chunks_per_row;
     uint4 out = make_uint4(0, 0, 0, 0);
-    if (n < N) {
+    if (n < N && kc < hchunks) {
       const uint4 in = *reinterpret_cast<const uint4*>(H + n * D + kc * 8);
       const uint32_t w[4] = {in.x, in.y, in.z, in.w};
       uint32_t o[4];
@@ -507,18 +595,29 @@ __global__ void __launch_bounds__(256) convert_h_blocked_kernel(const uint16_t* 
       out = make_uint4(o[0], o[1], o[2], o[3]);
     }
     const int64_t tt = n / nt, nn = n - tt * nt;
-    const int64_t kb = kc >> 4, half = (kc >> 3) & 1, c = kc & 7;
-    const int64_t off = (tt * nkb + kb) * (int64_t)nt * 128 + half * (int64_t)nt * 64 + nn * 64 +
-                        ((c ^ (nn & 7)) * 8);
-    *reinterpret_cast<uint4*>(Hb + off) = out;
+    *reinterpret_cast<uint4*>(Hb + tc_image_offset(tt, kc >> 4, nkbt, nt, nn,
+                                                   (int)(kc & 15) * 8)) = out;
   }
   if (bad) atomicOr(err, kErrRangeH);
 }
 
+// Resident CTAs per SM of a kernel: registers (allocated per warp in units of 256), shared
+// memory (plus the 1 KB the driver reserves per CTA), warps and tensor-memory columns.
+int tc_residency(const cudaFuncAttributes& fa, size_t smem, int tmem_cols, int regs_sm,
+                 int smem_sm) {
+  const int warps = kTcThreads / 32;
+  const int regs_warp = (fa.numRegs * 32 + 255) / 256 * 256;
+  int occ = regs_sm / (regs_warp * warps);
+  const int by_smem = smem_sm / (int)(smem + fa.sharedSizeBytes + 1024);
+  if (by_smem < occ) occ = by_smem;
+  if (64 / warps < occ) occ = 64 / warps;
+  if (512 / tmem_cols < occ) occ = 512 / tmem_cols;
+  return occ;
+}
+
 template <int NT, int CPC, int DQ, int MODE>
 cudaError_t launch_tc_cfg(const TcParams& p, cudaStream_t st) {
-  const int RR = p.r_c + p.r_r;
-  const size_t smem = tc_smem_bytes<NT, MODE>(RR, (int)(p.D >> p.g_shift));
+  const size_t smem = tc_smem_bytes<NT>(p.sb, (int)(p.D >> p.g_shift), MODE == 1);
   auto kern = residual_tc_kernel<NT, CPC, DQ, MODE>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -533,15 +632,7 @@ cudaError_t launch_tc_cfg(const TcParams& p, cudaStream_t st) {
     return e;
   cudaFuncAttributes fa;
   if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
-  // resident CTAs per SM: registers (allocated per warp in units of 256), shared memory
-  // (plus the 1 KB the driver reserves per CTA), warps, and tensor-memory columns
-  const int warps = kTcThreads / 32;
-  const int regs_warp = (fa.numRegs * 32 + 255) / 256 * 256;
-  int occ = regs_sm / (regs_warp * warps);
-  const int by_smem = smem_sm / (int)(smem + fa.sharedSizeBytes + 1024);
-  if (by_smem < occ) occ = by_smem;
-  if (64 / warps < occ) occ = 64 / warps;
-  if (512 / TcCfg<NT>::TMEM_COLS < occ) occ = 512 / TcCfg<NT>::TMEM_COLS;
+  int occ = tc_residency(fa, smem, TcCfg<NT>::TMEM_COLS, regs_sm, smem_sm);
   if (occ < 1) occ = 1;
   int64_t items = p.n_vtiles * p.n_tok_tiles;
   int64_t grid = (int64_t)sms * occ;
@@ -567,35 +658,64 @@ cudaError_t launch_tc_mode(const TcParams& p, int nt, int g, cudaStream_t st) {
   }
 }
 
+// Deepest B ring (2 .. max_sb stages) whose shared memory fits the budget, or 0.
+template <int NT>
+int fit_sb(int max_sb, int G, bool nll, size_t budget) {
+  for (int sb = max_sb; sb >= 2; --sb)
+    if (tc_smem_bytes<NT>(sb, G, nll) <= budget) return sb;
+  return 0;
+}
+
 }  // namespace
 
-int tc_token_tile(int64_t N, int RR) {
-  if (N <= 16) return 16;
-  if (N <= 32) return 32;
-  if (N <= 64 || RR > 128) return 64;
-  return 128;
+TcPlan tc_plan(const Shapes& s, bool nll) {
+  // Shared memory per SM is 228 KB with 1 KB reserved per CTA; a CTA may take 227 KB.
+  // Token tiles up to 64 use 256 TMEM columns and keep two CTAs per SM within budget.
+  const size_t two_per_sm = 228 * 1024 / 2 - 1024, one_per_sm = 227 * 1024;
+  const int G = (int)(s.D / s.g);
+  TcPlan pl = {0, 0, (s.r_c + s.r_r + 31) / 32};
+  if (s.N > 64) {
+    if ((pl.sb = fit_sb<128>(4, G, nll, one_per_sm))) pl.nt = 128;
+  }
+  if (!pl.nt) {
+    const int nt = s.N <= 16 ? 16 : (s.N <= 32 ? 32 : 64);
+    const int max_sb = nt == 16 ? 8 : (nt == 32 ? 6 : 4);
+    int sb = 0;
+    switch (nt) {
+      case 16: sb = fit_sb<16>(max_sb, G, nll, two_per_sm); break;
+      case 32: sb = fit_sb<32>(max_sb, G, nll, two_per_sm); break;
+      default: sb = fit_sb<64>(max_sb, G, nll, two_per_sm); break;
+    }
+    if (sb) {
+      pl.nt = nt;
+      pl.sb = sb;
+    }
+  }
+  return pl;
 }
 
 cudaError_t launch_prologue_blocked(const uint16_t* H, const archead_head* head,
-                                    const Shapes& s, int nt, __half* Hb, float* t,
+                                    const Shapes& s, const TcPlan& plan, __half* Hb,
                                     unsigned* err, cudaStream_t st, int* launches) {
+  const int nt = plan.nt;
   const int64_t Npad = (s.N + nt - 1) / nt * nt;
-  int64_t blocks = (Npad * s.D / 8 + 255) / 256;
+  const int64_t nkbt = s.D / 128 + plan.nrb;
+  int64_t blocks = (Npad * nkbt * 16 + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
   convert_h_blocked_kernel<<<(unsigned)(blocks < 1 ? 1 : blocks), 256, 0, st>>>(
-      H, Hb, s.N, Npad, s.D, nt, err);
+      H, Hb, s.N, Npad, s.D, nkbt, nt, err);
   ++*launches;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_lowrank_t(H, head, s, t, st, launches);
+  return launch_lowrank_t(H, head, s, nullptr, Hb, nt, nkbt, err, st, launches);
 }
 
-cudaError_t launch_residual_tc(const __half* Hb, const float* t, const archead_head* head,
-                               const Shapes& s, float* Y, const int32_t* targets, float2* part,
-                               float* tlogit, unsigned* err, cudaStream_t st, int* launches) {
+cudaError_t launch_residual_tc(const __half* Hb, const archead_head* head, const Shapes& s,
+                               const TcPlan& plan, float* Y, const int32_t* targets,
+                               float2* part, float* tlogit, unsigned* err, cudaStream_t st,
+                               int* launches) {
   TcParams p;
   p.Hb = Hb;
-  p.t = t;
   p.nib = head->r_nib;
   p.code = head->r_code;
   p.sup = head->r_super;
@@ -615,11 +735,17 @@ cudaError_t launch_residual_tc(const __half* Hb, const float* t, const archead_h
   int gs = 0;
   while ((1 << gs) < s.g) ++gs;
   p.g_shift = gs;
+  p.nrb = plan.nrb;
+  p.rank_steps = (4 * (s.r_c + s.r_r) + 15) / 16;
+  // factor rows as aligned words: both ranks multiples of 4 (bases are 16-byte aligned)
+  p.a_words = (s.r_c % 4 == 0 && s.r_r % 4 == 0) ? 1 : 0;
+  p.sb = plan.sb;
   p.err = err;
-  const int nt = tc_token_tile(s.N, s.r_c + s.r_r);
-  p.n_tok_tiles = (int)((s.N + nt - 1) / nt);
+  p.n_tok_tiles = (int)((s.N + plan.nt - 1) / plan.nt);
   p.n_vtiles = (s.V + 127) / 128;
-  cudaError_t e = Y ? launch_tc_mode<0>(p, nt, s.g, st) : launch_tc_mode<1>(p, nt, s.g, st);
+  if (plan.nt == 0 || plan.sb < 2 || plan.sb > kMaxSB) return cudaErrorInvalidValue;
+  cudaError_t e = Y ? launch_tc_mode<0>(p, plan.nt, s.g, st)
+                    : launch_tc_mode<1>(p, plan.nt, s.g, st);
   ++*launches;
   return e;
 }

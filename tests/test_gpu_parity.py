@@ -97,6 +97,22 @@ def test_logits_shapes_groups_ranks(dev, g, r_c, r_r, V, D):
         _assert_logits(Y.cpu().numpy(), oracle.logits(head, bf16_bits(H)), f"{g} {N}")
 
 
+@pytest.mark.parametrize("sup_exp,fac_exp", [((-40, -30), (-5, -3)), ((-4, -2), (-30, -25)),
+                                             ((-20, -20), (-9, -9))])
+def test_logits_extreme_scale_ratios(dev, sup_exp, fac_exp):
+    """Factor scales far above the residual super-scale (the per-row accumulator exponent
+    at its upper clamp, the residual below FP16 resolution there), far below it (lower
+    clamp, factor pieces subnormal in FP16), and one fixed ratio, on both paths."""
+    head = random_canonical_head(515, 512, 12, 20, 64, seed=77, zero_rows=5,
+                                 super_exp_range=sup_exp, factor_exp_range=fac_exp)
+    dh = ah.DeviceHead.from_canonical(head, dev)
+    for N in (3, 40, 130):
+        H = _rand_H(N, 512, 500 + N)
+        Y = ah.logits(H.to(dev), dh)
+        ah.check()
+        _assert_logits(Y.cpu().numpy(), oracle.logits(head, bf16_bits(H)), f"{sup_exp} {N}")
+
+
 @pytest.fixture(scope="module")
 def nhead(dev):
     """Random packed bytes scaled so that rms(Y) is a few units, the regime of language-model
