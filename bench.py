@@ -39,7 +39,11 @@ from workloads import (WORKLOADS, bf16_bits, make_channel_scales, make_hidden,  
 L2_BYTES = 126 * 2 ** 20
 METRIC = "packed LM-head tokens/s; decode HBM GB/s and prefill TFLOP/s vs B200 roofline"
 MAIN_KERNEL_SRC = ["packed_int4_lm_b200/csrc/residual_mma.cu",
+                   "packed_int4_lm_b200/csrc/residual_tc.cu",
+                   "packed_int4_lm_b200/csrc/tc_common.cuh",
                    "packed_int4_lm_b200/csrc/archead_internal.cuh"]
+# token counts up to this go to the warp-MMA kernel, larger ones to the tcgen05 kernel
+WARP_MMA_MAX_N = 8
 
 
 def parse():
@@ -51,6 +55,9 @@ def parse():
     ap.add_argument("--workload", default="qwen_decode", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--ns", default=None,
+                    help="comma-separated token counts replacing the workload's (profiling "
+                         "a smaller case of the same head)")
     return ap.parse_args()
 
 
@@ -202,7 +209,7 @@ def main():
     K, Wm = DEFAULT_STEPS[a.workload]
     K = a.steps if a.steps is not None else K
     Wm = a.warmup if a.warmup is not None else Wm
-    Ns = list(w.Ns)
+    Ns = [int(x) for x in a.ns.split(",")] if a.ns else list(w.Ns)
     nll_mode = w.nll
     cfg = {"workload": f"{w.name}: V={w.V} D={w.D} N={','.join(map(str, Ns))} "
                        f"r_c={w.r_c} r_r={w.r_r} g={w.g} p={w.p} lam={w.lam}"
@@ -316,7 +323,9 @@ def main():
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_sustained"],
                 "unit": "TFLOP/s", "frac": achieved / peaks["bf16_sustained"]}
     roof["peak_source"] = peaks["source"]
-    roof["kernel"] = "residual_mma_kernel"
+    roof["kernel"] = ", ".join(
+        (["residual_mma_kernel (N<=%d)" % WARP_MMA_MAX_N] if min(Ns) <= WARP_MMA_MAX_N else [])
+        + (["residual_tc_kernel (N>%d)" % WARP_MMA_MAX_N] if max(Ns) > WARP_MMA_MAX_N else []))
     roof["traffic"] = profiled_traffic(w.name, Ns)
     roof["main_kernel_share"] = main_ms / max(elapsed_ms, 1e-9)
 
