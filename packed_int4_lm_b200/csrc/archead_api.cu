@@ -111,6 +111,46 @@ struct Carve {
   }
 };
 
+int run_dec(const uint16_t* H, const archead_head* head, float* Y, const int32_t* targets,
+            float* nll, const Shapes& s, const DecPlan& pl, DeviceState* ds, cudaStream_t st) {
+  int launches = 0;
+  const int RR = s.r_c + s.r_r;
+  const bool nll_mode = nll != nullptr;
+  const int64_t nvt = (s.V + 127) / 128;
+  Carve cv;
+  const size_t o_img = cv.take(dec_image_bytes(s, pl));
+  const size_t o_t = cv.take((size_t)s.N * RR * 4);
+  const size_t o_cnt = cv.take((size_t)nvt * 4);
+  const size_t o_scr = cv.take(dec_partial_bytes(pl));
+  const size_t o_part = nll_mode ? cv.take((size_t)s.N * nvt * 8) : 0;
+  const size_t o_tl = nll_mode ? cv.take((size_t)s.N * 4) : 0;
+  void* base = nullptr;
+  if (cudaMallocFromPoolAsync(&base, cv.off, ds->pool, st) != cudaSuccess) {
+    cudaGetLastError();
+    return ARCHEAD_ERR_NOMEM;
+  }
+  char* b = static_cast<char*>(base);
+  __half* img = reinterpret_cast<__half*>(b + o_img);
+  float* t = reinterpret_cast<float*>(b + o_t);
+  unsigned* cnt = reinterpret_cast<unsigned*>(b + o_cnt);
+  float4* scr = reinterpret_cast<float4*>(b + o_scr);
+  float2* part = nll_mode ? reinterpret_cast<float2*>(b + o_part) : nullptr;
+  float* tl = nll_mode ? reinterpret_cast<float*>(b + o_tl) : nullptr;
+  cudaError_t e = launch_dec_prologue(H, head, s, pl, img, t, cnt, ds->err, st, &launches);
+  if (e == cudaSuccess) {
+    prof_mark(0, st);
+    e = launch_residual_dec(img, t, head, s, pl, nll_mode ? nullptr : Y, targets, part, tl, scr,
+                            cnt, ds->err, st, &launches);
+    prof_mark(1, st);
+    if (e == cudaSuccess && nll_mode)
+      e = launch_nll_combine(part, tl, targets, s, nll, ds->err, st, &launches);
+  }
+  cudaFreeAsync(base, st);
+  if (e != cudaSuccess) return ARCHEAD_ERR_CUDA;
+  t_last_launches = launches;
+  return ARCHEAD_OK;
+}
+
 int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* targets,
         float* nll, const Shapes& s, cudaStream_t st) {
   DeviceState* ds;
@@ -122,6 +162,9 @@ int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* ta
   // N <= 8 on the warp-MMA kernel (one token block), larger N on the tensor-memory
   // (tcgen05) kernel when its shared-memory rings fit the shape; both have a fused
   // split-vocabulary NLL epilogue
+  // N <= 16: the persistent decode kernel with H resident in shared memory, when it fits
+  const DecPlan dplan = dec_plan(s, nll_mode);
+  if (dplan.nt8 > 0) return run_dec(H, head, Y, targets, nll, s, dplan, ds, st);
   const TcPlan plan = s.N > 8 ? tc_plan(s, nll_mode) : TcPlan{0, 0, 0};
   const bool use_tc = plan.nt > 0;
   const int64_t tb = use_tc ? plan.nt : residual_token_block(s.N);

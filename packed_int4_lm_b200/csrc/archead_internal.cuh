@@ -79,6 +79,24 @@ __device__ __forceinline__ void dequant_word_lite(uint32_t w, __half2 c2, __half
   out[3] = __hmul2(__hfma2(*reinterpret_cast<__half2*>(&x3), k16, k72), c2);
 }
 
+// Exact FP16 q of the eight nibbles of one device-layout word, without a group scale
+// (for kernels that apply the scale to FP32 partial sums): the magic-number reads of
+// dequant_word_lite minus their offsets.
+__device__ __forceinline__ void dequant_word_q(uint32_t w, __half2 out[4]) {
+  const uint32_t w2 = w >> 8;
+  uint32_t x0 = and_xor(w, 0x000F000Fu, 0x64086408u);
+  uint32_t x1 = and_xor(w, 0x00F000F0u, 0x64806480u);
+  uint32_t x2 = and_xor(w2, 0x000F000Fu, 0x64086408u);
+  uint32_t x3 = and_xor(w2, 0x00F000F0u, 0x64806480u);
+  const __half2 k1032 = __float2half2_rn(1032.f);
+  const __half2 k16 = __float2half2_rn(0.0625f);
+  const __half2 k72 = __float2half2_rn(-72.f);
+  out[0] = __hsub2(*reinterpret_cast<__half2*>(&x0), k1032);
+  out[1] = __hfma2(*reinterpret_cast<__half2*>(&x1), k16, k72);
+  out[2] = __hsub2(*reinterpret_cast<__half2*>(&x2), k1032);
+  out[3] = __hfma2(*reinterpret_cast<__half2*>(&x3), k16, k72);
+}
+
 // Device nibble layout, tiled: rows are padded to a multiple of 128 and every 128-row
 // tile's 128-column block (64 bytes per row) is one contiguous 8 KB region, so each tile
 // streams sequentially from HBM.  Inside the region, 16-byte chunk i (i = 0..3) of row s
@@ -179,6 +197,27 @@ cudaError_t launch_residual_tc(const __half* Hb, const archead_head* head, const
                                const TcPlan& plan, float* Y, const int32_t* targets,
                                float2* part, float* tlogit, unsigned* err, cudaStream_t st,
                                int* launches);
+
+// Decode path (N <= 16): persistent bulk-copy-fed warp-MMA kernel with H resident in
+// shared memory.  nt8 = 0 when the shape does not fit (then the token-block kernel runs).
+struct DecPlan {
+  int nt8;   // 8-token MMA column tiles: 1 (N <= 8) or 2 (N <= 16)
+  int sp;    // packed ring stages
+  int grid;  // CTAs (one per SM)
+};
+DecPlan dec_plan(const Shapes& s, bool nll);
+size_t dec_image_bytes(const Shapes& s, const DecPlan& pl);  // resident H image
+size_t dec_partial_bytes(const DecPlan& pl);                 // split-tile partials
+// H image + zeroed per-tile counters (ceil(V/128) words), then t (N x RR FP32).
+cudaError_t launch_dec_prologue(const uint16_t* H, const archead_head* head, const Shapes& s,
+                                const DecPlan& pl, __half* img, float* t, unsigned* counters,
+                                unsigned* err, cudaStream_t st, int* launches);
+// Y != nullptr: logits; else fused-NLL partials as in launch_residual_gemm mode 1.
+cudaError_t launch_residual_dec(const __half* img, const float* t, const archead_head* head,
+                                const Shapes& s, const DecPlan& pl, float* Y,
+                                const int32_t* targets, float2* part, float* tlogit,
+                                float4* scratch, unsigned* counters, unsigned* err,
+                                cudaStream_t st, int* launches);
 
 // Residual dequant-contraction over token blocks of up to 64 (mma.sync path).
 // mode 0: write logits Y.  mode 1: write NLL partials (max, sum exp) per (token, vocabulary

@@ -1,0 +1,722 @@
+// Small-batch (decode) logits: the memory-bound regime of the ARCHead logit formula
+//
+//   Y[n, v] = S_v sum_d h[n, d] q[v, d] c[v, d / g]                 (SC4 residual, Sec. 3)
+//           + sAc[v] sum_j Ac[v, j] t[n, j] + sAw[v] sum_j Aw[v, j] t[n, r_c + j]
+//
+// for N <= 16 tokens, where every packed byte is used by at most 16 tokens and the kernel
+// has to stream the head at HBM speed.  Design:
+//  * persistent grid, one CTA per SM: warp 8 is a producer that bulk-copies (TMA engine,
+//    no tensor map, no multicast) the 8 KB packed blocks of 128-row tiles into a deep
+//    shared-memory ring, plus each tile's group codes and INT8 factor rows; warps 0-7
+//    each own 16 rows of the tile;
+//  * the FP16 hidden states of all (<= 16) tokens stay resident in shared memory for the
+//    whole launch, stored with a chunk swizzle that makes the B-fragment reads
+//    conflict-free;
+//  * A fragments come from the ring with ldmatrix: in the tiled device layout the 16-byte
+//    chunk i of 8 consecutive rows is 128 contiguous bytes, so each 8x8 matrix load is
+//    conflict-free, and thread (g, q) receives word q of chunk i of row g -- exactly the
+//    eight columns it dequantises (exact FP16 q*c) into an m16n8k16 fragment;
+//  * the work is split evenly over CTAs in units of (tile, 128-column block), so all CTAs
+//    finish together.  A tile split between CTAs is finished by the CTA that arrives
+//    last (an atomic counter per tile, no waiting): it sums the partial accumulators of
+//    all contributors in CTA order, so the result does not depend on arrival order;
+//  * epilogue: S_v times the accumulator plus the rank terms in FP32 from t; MODE 1
+//    writes split-vocabulary (max, sum exp) partials and target logits instead of Y.
+// Every mbarrier wait is bounded; a wait that gives up sets the device error word and the
+// warp skips its remaining waits, so the launch always ends.
+#include "tc_common.cuh"
+
+namespace archead {
+namespace {
+
+constexpr int kDecConsumers = 8;                        // consumer warps (16 rows each)
+constexpr int kDecThreads = (kDecConsumers + 1) * 32;   // + producer warp
+constexpr int kDecPk = 8192;                            // packed block of one tile
+
+struct DecParams {
+  const __half* Himg;  // NTOK x D FP16, chunk-swizzled rows (dec_h_offset)
+  const float* t;      // N x RR
+  const uint8_t* nib;
+  const uint8_t* code;  // Vpad x G
+  const uint16_t* sup;
+  const int8_t* Ac;
+  const float* sAc;
+  const int8_t* Aw;
+  const float* sAw;
+  float* Y;
+  const int32_t* targets;
+  float2* part;
+  float* tlogit;
+  float4* scratch;     // partial accumulators: [CTA][2 slots][256 threads][NT8]
+  unsigned* counters;  // arrivals per tile (zeroed by the prologue)
+  int64_t N, V, D;
+  int r_c, r_r, g_shift;
+  int sp;  // packed ring stages
+  int64_t n_vtiles;
+  unsigned* err;
+};
+
+// FP16 element offset of (token n, column d) in the resident H image: rows of D
+// elements; the 16-byte chunk q = d / 8 is stored at q ^ 2 [bit 3 of q] ^ [n odd], which
+// spreads the eight 16-byte reads of each quarter warp over distinct bank groups.
+__host__ __device__ __forceinline__ int64_t dec_h_offset(int64_t n, int64_t d, int64_t D) {
+  const int64_t q = d >> 3;
+  const int64_t pq = q ^ (((q >> 3) & 1) << 1) ^ (n & 1);
+  return n * D + pq * 8 + (d & 7);
+}
+
+template <int NT8>
+struct DecCfg {
+  static constexpr int NTOK = 8 * NT8;
+};
+
+__host__ __device__ inline size_t dec_round16(size_t x) { return (x + 15) & ~(size_t)15; }
+
+struct DecSmem {
+  size_t h, pk, codes, arow_c, arow_w, ts, red, bars, total;
+};
+
+// Shared-memory carve-up (offsets from a 128-byte aligned base).
+template <int NT8, int MODE>
+__host__ __device__ inline DecSmem dec_smem(int64_t D, int G, int r_c, int r_r, int sp) {
+  constexpr int NTOK = DecCfg<NT8>::NTOK;
+  DecSmem m;
+  size_t o = 0;
+  m.h = o;  // H image [NTOK x D] FP16, then corr [D / 128][NTOK] FP32
+  o += dec_round16((size_t)NTOK * D * 2 + (size_t)(D / 128) * NTOK * 4);
+  m.pk = o;  // ring of sp stages of two packed blocks
+  o += (size_t)sp * 2 * kDecPk;
+  m.codes = o;  // [2][128 x G]
+  o += 2 * dec_round16((size_t)128 * G);
+  m.arow_c = o;  // [2][128 x r_c]
+  o += 2 * dec_round16((size_t)128 * r_c);
+  m.arow_w = o;  // [2][128 x r_r]
+  o += 2 * dec_round16((size_t)128 * r_r);
+  m.ts = o;  // [NTOK][RR + 1] FP32
+  o += dec_round16((size_t)NTOK * (r_c + r_r + 1) * 4);
+  m.red = o;  // MODE 1: [8 warps][NTOK] float2
+  o += MODE ? dec_round16((size_t)kDecConsumers * NTOK * 8) : 0;
+  m.bars = o;
+  o += 256;
+  m.total = o;
+  return m;
+}
+
+// The CTA whose unit range holds unit u, for U units split over C CTAs as
+// [U c / C, U (c + 1) / C).
+__device__ __forceinline__ int64_t dec_cta_of(int64_t u, int64_t U, int64_t C) {
+  return ((u + 1) * C + U - 1) / U - 1;
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t saddr, uint32_t r[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(saddr)
+               : "memory");
+}
+
+// Bounded wait that is skipped once this warp has already given up.
+__device__ __forceinline__ bool dec_wait(uint64_t* bar, uint32_t parity, unsigned* err,
+                                         bool ok) {
+  if (!ok) return false;
+  return __all_sync(0xffffffffu, tc::mbar_wait(bar, parity, err));
+}
+
+// Prologue of this path: the resident H image (zero rows up to NTOK), followed by the
+// offset corrections corr[kb][n], and zeroed tile counters.  One warp per (token, block);
+// lane l converts columns 4l .. 4l + 3 of the block.
+//
+// With scale_b (one group code per 128-column block), the kernel feeds the MMA the raw
+// magic-number reads of the nibbles: 1032 + q for columns with (d & 2) == 0 and
+// 1152 + 16 q for the others, whose H values are stored divided by 16 (exact: a power of
+// two).  Each k-block sum then carries the constant 1032 sum_A b + 1152 sum_B b over the
+// stored values b, which corr holds and the kernel subtracts before scaling by the code.
+// Non-finite or out-of-range FP16 values set kErrRangeH.
+__global__ void __launch_bounds__(256) dec_convert_h_kernel(const uint16_t* __restrict__ H,
+                                                            __half* __restrict__ img,
+                                                            int64_t N, int ntok, int64_t D,
+                                                            int scale_b,
+                                                            unsigned* __restrict__ counters,
+                                                            int64_t n_counters,
+                                                            unsigned* err) {
+  const int64_t nkb = D / 128;
+  const int lane = threadIdx.x & 31;
+  const int64_t gw = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  float* corr = reinterpret_cast<float*>(img + (int64_t)ntok * D);  // [nkb][ntok]
+  bool bad = false;
+  for (int64_t wi = gw; wi < (int64_t)ntok * nkb; wi += nw) {
+    const int64_t n = wi / nkb, kb = wi - n * nkb;
+    const int64_t d = kb * 128 + 4 * lane;
+    float f[4] = {0.f, 0.f, 0.f, 0.f};
+    if (n < N) {
+      const uint2 in = *reinterpret_cast<const uint2*>(H + n * D + d);
+      f[0] = __uint_as_float(in.x << 16);
+      f[1] = __uint_as_float(in.x & 0xFFFF0000u);
+      f[2] = __uint_as_float(in.y << 16);
+      f[3] = __uint_as_float(in.y & 0xFFFF0000u);
+    }
+    float sum = 0.f;
+    __half hv[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const bool typeb = ((d + e) & 2) != 0;
+      hv[e] = __float2half_rn(scale_b && typeb ? f[e] * 0.0625f : f[e]);
+      const float b = __half2float(hv[e]);
+      bad |= !(fabsf(b) <= 65504.f);
+      sum += (typeb ? 1152.f : 1032.f) * b;
+    }
+    const uint32_t lo = (uint32_t)__half_as_ushort(hv[0]) | ((uint32_t)__half_as_ushort(hv[1]) << 16);
+    const uint32_t hi = (uint32_t)__half_as_ushort(hv[2]) | ((uint32_t)__half_as_ushort(hv[3]) << 16);
+    *reinterpret_cast<uint2*>(img + dec_h_offset(n, d, D)) = make_uint2(lo, hi);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane == 0) corr[kb * ntok + n] = scale_b ? sum : 0.f;
+  }
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n_counters;
+       i += (int64_t)gridDim.x * blockDim.x)
+    counters[i] = 0u;
+  if (bad) atomicOr(err, kErrRangeH);
+}
+
+constexpr int kDecMaxSP = 8;
+
+// Whether the producer copies the tile's INT8 factor rows into shared memory (each bulk
+// copy must be a multiple of 16 bytes; a ragged last tile may read them from global).
+__host__ __device__ __forceinline__ bool dec_arow_copy(int64_t rows, int r_c, int r_r) {
+  return ((rows * r_c) % 16) == 0 && ((rows * r_r) % 16) == 0;
+}
+
+// m16n8k16 FP16 MMA with a zero accumulator input: d = a * b.
+__device__ __forceinline__ void mma_f16_16816_z(float d[4], const uint32_t a[4], uint32_t b0,
+                                                uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%10, %10, %10, %10};\n"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
+}
+
+// Raw magic-number reads of the eight nibbles of a device-layout word (no FP16 math):
+// pairs 0 and 2 read 1032 + q, pairs 1 and 3 read 1152 + 16 q (see dec_convert_h_kernel).
+__device__ __forceinline__ void nibble_reads(uint32_t w, uint32_t x[4]) {
+  const uint32_t w2 = w >> 8;
+  x[0] = and_xor(w, 0x000F000Fu, 0x64086408u);
+  x[1] = and_xor(w, 0x00F000F0u, 0x64806480u);
+  x[2] = and_xor(w2, 0x000F000Fu, 0x64086408u);
+  x[3] = and_xor(w2, 0x00F000F0u, 0x64806480u);
+}
+
+template <int NT8, int CPC, int MODE>
+__global__ void __launch_bounds__(kDecThreads, 1) residual_dec_kernel(const DecParams p) {
+  constexpr int NTOK = DecCfg<NT8>::NTOK;
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int64_t D = p.D;
+  const int nkb = (int)(D / 128);
+  const int G = (int)(D >> p.g_shift);
+  const int RR = p.r_c + p.r_r;
+  const int SP = p.sp;
+  const DecSmem m = dec_smem<NT8, MODE>(D, G, p.r_c, p.r_r, SP);
+  const unsigned char* Hb = smem + m.h;
+  const float* corr = reinterpret_cast<const float*>(smem + m.h + (size_t)NTOK * D * 2);
+  unsigned char* pk = smem + m.pk;
+  unsigned char* cds = smem + m.codes;
+  int8_t* arc = reinterpret_cast<int8_t*>(smem + m.arow_c);
+  int8_t* arw = reinterpret_cast<int8_t*>(smem + m.arow_w);
+  float* ts = reinterpret_cast<float*>(smem + m.ts);  // ts[j * NTOK + n]
+  float2* red = reinterpret_cast<float2*>(smem + m.red);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + m.bars);
+  uint64_t* h_full = bars;       // [1]
+  uint64_t* c_full = bars + 1;   // [2]
+  uint64_t* c_empty = bars + 3;  // [2]
+  uint64_t* p_full = bars + 5;   // [SP]
+  uint64_t* p_empty = p_full + SP;
+  int* flag = reinterpret_cast<int*>(p_empty + SP);
+  const int code_bytes = 128 * G;
+  const size_t code_slot = dec_round16((size_t)code_bytes);
+  const size_t arc_slot = dec_round16((size_t)128 * p.r_c);
+  const size_t arw_slot = dec_round16((size_t)128 * p.r_r);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // this CTA's units (tile, 128-column block), tile-major: [u0, u1)
+  const int64_t U = p.n_vtiles * nkb, C = gridDim.x;
+  const int64_t u0 = U * blockIdx.x / C, u1 = U * (blockIdx.x + 1) / C;
+
+  if (threadIdx.x == 0) {
+    tc::mbar_init(h_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&c_full[s], 1);
+      tc::mbar_init(&c_empty[s], kDecConsumers);
+    }
+    for (int s = 0; s < SP; ++s) {
+      tc::mbar_init(&p_full[s], 1);
+      tc::mbar_init(&p_empty[s], kDecConsumers);
+    }
+    tc::mbar_fence_init();
+  }
+  __syncthreads();
+
+  if (warp == kDecConsumers) {
+    // ---------------- producer (one thread) ----------------
+    // A stage holds up to two consecutive blocks of one tile (contiguous in the device
+    // layout, so one bulk copy).
+    if (lane == 0) {
+      bool ok = true;
+      const uint32_t hbytes = (uint32_t)(NTOK * D * 2 + (int64_t)nkb * NTOK * 4);
+      tc::mbar_arrive_expect_tx(h_full, hbytes);
+      tc::bulk_g2s(smem + m.h, p.Himg, hbytes, h_full);
+      int k = 0, np = 0, nc = 0, s = 0;
+      for (int64_t u = u0; ok && u < u1; ++s) {
+        const int64_t T = u / nkb;
+        const int kb0 = (int)(u - T * nkb);
+        const int kb1 = (int)((int64_t)nkb < kb0 + (u1 - u) ? (int64_t)nkb : kb0 + (u1 - u));
+        const int cs = s & 1;
+        if (s >= 2 && !tc::mbar_wait(&c_empty[cs], ((s >> 1) - 1) & 1, p.err)) {
+          ok = false;
+          break;
+        }
+        tc::fence_proxy_async_smem();  // the slot was read with generic loads
+        const int64_t row0 = T * 128;
+        const int64_t rows = p.V - row0 < 128 ? p.V - row0 : 128;
+        const bool acopy = dec_arow_copy(rows, p.r_c, p.r_r);
+        const uint32_t abytes_c = acopy ? (uint32_t)(rows * p.r_c) : 0u;
+        const uint32_t abytes_w = acopy ? (uint32_t)(rows * p.r_r) : 0u;
+        tc::mbar_arrive_expect_tx(&c_full[cs], (uint32_t)code_bytes + abytes_c + abytes_w);
+        tc::bulk_g2s(cds + cs * code_slot, p.code + row0 * G, (uint32_t)code_bytes, &c_full[cs]);
+        if (abytes_c) tc::bulk_g2s(arc + cs * arc_slot, p.Ac + row0 * p.r_c, abytes_c, &c_full[cs]);
+        if (abytes_w) tc::bulk_g2s(arw + cs * arw_slot, p.Aw + row0 * p.r_r, abytes_w, &c_full[cs]);
+        ++nc;
+        for (int kb = kb0; kb < kb1; kb += 2, ++k) {
+          const int st = k % SP;
+          const uint32_t bytes = (uint32_t)(kb + 1 < kb1 ? 2 * kDecPk : kDecPk);
+          if (k >= SP && !tc::mbar_wait(&p_empty[st], ((k / SP) - 1) & 1, p.err)) {
+            ok = false;
+            break;
+          }
+          tc::fence_proxy_async_smem();
+          tc::mbar_arrive_expect_tx(&p_full[st], bytes);
+          tc::bulk_g2s(pk + (size_t)st * 2 * kDecPk, p.nib + ((T * nkb + kb) << 13), bytes,
+                       &p_full[st]);
+          ++np;
+        }
+        u += kb1 - kb0;
+      }
+      tc::mbar_wait(h_full, 0, p.err);
+      if (!ok) {  // drain copies still in flight before the CTA exits
+        for (int q = np - SP < 0 ? 0 : np - SP; q < np; ++q)
+          tc::mbar_wait(&p_full[q % SP], (q / SP) & 1, p.err);
+        for (int q = nc - 2 < 0 ? 0 : nc - 2; q < nc; ++q)
+          tc::mbar_wait(&c_full[q & 1], (q >> 1) & 1, p.err);
+      }
+    }
+    return;
+  }
+
+  // ---------------- consumers: warp w owns tile rows 16w .. 16w + 15 ----------------
+  const int gid = lane >> 2, tq = lane & 3;
+  const int ctid = threadIdx.x;  // 0 .. 255
+  bool ok = dec_wait(h_full, 0, p.err, true);
+  for (int i = ctid; i < NTOK * RR; i += kDecConsumers * 32) {  // ts[j * NTOK + n]
+    const int j = i / NTOK, n = i - j * NTOK;
+    ts[i] = n < p.N ? __ldg(p.t + (int64_t)n * RR + j) : 0.f;
+  }
+  asm volatile("bar.sync 1, 256;\n" ::: "memory");
+
+  const uint32_t pk_base = tc::smem_u32(pk);
+  // ldmatrix row address of this lane: matrix lane / 8 = (chunk lane / 16, row half
+  // (lane / 8) % 2), row lane % 8; the second load takes chunks 2 and 3
+  const uint32_t lm_off =
+      (uint32_t)(((lane >> 4) * 128 + 16 * warp + 8 * ((lane >> 3) & 1) + (lane & 7)) * 16);
+  const int r_lo = 16 * warp + gid, r_hi = r_lo + 8;
+  const float NEG_INF = __int_as_float(0xff800000);
+  // B reads: byte offset of token 8j + gid's columns 32 tq + 8c of block kb in the
+  // resident image is hrow[j] + 256 kb + hoff[c] (dec_h_offset unrolled)
+  int hrow[NT8];
+#pragma unroll
+  for (int j = 0; j < NT8; ++j) hrow[j] = (8 * j + gid) * (int)D * 2 + 64 * tq;
+  const int hx = (((tq >> 1) & 1) << 1) ^ (gid & 1);
+  int hoff[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) hoff[c] = 16 * (c ^ hx);
+
+  int k = 0, s = 0;
+  for (int64_t u = u0; u < u1; ++s) {
+    const int64_t T = u / nkb;
+    const int kb0 = (int)(u - T * nkb);
+    const int kb1 = (int)((int64_t)nkb < kb0 + (u1 - u) ? (int64_t)nkb : kb0 + (u1 - u));
+    const int cs = s & 1;
+    const int64_t row0 = T * 128;
+    const int64_t v_lo = row0 + r_lo, v_hi = row0 + r_hi;
+    const int64_t vc_lo = v_lo < p.V ? v_lo : p.V - 1, vc_hi = v_hi < p.V ? v_hi : p.V - 1;
+    // row scales for the epilogue: the loads overlap the block loop
+    const float S_lo = bf16_bits_to_float(__ldg(p.sup + vc_lo));
+    const float S_hi = bf16_bits_to_float(__ldg(p.sup + vc_hi));
+    const float sac_lo = p.r_c ? __ldg(p.sAc + vc_lo) : 0.f, sac_hi = p.r_c ? __ldg(p.sAc + vc_hi) : 0.f;
+    const float saw_lo = p.r_r ? __ldg(p.sAw + vc_lo) : 0.f, saw_hi = p.r_r ? __ldg(p.sAw + vc_hi) : 0.f;
+    ok = dec_wait(&c_full[cs], (s >> 1) & 1, p.err, ok);
+    const unsigned char* crow_lo = cds + cs * code_slot + r_lo * G;
+    const unsigned char* crow_hi = cds + cs * code_slot + r_hi * G;
+
+    float acc[NT8][4];
+#pragma unroll
+    for (int j = 0; j < NT8; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
+
+    int st = k % SP;
+    uint32_t ph = (uint32_t)(k / SP) & 1u;
+    for (int kb2 = kb0; kb2 < kb1; kb2 += 2, ++k) {
+      ok = dec_wait(&p_full[st], ph, p.err, ok);
+      const int nb = kb2 + 1 < kb1 ? 2 : 1;
+      uint32_t wlo[2][4], whi[2][4];  // [block][chunk]: word tq of rows r_lo, r_hi
+      uint32_t clo[2], chi[2];
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        if (b < nb) {
+          const uint32_t sa = pk_base + (uint32_t)(st * 2 + b) * kDecPk + lm_off;
+          uint32_t r[4];
+          ldmatrix_x4(sa, r);
+          wlo[b][0] = r[0]; whi[b][0] = r[1]; wlo[b][1] = r[2]; whi[b][1] = r[3];
+          ldmatrix_x4(sa + 2 * 128 * 16, r);
+          wlo[b][2] = r[0]; whi[b][2] = r[1]; wlo[b][3] = r[2]; whi[b][3] = r[3];
+          // group code of this thread's 32-column window (columns 32 tq .. 32 tq + 31)
+          const int kb = kb2 + b;
+          const int ci = CPC == 1 ? ((kb * 128) >> p.g_shift)
+                                  : (CPC == 2 ? kb * 2 + (tq >> 1) : kb * 4 + tq);
+          clo[b] = crow_lo[ci];
+          chi[b] = crow_hi[ci];
+        }
+      }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&p_empty[st]);
+      if (++st == SP) {
+        st = 0;
+        ph ^= 1u;
+      }
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        if (b >= nb) break;
+        const int kb = kb2 + b;
+        const int hb = kb * 256;
+        if (CPC == 1) {
+          // raw nibble reads into two FP32 partial sums, minus the offset correction,
+          // times the block's code
+          float t0[NT8][4], t1[NT8][4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t xa[4], xb[4];
+            nibble_reads(wlo[b][c], xa);
+            nibble_reads(whi[b][c], xb);
+            const uint32_t a0[4] = {xa[0], xb[0], xa[1], xb[1]};
+            const uint32_t a1[4] = {xa[2], xb[2], xa[3], xb[3]};
+#pragma unroll
+            for (int j = 0; j < NT8; ++j) {
+              const uint4 hv = *reinterpret_cast<const uint4*>(Hb + hrow[j] + hb + hoff[c]);
+              float* tt = (c & 1) ? t1[j] : t0[j];
+              if (c < 2) mma_f16_16816_z(tt, a0, hv.x, hv.y);
+              else mma_f16_16816(tt, a0, hv.x, hv.y);
+              mma_f16_16816(tt, a1, hv.z, hv.w);
+            }
+          }
+          const float fl = (float)clo[b], fh = (float)chi[b];
+#pragma unroll
+          for (int j = 0; j < NT8; ++j) {
+            const float2 cr = *reinterpret_cast<const float2*>(corr + kb * NTOK + 8 * j + 2 * tq);
+            acc[j][0] = fmaf(fl, (t0[j][0] + t1[j][0]) - cr.x, acc[j][0]);
+            acc[j][1] = fmaf(fl, (t0[j][1] + t1[j][1]) - cr.y, acc[j][1]);
+            acc[j][2] = fmaf(fh, (t0[j][2] + t1[j][2]) - cr.x, acc[j][2]);
+            acc[j][3] = fmaf(fh, (t0[j][3] + t1[j][3]) - cr.y, acc[j][3]);
+          }
+        } else {
+          const __half2 c2lo = __half2half2(__ushort2half_rn((unsigned short)clo[b]));
+          const __half2 c2hi = __half2half2(__ushort2half_rn((unsigned short)chi[b]));
+          const __half2 m24 = __float2half2_rn(-24.f);
+          const __half2 n2lo = __hmul2(c2lo, m24), n2hi = __hmul2(c2hi, m24);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            __half2 pa[4], pb[4];
+            dequant_word(wlo[b][c], c2lo, n2lo, pa);
+            dequant_word(whi[b][c], c2hi, n2hi, pb);
+            const uint32_t a0[4] = {h2_bits(pa[0]), h2_bits(pb[0]), h2_bits(pa[1]), h2_bits(pb[1])};
+            const uint32_t a1[4] = {h2_bits(pa[2]), h2_bits(pb[2]), h2_bits(pa[3]), h2_bits(pb[3])};
+#pragma unroll
+            for (int j = 0; j < NT8; ++j) {
+              const uint4 hv = *reinterpret_cast<const uint4*>(Hb + hrow[j] + hb + hoff[c]);
+              mma_f16_16816(acc[j], a0, hv.x, hv.y);
+              mma_f16_16816(acc[j], a1, hv.z, hv.w);
+            }
+          }
+        }
+      }
+    }
+
+    // ---- a tile split between CTAs: the last contributor to arrive finishes it ----
+    bool finish = kb0 == 0 && kb1 == nkb;
+    if (!finish) {
+      const int slot = u == u0 ? 0 : 1;
+      float4* dst = p.scratch + (((int64_t)blockIdx.x * 2 + slot) * 256 + ctid) * NT8;
+#pragma unroll
+      for (int j = 0; j < NT8; ++j) dst[j] = make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
+      __threadfence();
+      asm volatile("bar.sync 1, 256;\n" ::: "memory");
+      const int64_t cf = dec_cta_of(T * nkb, U, C), cl = dec_cta_of(T * nkb + nkb - 1, U, C);
+      if (ctid == 0) {
+        const unsigned old = atomicAdd(p.counters + T, 1u);
+        *flag = (int64_t)old + 1 == cl - cf + 1;
+      }
+      asm volatile("bar.sync 1, 256;\n" ::: "memory");
+      finish = *flag != 0;
+      if (finish) {
+        __threadfence();
+#pragma unroll
+        for (int j = 0; j < NT8; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
+        for (int64_t c = cf; c <= cl; ++c) {  // fixed order: the sum is deterministic
+          const int64_t first_tile = (U * c / C) / nkb;
+          const int sl = T == first_tile ? 0 : 1;
+          const float4* src = p.scratch + ((c * 2 + sl) * 256 + ctid) * NT8;
+#pragma unroll
+          for (int j = 0; j < NT8; ++j) {
+            const float4 q = __ldcg(src + j);
+            acc[j][0] += q.x; acc[j][1] += q.y; acc[j][2] += q.z; acc[j][3] += q.w;
+          }
+        }
+      }
+    }
+
+    if (finish) {
+      // ---- epilogue: S_v acc + sAc Ac . t_c + sAw Aw . t_w ----
+      const int64_t rows = p.V - row0 < 128 ? p.V - row0 : 128;
+      const bool acopy = dec_arow_copy(rows, p.r_c, p.r_r);
+      float y[NT8][4];
+#pragma unroll
+      for (int j = 0; j < NT8; ++j) {
+        y[j][0] = S_lo * acc[j][0];
+        y[j][1] = S_lo * acc[j][1];
+        y[j][2] = S_hi * acc[j][2];
+        y[j][3] = S_hi * acc[j][3];
+      }
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        const int rank = part == 0 ? p.r_c : p.r_r;
+        if (rank == 0) continue;
+        const int8_t* abase = acopy ? (part == 0 ? arc + cs * arc_slot : arw + cs * arw_slot)
+                                    : (part == 0 ? p.Ac : p.Aw);
+        const int8_t* alo = abase + (acopy ? (int64_t)r_lo : vc_lo) * rank;
+        const int8_t* ahi = abase + (acopy ? (int64_t)r_hi : vc_hi) * rank;
+        const float* tcol = ts + (part == 0 ? 0 : p.r_c) * NTOK + 2 * tq;
+        float llo[NT8][2], lhi[NT8][2];
+#pragma unroll
+        for (int j = 0; j < NT8; ++j) llo[j][0] = llo[j][1] = lhi[j][0] = lhi[j][1] = 0.f;
+        auto step = [&](float al, float ah, int i) {
+#pragma unroll
+          for (int j = 0; j < NT8; ++j) {
+            const float2 tv = *reinterpret_cast<const float2*>(tcol + i * NTOK + 8 * j);
+            llo[j][0] = fmaf(al, tv.x, llo[j][0]);
+            llo[j][1] = fmaf(al, tv.y, llo[j][1]);
+            lhi[j][0] = fmaf(ah, tv.x, lhi[j][0]);
+            lhi[j][1] = fmaf(ah, tv.y, lhi[j][1]);
+          }
+        };
+        int i = 0;
+        if ((rank & 3) == 0) {  // four INT8 entries per 32-bit load (rows 4-byte aligned)
+          for (; i < rank; i += 4) {
+            const uint32_t wl = *reinterpret_cast<const uint32_t*>(alo + i);
+            const uint32_t wh = *reinterpret_cast<const uint32_t*>(ahi + i);
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+              step((float)(int8_t)(wl >> (8 * b)), (float)(int8_t)(wh >> (8 * b)), i + b);
+          }
+        }
+        for (; i < rank; ++i) step((float)alo[i], (float)ahi[i], i);
+        const float sl = part == 0 ? sac_lo : saw_lo, sh = part == 0 ? sac_hi : saw_hi;
+#pragma unroll
+        for (int j = 0; j < NT8; ++j) {
+          y[j][0] = fmaf(sl, llo[j][0], y[j][0]);
+          y[j][1] = fmaf(sl, llo[j][1], y[j][1]);
+          y[j][2] = fmaf(sh, lhi[j][0], y[j][2]);
+          y[j][3] = fmaf(sh, lhi[j][1], y[j][3]);
+        }
+      }
+      if (MODE == 0) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int64_t v = h ? v_hi : v_lo;
+          if (v >= p.V) continue;
+#pragma unroll
+          for (int j = 0; j < NT8; ++j)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int64_t tok = 8 * j + 2 * tq + e;
+              if (tok < p.N) p.Y[tok * p.V + v] = y[j][2 * h + e];
+            }
+        }
+      } else {
+        // ---- fused NLL: per token (max, sum exp) over the tile's rows, target logit ----
+#pragma unroll
+        for (int j = 0; j < NT8; ++j)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            float mx = NEG_INF;
+            if (v_lo < p.V) mx = fmaxf(mx, y[j][e]);
+            if (v_hi < p.V) mx = fmaxf(mx, y[j][2 + e]);
+            float sm = 0.f;
+            if (v_lo < p.V) sm += __expf(y[j][e] - mx);
+            if (v_hi < p.V) sm += __expf(y[j][2 + e] - mx);
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) {  // the 8 lanes sharing this token
+              const float mo = __shfl_xor_sync(0xffffffffu, mx, o);
+              const float so = __shfl_xor_sync(0xffffffffu, sm, o);
+              const float mn = fmaxf(mx, mo);
+              sm = (mx == NEG_INF ? 0.f : sm * __expf(mx - mn)) +
+                   (mo == NEG_INF ? 0.f : so * __expf(mo - mn));
+              mx = mn;
+            }
+            const int n = 8 * j + 2 * tq + e;
+            if (gid == 0) red[warp * NTOK + n] = make_float2(mx, sm);
+            if (n < p.N) {
+              const int64_t tgt = __ldg(p.targets + n);
+              if (v_lo == tgt && v_lo < p.V) p.tlogit[n] = y[j][e];
+              if (v_hi == tgt && v_hi < p.V) p.tlogit[n] = y[j][2 + e];
+            }
+          }
+        asm volatile("bar.sync 1, 256;\n" ::: "memory");
+        for (int n = ctid; n < NTOK; n += kDecConsumers * 32) {
+          if (n >= p.N) continue;
+          float mx = NEG_INF, sm = 0.f;
+          for (int w = 0; w < kDecConsumers; ++w) {
+            const float2 q = red[w * NTOK + n];
+            const float mn = fmaxf(mx, q.x);
+            sm = (mx == NEG_INF ? 0.f : sm * __expf(mx - mn)) +
+                 (q.x == NEG_INF ? 0.f : q.y * __expf(q.x - mn));
+            mx = mn;
+          }
+          p.part[(int64_t)n * p.n_vtiles + T] = make_float2(mx, sm);
+        }
+        asm volatile("bar.sync 1, 256;\n" ::: "memory");
+      }
+    }
+    __syncwarp();
+    if (lane == 0) tc::mbar_arrive(&c_empty[cs]);
+    u += kb1 - kb0;
+  }
+}
+
+template <int NT8, int CPC, int MODE>
+cudaError_t launch_dec_cfg(const DecParams& p, int grid, cudaStream_t st) {
+  const int G = (int)(p.D >> p.g_shift);
+  const size_t smem = dec_smem<NT8, MODE>(p.D, G, p.r_c, p.r_r, p.sp).total;
+  auto kern = residual_dec_kernel<NT8, CPC, MODE>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<(unsigned)grid, kDecThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <int NT8, int MODE>
+cudaError_t launch_dec_nt(const DecParams& p, int g, int grid, cudaStream_t st) {
+  if (g == 32) return launch_dec_cfg<NT8, 4, MODE>(p, grid, st);
+  if (g == 64) return launch_dec_cfg<NT8, 2, MODE>(p, grid, st);
+  return launch_dec_cfg<NT8, 1, MODE>(p, grid, st);
+}
+
+template <int NT8, int MODE>
+int fit_sp(const Shapes& s, size_t budget) {
+  const int G = (int)(s.D / s.g);
+  for (int sp = kDecMaxSP; sp >= 3; --sp)
+    if (dec_smem<NT8, MODE>(s.D, G, s.r_c, s.r_r, sp).total <= budget) return sp;
+  return 0;
+}
+
+}  // namespace
+
+DecPlan dec_plan(const Shapes& s, bool nll) {
+  DecPlan pl = {0, 0, 0};
+  if (s.N < 1 || s.N > 16) return pl;
+  const size_t budget = 227 * 1024;  // one CTA per SM
+  const int nt8 = s.N <= 8 ? 1 : 2;
+  int sp;
+  if (nt8 == 1) sp = nll ? fit_sp<1, 1>(s, budget) : fit_sp<1, 0>(s, budget);
+  else sp = nll ? fit_sp<2, 1>(s, budget) : fit_sp<2, 0>(s, budget);
+  if (!sp) return pl;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return pl;
+  const int64_t units = (s.V + 127) / 128 * (s.D / 128);
+  pl.nt8 = nt8;
+  pl.sp = sp;
+  pl.grid = (int)(units < sms ? units : sms);
+  return pl;
+}
+
+size_t dec_image_bytes(const Shapes& s, const DecPlan& pl) {
+  return (size_t)8 * pl.nt8 * s.D * 2 + (size_t)(s.D / 128) * 8 * pl.nt8 * 4;
+}
+size_t dec_partial_bytes(const DecPlan& pl) { return (size_t)pl.grid * 2 * 256 * pl.nt8 * 16; }
+
+cudaError_t launch_dec_prologue(const uint16_t* H, const archead_head* head, const Shapes& s,
+                                const DecPlan& pl, __half* img, float* t, unsigned* counters,
+                                unsigned* err, cudaStream_t st, int* launches) {
+  const int64_t ntok = 8 * pl.nt8;
+  const int64_t n_counters = (s.V + 127) / 128;
+  // one warp per (token, 128-column block); the counters ride on the same grid
+  int64_t blocks = (ntok * (s.D / 128) * 32 + 255) / 256;
+  const int64_t cb = (n_counters + 255) / 256;
+  if (cb > blocks) blocks = cb;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  dec_convert_h_kernel<<<(unsigned)blocks, 256, 0, st>>>(H, img, s.N, (int)ntok, s.D,
+                                                         s.g >= 128 ? 1 : 0, counters,
+                                                         n_counters, err);
+  ++*launches;
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_lowrank_t(H, head, s, t, nullptr, 0, 0, err, st, launches);
+}
+
+cudaError_t launch_residual_dec(const __half* img, const float* t, const archead_head* head,
+                                const Shapes& s, const DecPlan& pl, float* Y,
+                                const int32_t* targets, float2* part, float* tlogit,
+                                float4* scratch, unsigned* counters, unsigned* err,
+                                cudaStream_t st, int* launches) {
+  DecParams p;
+  p.Himg = img;
+  p.t = t;
+  p.nib = head->r_nib;
+  p.code = head->r_code;
+  p.sup = head->r_super;
+  p.Ac = head->Ac;
+  p.sAc = head->sAc;
+  p.Aw = head->Aw;
+  p.sAw = head->sAw;
+  p.Y = Y;
+  p.targets = targets;
+  p.part = part;
+  p.tlogit = tlogit;
+  p.scratch = scratch;
+  p.counters = counters;
+  p.N = s.N;
+  p.V = s.V;
+  p.D = s.D;
+  p.r_c = s.r_c;
+  p.r_r = s.r_r;
+  int gs = 0;
+  while ((1 << gs) < s.g) ++gs;
+  p.g_shift = gs;
+  p.sp = pl.sp;
+  p.n_vtiles = (s.V + 127) / 128;
+  p.err = err;
+  if (pl.nt8 < 1 || pl.nt8 > 2 || pl.sp < 3 || pl.sp > kDecMaxSP || pl.grid < 1)
+    return cudaErrorInvalidValue;
+  cudaError_t e;
+  if (pl.nt8 == 1)
+    e = Y ? launch_dec_nt<1, 0>(p, s.g, pl.grid, st) : launch_dec_nt<1, 1>(p, s.g, pl.grid, st);
+  else
+    e = Y ? launch_dec_nt<2, 0>(p, s.g, pl.grid, st) : launch_dec_nt<2, 1>(p, s.g, pl.grid, st);
+  ++*launches;
+  return e;
+}
+
+}  // namespace archead
