@@ -29,8 +29,7 @@
 namespace archead {
 namespace {
 
-constexpr int kDecConsumers = 8;                        // consumer warps (16 rows each)
-constexpr int kDecThreads = (kDecConsumers + 1) * 32;   // + producer warp
+constexpr int kDecRows = 8;  // 16-row groups of a 128-row tile (one warp each per stage)
 constexpr int kDecPk = 8192;                            // packed block of one tile
 
 struct DecParams {
@@ -68,13 +67,25 @@ __host__ __device__ __forceinline__ int64_t dec_h_offset(int64_t n, int64_t d, i
 template <int NT8>
 struct DecCfg {
   static constexpr int NTOK = 8 * NT8;
+  // consumer warps per row group, taking alternate ring stages (latency hiding where the
+  // registers allow two)
+  static constexpr int PAR = NT8 == 1 ? 2 : 1;
+  static constexpr int CONSUMERS = kDecRows * PAR;
+  static constexpr int THREADS = (CONSUMERS + 1) * 32;  // + producer warp
 };
 
 __host__ __device__ inline size_t dec_round16(size_t x) { return (x + 15) & ~(size_t)15; }
 
 struct DecSmem {
-  size_t h, pk, codes, arow_c, arow_w, ts, red, bars, total;
+  size_t h, pk, codes, arow_c, arow_w, ts, ts16, red, xch, bars, total;
 };
+
+// Row stride in bytes of the FP16 t pieces: RR halves rounded up to 128 bytes plus 32, so
+// the stride in 32-bit words is 8 mod 32 and the 64-bit B-fragment reads of a half warp
+// (four tokens x four K offsets) fall in distinct banks.
+__host__ __device__ inline size_t dec_ts16_stride(int RR) {
+  return ((size_t)RR * 2 + 127) / 128 * 128 + 32;
+}
 
 // Shared-memory carve-up (offsets from a 128-byte aligned base).
 template <int NT8, int MODE>
@@ -94,8 +105,12 @@ __host__ __device__ inline DecSmem dec_smem(int64_t D, int G, int r_c, int r_r, 
   o += 2 * dec_round16((size_t)128 * r_r);
   m.ts = o;  // [NTOK][RR + 1] FP32
   o += dec_round16((size_t)NTOK * (r_c + r_r + 1) * 4);
+  m.ts16 = o;  // [2 pieces][NTOK rows of dec_ts16_stride bytes] FP16 hi / lo of t
+  o += (size_t)2 * NTOK * dec_ts16_stride(r_c + r_r);
   m.red = o;  // MODE 1: [8 warps][NTOK] float2
-  o += MODE ? dec_round16((size_t)kDecConsumers * NTOK * 8) : 0;
+  o += MODE ? dec_round16((size_t)kDecRows * NTOK * 8) : 0;
+  m.xch = o;  // paired warps: [2][256][NT8] float4 partial sums handed over per tile
+  o += DecCfg<NT8>::PAR == 2 ? (size_t)2 * 256 * NT8 * 16 : 0;
   m.bars = o;
   o += 256;
   m.total = o;
@@ -207,9 +222,61 @@ __device__ __forceinline__ void nibble_reads(uint32_t w, uint32_t x[4]) {
   x[3] = and_xor(w2, 0x00F000F0u, 0x64806480u);
 }
 
+// NB (1 or 2) consecutive blocks with one group code each (g >= 128): raw nibble reads
+// (nibble_reads) times the resident B image, one independent two-MMA chain per (block,
+// chunk), then acc += code * (sum of the chains - corr).  The chains are summed in a fixed
+// order.
+template <int NT8, int NB>
+__device__ __forceinline__ void dec_blocks_q(const uint32_t (&wlo)[2][4],
+                                             const uint32_t (&whi)[2][4],
+                                             const uint32_t (&clo)[2], const uint32_t (&chi)[2],
+                                             const unsigned char* Hb, const int (&hrow)[NT8],
+                                             const int (&hoff)[4], const float* corr, int kb2,
+                                             int tq, float (&acc)[NT8][4]) {
+  constexpr int NTOK = 8 * NT8;
+  float t[NB][4][NT8][4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      uint32_t xa[4], xb[4];
+      nibble_reads(wlo[b][c], xa);
+      nibble_reads(whi[b][c], xb);
+      const uint32_t a0[4] = {xa[0], xb[0], xa[1], xb[1]};
+      const uint32_t a1[4] = {xa[2], xb[2], xa[3], xb[3]};
+#pragma unroll
+      for (int j = 0; j < NT8; ++j) {
+        const uint4 hv =
+            *reinterpret_cast<const uint4*>(Hb + hrow[j] + (kb2 + b) * 256 + hoff[c]);
+        mma_f16_16816_z(t[b][c][j], a0, hv.x, hv.y);
+        mma_f16_16816(t[b][c][j], a1, hv.z, hv.w);
+      }
+    }
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    const float fl = (float)clo[b], fh = (float)chi[b];
+#pragma unroll
+    for (int j = 0; j < NT8; ++j) {
+      const float2 cr =
+          *reinterpret_cast<const float2*>(corr + (kb2 + b) * NTOK + 8 * j + 2 * tq);
+      float sm[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        sm[e] = (t[b][0][j][e] + t[b][1][j][e]) + (t[b][2][j][e] + t[b][3][j][e]);
+      acc[j][0] = fmaf(fl, sm[0] - cr.x, acc[j][0]);
+      acc[j][1] = fmaf(fl, sm[1] - cr.y, acc[j][1]);
+      acc[j][2] = fmaf(fh, sm[2] - cr.x, acc[j][2]);
+      acc[j][3] = fmaf(fh, sm[3] - cr.y, acc[j][3]);
+    }
+  }
+}
+
 template <int NT8, int CPC, int MODE>
-__global__ void __launch_bounds__(kDecThreads, 1) residual_dec_kernel(const DecParams p) {
+__global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
+    residual_dec_kernel(const DecParams p) {
   constexpr int NTOK = DecCfg<NT8>::NTOK;
+  constexpr int PAR = DecCfg<NT8>::PAR;
+  constexpr int CONSUMERS = DecCfg<NT8>::CONSUMERS;
   extern __shared__ __align__(128) unsigned char smem[];
   const int64_t D = p.D;
   const int nkb = (int)(D / 128);
@@ -224,7 +291,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) residual_dec_kernel(const DecP
   int8_t* arc = reinterpret_cast<int8_t*>(smem + m.arow_c);
   int8_t* arw = reinterpret_cast<int8_t*>(smem + m.arow_w);
   float* ts = reinterpret_cast<float*>(smem + m.ts);  // ts[j * NTOK + n]
+  unsigned char* ts16 = smem + m.ts16;
+  const int tsb = (int)dec_ts16_stride(p.r_c + p.r_r);
+  // rank terms on the tensor cores when both ranks are whole K=16 steps
+  const bool rank_mma = (p.r_c % 16) == 0 && (p.r_r % 16) == 0;
   float2* red = reinterpret_cast<float2*>(smem + m.red);
+  float4* xch = reinterpret_cast<float4*>(smem + m.xch);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + m.bars);
   uint64_t* h_full = bars;       // [1]
   uint64_t* c_full = bars + 1;   // [2]
@@ -246,17 +318,17 @@ __global__ void __launch_bounds__(kDecThreads, 1) residual_dec_kernel(const DecP
     tc::mbar_init(h_full, 1);
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&c_full[s], 1);
-      tc::mbar_init(&c_empty[s], kDecConsumers);
+      tc::mbar_init(&c_empty[s], CONSUMERS);
     }
     for (int s = 0; s < SP; ++s) {
       tc::mbar_init(&p_full[s], 1);
-      tc::mbar_init(&p_empty[s], kDecConsumers);
+      tc::mbar_init(&p_empty[s], kDecRows);  // one warp per row group takes a stage
     }
     tc::mbar_fence_init();
   }
   __syncthreads();
 
-  if (warp == kDecConsumers) {
+  if (warp == CONSUMERS) {
     // ---------------- producer (one thread) ----------------
     // A stage holds up to two consecutive blocks of one tile (contiguous in the device
     // layout, so one bulk copy).
@@ -312,22 +384,32 @@ __global__ void __launch_bounds__(kDecThreads, 1) residual_dec_kernel(const DecP
     return;
   }
 
-  // ---------------- consumers: warp w owns tile rows 16w .. 16w + 15 ----------------
+  // ---- consumers: warps w and w + 8 own tile rows 16w .. 16w + 15, taking the even and
+  // the odd ring stages (PAR = 2) ----
   const int gid = lane >> 2, tq = lane & 3;
-  const int ctid = threadIdx.x;  // 0 .. 255
+  const int par = warp / kDecRows;
+  const int ctid = threadIdx.x;  // the first eight warps: 0 .. 255
   bool ok = dec_wait(h_full, 0, p.err, true);
-  for (int i = ctid; i < NTOK * RR; i += kDecConsumers * 32) {  // ts[j * NTOK + n]
+  for (int i = ctid; i < NTOK * RR; i += CONSUMERS * 32) {  // ts[j * NTOK + n]
     const int j = i / NTOK, n = i - j * NTOK;
-    ts[i] = n < p.N ? __ldg(p.t + (int64_t)n * RR + j) : 0.f;
+    const float tv = n < p.N ? __ldg(p.t + (int64_t)n * RR + j) : 0.f;
+    ts[i] = tv;
+    // FP16 pieces: t1 + t2 carries 22 significant bits of t
+    const __half t1 = __float2half_rn(tv);
+    const __half t2 = __float2half_rn(tv - __half2float(t1));
+    if (rank_mma && !(fabsf(tv) < 65504.f) && blockIdx.x == 0) atomicOr(p.err, kErrRangeH);
+    *reinterpret_cast<__half*>(ts16 + n * tsb + j * 2) = t1;
+    *reinterpret_cast<__half*>(ts16 + (NTOK + n) * tsb + j * 2) = t2;
   }
-  asm volatile("bar.sync 1, 256;\n" ::: "memory");
+  asm volatile("bar.sync 10, %0;\n" ::"r"(CONSUMERS * 32) : "memory");
 
   const uint32_t pk_base = tc::smem_u32(pk);
   // ldmatrix row address of this lane: matrix lane / 8 = (chunk lane / 16, row half
   // (lane / 8) % 2), row lane % 8; the second load takes chunks 2 and 3
   const uint32_t lm_off =
-      (uint32_t)(((lane >> 4) * 128 + 16 * warp + 8 * ((lane >> 3) & 1) + (lane & 7)) * 16);
-  const int r_lo = 16 * warp + gid, r_hi = r_lo + 8;
+      (uint32_t)(((lane >> 4) * 128 + 16 * (warp % kDecRows) + 8 * ((lane >> 3) & 1) +
+                  (lane & 7)) * 16);
+  const int r_lo = 16 * (warp % kDecRows) + gid, r_hi = r_lo + 8;
   const float NEG_INF = __int_as_float(0xff800000);
   // B reads: byte offset of token 8j + gid's columns 32 tq + 8c of block kb in the
   // resident image is hrow[j] + 256 kb + hoff[c] (dec_h_offset unrolled)
@@ -366,6 +448,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) residual_dec_kernel(const DecP
     int st = k % SP;
     uint32_t ph = (uint32_t)(k / SP) & 1u;
     for (int kb2 = kb0; kb2 < kb1; kb2 += 2, ++k) {
+      if (PAR == 2 && (k & 1) != par) {  // the other warp of the pair takes this stage
+        if (++st == SP) {
+          st = 0;
+          ph ^= 1u;
+        }
+        continue;
+      }
       ok = dec_wait(&p_full[st], ph, p.err, ok);
       const int nb = kb2 + 1 < kb1 ? 2 : 1;
       uint32_t wlo[2][4], whi[2][4];  // [block][chunk]: word tq of rows r_lo, r_hi
@@ -393,41 +482,16 @@ __global__ void __launch_bounds__(kDecThreads, 1) residual_dec_kernel(const DecP
         st = 0;
         ph ^= 1u;
       }
+      if (CPC == 1) {
+        if (nb == 2)
+          dec_blocks_q<NT8, 2>(wlo, whi, clo, chi, Hb, hrow, hoff, corr, kb2, tq, acc);
+        else
+          dec_blocks_q<NT8, 1>(wlo, whi, clo, chi, Hb, hrow, hoff, corr, kb2, tq, acc);
+      } else {
 #pragma unroll
-      for (int b = 0; b < 2; ++b) {
-        if (b >= nb) break;
-        const int kb = kb2 + b;
-        const int hb = kb * 256;
-        if (CPC == 1) {
-          // raw nibble reads into two FP32 partial sums, minus the offset correction,
-          // times the block's code
-          float t0[NT8][4], t1[NT8][4];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t xa[4], xb[4];
-            nibble_reads(wlo[b][c], xa);
-            nibble_reads(whi[b][c], xb);
-            const uint32_t a0[4] = {xa[0], xb[0], xa[1], xb[1]};
-            const uint32_t a1[4] = {xa[2], xb[2], xa[3], xb[3]};
-#pragma unroll
-            for (int j = 0; j < NT8; ++j) {
-              const uint4 hv = *reinterpret_cast<const uint4*>(Hb + hrow[j] + hb + hoff[c]);
-              float* tt = (c & 1) ? t1[j] : t0[j];
-              if (c < 2) mma_f16_16816_z(tt, a0, hv.x, hv.y);
-              else mma_f16_16816(tt, a0, hv.x, hv.y);
-              mma_f16_16816(tt, a1, hv.z, hv.w);
-            }
-          }
-          const float fl = (float)clo[b], fh = (float)chi[b];
-#pragma unroll
-          for (int j = 0; j < NT8; ++j) {
-            const float2 cr = *reinterpret_cast<const float2*>(corr + kb * NTOK + 8 * j + 2 * tq);
-            acc[j][0] = fmaf(fl, (t0[j][0] + t1[j][0]) - cr.x, acc[j][0]);
-            acc[j][1] = fmaf(fl, (t0[j][1] + t1[j][1]) - cr.y, acc[j][1]);
-            acc[j][2] = fmaf(fh, (t0[j][2] + t1[j][2]) - cr.x, acc[j][2]);
-            acc[j][3] = fmaf(fh, (t0[j][3] + t1[j][3]) - cr.y, acc[j][3]);
-          }
-        } else {
+        for (int b = 0; b < 2; ++b) {
+          if (b >= nb) break;
+          const int hb = (kb2 + b) * 256;
           const __half2 c2lo = __half2half2(__ushort2half_rn((unsigned short)clo[b]));
           const __half2 c2hi = __half2half2(__ushort2half_rn((unsigned short)chi[b]));
           const __half2 m24 = __float2half2_rn(-24.f);
@@ -447,6 +511,27 @@ __global__ void __launch_bounds__(kDecThreads, 1) residual_dec_kernel(const DecP
             }
           }
         }
+      }
+    }
+
+    // ---- paired warps: the odd-stage warp hands its sums to the even-stage warp ----
+    if (PAR == 2) {
+      float4* xs = xch + ((size_t)(s & 1) * 256 + (warp % kDecRows) * 32 + lane) * NT8;
+      if (par) {
+#pragma unroll
+        for (int j = 0; j < NT8; ++j) xs[j] = make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
+      }
+      asm volatile("bar.sync %0, 64;\n" ::"r"(2 + warp % kDecRows) : "memory");
+      if (par) {
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&c_empty[cs]);
+        u += kb1 - kb0;
+        continue;
+      }
+#pragma unroll
+      for (int j = 0; j < NT8; ++j) {
+        const float4 q = xs[j];
+        acc[j][0] += q.x; acc[j][1] += q.y; acc[j][2] += q.z; acc[j][3] += q.w;
       }
     }
 
@@ -497,46 +582,92 @@ __global__ void __launch_bounds__(kDecThreads, 1) residual_dec_kernel(const DecP
         y[j][2] = S_hi * acc[j][2];
         y[j][3] = S_hi * acc[j][3];
       }
+      if (rank_mma) {
+        // [A_c | A_w] rows (INT8, exact in FP16) x FP16 hi / lo pieces of t, one FP32
+        // accumulator per factor; thread q's K slots hold factor entries 16 s + 4 q + 0..3
 #pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        const int rank = part == 0 ? p.r_c : p.r_r;
-        if (rank == 0) continue;
-        const int8_t* abase = acopy ? (part == 0 ? arc + cs * arc_slot : arw + cs * arw_slot)
-                                    : (part == 0 ? p.Ac : p.Aw);
-        const int8_t* alo = abase + (acopy ? (int64_t)r_lo : vc_lo) * rank;
-        const int8_t* ahi = abase + (acopy ? (int64_t)r_hi : vc_hi) * rank;
-        const float* tcol = ts + (part == 0 ? 0 : p.r_c) * NTOK + 2 * tq;
-        float llo[NT8][2], lhi[NT8][2];
+        for (int part = 0; part < 2; ++part) {
+          const int rank = part == 0 ? p.r_c : p.r_r;
+          if (rank == 0) continue;
+          const int8_t* abase = acopy ? (part == 0 ? arc + cs * arc_slot : arw + cs * arw_slot)
+                                      : (part == 0 ? p.Ac : p.Aw);
+          const int8_t* alo = abase + (acopy ? (int64_t)r_lo : vc_lo) * rank;
+          const int8_t* ahi = abase + (acopy ? (int64_t)r_hi : vc_hi) * rank;
+          const int off = part == 0 ? 0 : p.r_c;
+          float L[NT8][4];
 #pragma unroll
-        for (int j = 0; j < NT8; ++j) llo[j][0] = llo[j][1] = lhi[j][0] = lhi[j][1] = 0.f;
-        auto step = [&](float al, float ah, int i) {
+          for (int j = 0; j < NT8; ++j) L[j][0] = L[j][1] = L[j][2] = L[j][3] = 0.f;
+          const __half2 k1152 = __float2half2_rn(1152.f);
+          for (int st16 = 0; st16 < rank; st16 += 16) {
+            const uint32_t wl = *reinterpret_cast<const uint32_t*>(alo + st16 + 4 * tq) ^ 0x80808080u;
+            const uint32_t wh = *reinterpret_cast<const uint32_t*>(ahi + st16 + 4 * tq) ^ 0x80808080u;
+            // bytes b + 128 under the FP16 pattern 0x6400 read 1024 + b + 128: minus 1152
+            uint32_t q0 = __byte_perm(wl, 0x64646464u, 0x5140), q1 = __byte_perm(wl, 0x64646464u, 0x7352);
+            uint32_t q2 = __byte_perm(wh, 0x64646464u, 0x5140), q3 = __byte_perm(wh, 0x64646464u, 0x7352);
+            const uint32_t a[4] = {h2_bits(__hsub2(*reinterpret_cast<__half2*>(&q0), k1152)),
+                                   h2_bits(__hsub2(*reinterpret_cast<__half2*>(&q2), k1152)),
+                                   h2_bits(__hsub2(*reinterpret_cast<__half2*>(&q1), k1152)),
+                                   h2_bits(__hsub2(*reinterpret_cast<__half2*>(&q3), k1152))};
+#pragma unroll
+            for (int pc = 0; pc < 2; ++pc)
+#pragma unroll
+              for (int j = 0; j < NT8; ++j) {
+                const uint2 bv = *reinterpret_cast<const uint2*>(
+                    ts16 + (pc * NTOK + 8 * j + gid) * tsb + (off + st16 + 4 * tq) * 2);
+                mma_f16_16816(L[j], a, bv.x, bv.y);
+              }
+          }
+          const float sl = part == 0 ? sac_lo : saw_lo, sh = part == 0 ? sac_hi : saw_hi;
 #pragma unroll
           for (int j = 0; j < NT8; ++j) {
-            const float2 tv = *reinterpret_cast<const float2*>(tcol + i * NTOK + 8 * j);
-            llo[j][0] = fmaf(al, tv.x, llo[j][0]);
-            llo[j][1] = fmaf(al, tv.y, llo[j][1]);
-            lhi[j][0] = fmaf(ah, tv.x, lhi[j][0]);
-            lhi[j][1] = fmaf(ah, tv.y, lhi[j][1]);
-          }
-        };
-        int i = 0;
-        if ((rank & 3) == 0) {  // four INT8 entries per 32-bit load (rows 4-byte aligned)
-          for (; i < rank; i += 4) {
-            const uint32_t wl = *reinterpret_cast<const uint32_t*>(alo + i);
-            const uint32_t wh = *reinterpret_cast<const uint32_t*>(ahi + i);
-#pragma unroll
-            for (int b = 0; b < 4; ++b)
-              step((float)(int8_t)(wl >> (8 * b)), (float)(int8_t)(wh >> (8 * b)), i + b);
+            y[j][0] = fmaf(sl, L[j][0], y[j][0]);
+            y[j][1] = fmaf(sl, L[j][1], y[j][1]);
+            y[j][2] = fmaf(sh, L[j][2], y[j][2]);
+            y[j][3] = fmaf(sh, L[j][3], y[j][3]);
           }
         }
-        for (; i < rank; ++i) step((float)alo[i], (float)ahi[i], i);
-        const float sl = part == 0 ? sac_lo : saw_lo, sh = part == 0 ? sac_hi : saw_hi;
+      } else {
 #pragma unroll
-        for (int j = 0; j < NT8; ++j) {
-          y[j][0] = fmaf(sl, llo[j][0], y[j][0]);
-          y[j][1] = fmaf(sl, llo[j][1], y[j][1]);
-          y[j][2] = fmaf(sh, lhi[j][0], y[j][2]);
-          y[j][3] = fmaf(sh, lhi[j][1], y[j][3]);
+        for (int part = 0; part < 2; ++part) {
+          const int rank = part == 0 ? p.r_c : p.r_r;
+          if (rank == 0) continue;
+          const int8_t* abase = acopy ? (part == 0 ? arc + cs * arc_slot : arw + cs * arw_slot)
+                                      : (part == 0 ? p.Ac : p.Aw);
+          const int8_t* alo = abase + (acopy ? (int64_t)r_lo : vc_lo) * rank;
+          const int8_t* ahi = abase + (acopy ? (int64_t)r_hi : vc_hi) * rank;
+          const float* tcol = ts + (part == 0 ? 0 : p.r_c) * NTOK + 2 * tq;
+          float llo[NT8][2], lhi[NT8][2];
+  #pragma unroll
+          for (int j = 0; j < NT8; ++j) llo[j][0] = llo[j][1] = lhi[j][0] = lhi[j][1] = 0.f;
+          auto step = [&](float al, float ah, int i) {
+  #pragma unroll
+            for (int j = 0; j < NT8; ++j) {
+              const float2 tv = *reinterpret_cast<const float2*>(tcol + i * NTOK + 8 * j);
+              llo[j][0] = fmaf(al, tv.x, llo[j][0]);
+              llo[j][1] = fmaf(al, tv.y, llo[j][1]);
+              lhi[j][0] = fmaf(ah, tv.x, lhi[j][0]);
+              lhi[j][1] = fmaf(ah, tv.y, lhi[j][1]);
+            }
+          };
+          int i = 0;
+          if ((rank & 3) == 0) {  // four INT8 entries per 32-bit load (rows 4-byte aligned)
+            for (; i < rank; i += 4) {
+              const uint32_t wl = *reinterpret_cast<const uint32_t*>(alo + i);
+              const uint32_t wh = *reinterpret_cast<const uint32_t*>(ahi + i);
+  #pragma unroll
+              for (int b = 0; b < 4; ++b)
+                step((float)(int8_t)(wl >> (8 * b)), (float)(int8_t)(wh >> (8 * b)), i + b);
+            }
+          }
+          for (; i < rank; ++i) step((float)alo[i], (float)ahi[i], i);
+          const float sl = part == 0 ? sac_lo : saw_lo, sh = part == 0 ? sac_hi : saw_hi;
+  #pragma unroll
+          for (int j = 0; j < NT8; ++j) {
+            y[j][0] = fmaf(sl, llo[j][0], y[j][0]);
+            y[j][1] = fmaf(sl, llo[j][1], y[j][1]);
+            y[j][2] = fmaf(sh, lhi[j][0], y[j][2]);
+            y[j][3] = fmaf(sh, lhi[j][1], y[j][3]);
+          }
         }
       }
       if (MODE == 0) {
@@ -582,10 +713,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) residual_dec_kernel(const DecP
             }
           }
         asm volatile("bar.sync 1, 256;\n" ::: "memory");
-        for (int n = ctid; n < NTOK; n += kDecConsumers * 32) {
+        for (int n = ctid; n < NTOK; n += kDecRows * 32) {
           if (n >= p.N) continue;
           float mx = NEG_INF, sm = 0.f;
-          for (int w = 0; w < kDecConsumers; ++w) {
+          for (int w = 0; w < kDecRows; ++w) {
             const float2 q = red[w * NTOK + n];
             const float mn = fmaxf(mx, q.x);
             sm = (mx == NEG_INF ? 0.f : sm * __expf(mx - mn)) +
@@ -611,7 +742,8 @@ cudaError_t launch_dec_cfg(const DecParams& p, int grid, cudaStream_t st) {
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<(unsigned)grid, kDecThreads, smem, st>>>(p);
+  if (DecCfg<NT8>::PAR == 2 && p.sp % 2 != 0) return cudaErrorInvalidValue;
+  kern<<<(unsigned)grid, DecCfg<NT8>::THREADS, smem, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -622,11 +754,17 @@ cudaError_t launch_dec_nt(const DecParams& p, int g, int grid, cudaStream_t st) 
   return launch_dec_cfg<NT8, 1, MODE>(p, grid, st);
 }
 
+// Paired warps take stages by the parity of the global stage index; with an even number
+// of ring slots every use of a slot then goes to the same warp, which never waits on a
+// slot's mbarrier more than one phase ahead (an odd count would let a fast warp skip a
+// phase and alias the parity test).
 template <int NT8, int MODE>
 int fit_sp(const Shapes& s, size_t budget) {
   const int G = (int)(s.D / s.g);
   for (int sp = kDecMaxSP; sp >= 3; --sp)
-    if (dec_smem<NT8, MODE>(s.D, G, s.r_c, s.r_r, sp).total <= budget) return sp;
+    if ((DecCfg<NT8>::PAR == 1 || sp % 2 == 0) &&
+        dec_smem<NT8, MODE>(s.D, G, s.r_c, s.r_r, sp).total <= budget)
+      return sp;
   return 0;
 }
 
