@@ -3,7 +3,7 @@
 //   * Hh = fp16(H), zero-padded to Npad rows -- the B operand of the residual contraction;
 //   * t  = H [Q8(B_c) | Q8(B_w)]^T, N x (r_c + r_r) FP32 -- the rank terms' left products
 //     (for the tcgen05 path, split into FP16 pieces inside the MMA's B image instead).
-#include "archead_internal.cuh"
+#include "tc_common.cuh"
 
 namespace archead {
 namespace {
@@ -49,6 +49,7 @@ __global__ void __launch_bounds__(256) lowrank_t_kernel(
     const float* __restrict__ sBw, int r_c, int r_r, int64_t N, int64_t D, int g,
     float* __restrict__ t, __half* __restrict__ img, int nt, int64_t nkbt,
     unsigned* err) {
+  allow_dependent_launch();
   const int j = blockIdx.y;
   const int RR = r_c + r_r;
   const int8_t* B;
@@ -104,6 +105,9 @@ __global__ void __launch_bounds__(256) lowrank_t_kernel(
 #pragma unroll
     for (int w = 0; w < 8; ++w) v += red[w][threadIdx.x];
     const int64_t n = n0 + threadIdx.x;
+    // the image's rank blocks were zero-filled by the previous kernel (this one may be a
+    // programmatic dependent launch of it)
+    if (img) grid_dependency_wait();
     if (!img) {
       t[n * RR + j] = v;
     } else {
@@ -144,9 +148,25 @@ cudaError_t launch_lowrank_t(const uint16_t* H, const archead_head* head, const 
   const int RR = s.r_c + s.r_r;
   if (RR > 0) {
     dim3 grid((unsigned)((s.N + kTN - 1) / kTN), RR);
-    lowrank_t_kernel<<<grid, 256, 0, st>>>(H, head->Bc, head->sBc, head->Bw, head->sBw,
-                                           s.r_c, s.r_r, s.N, s.D, s.g, t, img, nt, nkbt,
-                                           err);
+    if (img) {  // tcgen05 path: may start while the image kernel still runs
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = grid;
+      cfg.blockDim = dim3(256);
+      cfg.stream = st;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      cudaError_t e = cudaLaunchKernelEx(&cfg, lowrank_t_kernel, H, head->Bc, head->sBc,
+                                         head->Bw, head->sBw, s.r_c, s.r_r, s.N, s.D, s.g, t,
+                                         img, nt, nkbt, err);
+      if (e != cudaSuccess) return e;
+    } else {
+      lowrank_t_kernel<<<grid, 256, 0, st>>>(H, head->Bc, head->sBc, head->Bw, head->sBw,
+                                             s.r_c, s.r_r, s.N, s.D, s.g, t, img, nt, nkbt,
+                                             err);
+    }
     ++*launches;
   }
   return cudaGetLastError();

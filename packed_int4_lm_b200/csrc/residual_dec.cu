@@ -147,17 +147,17 @@ __device__ __forceinline__ bool dec_wait(uint64_t* bar, uint32_t parity, unsigne
 // two).  Each k-block sum then carries the constant 1032 sum_A b + 1152 sum_B b over the
 // stored values b, which corr holds and the kernel subtracts before scaling by the code.
 // Non-finite or out-of-range FP16 values set kErrRangeH.
-__global__ void __launch_bounds__(256) dec_convert_h_kernel(const uint16_t* __restrict__ H,
-                                                            __half* __restrict__ img,
-                                                            int64_t N, int ntok, int64_t D,
-                                                            int scale_b,
-                                                            unsigned* __restrict__ counters,
-                                                            int64_t n_counters,
-                                                            unsigned* err) {
+// Runs on blocks blk of nblk.
+__device__ __forceinline__ void dec_convert_h(const uint16_t* __restrict__ H,
+                                              __half* __restrict__ img, int64_t N, int ntok,
+                                              int64_t D, int scale_b,
+                                              unsigned* __restrict__ counters,
+                                              int64_t n_counters, unsigned* err, int64_t blk,
+                                              int64_t nblk) {
   const int64_t nkb = D / 128;
   const int lane = threadIdx.x & 31;
-  const int64_t gw = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
-  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int64_t gw = (blk * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = (nblk * (int64_t)blockDim.x) >> 5;
   float* corr = reinterpret_cast<float*>(img + (int64_t)ntok * D);  // [nkb][ntok]
   bool bad = false;
   for (int64_t wi = gw; wi < (int64_t)ntok * nkb; wi += nw) {
@@ -188,10 +188,80 @@ __global__ void __launch_bounds__(256) dec_convert_h_kernel(const uint16_t* __re
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     if (lane == 0) corr[kb * ntok + n] = scale_b ? sum : 0.f;
   }
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n_counters;
-       i += (int64_t)gridDim.x * blockDim.x)
+  for (int64_t i = blk * (int64_t)blockDim.x + threadIdx.x; i < n_counters;
+       i += nblk * (int64_t)blockDim.x)
     counters[i] = 0u;
   if (bad) atomicOr(err, kErrRangeH);
+}
+
+// t[n, j] = sum_d h[n, d] fl32(B[j, d] s[j, d / g]) for the N <= 16 tokens of this path,
+// B = [Q8(B_c) | Q8(B_w)]: one block per factor index j, 256 threads striding over D.
+__device__ __forceinline__ void dec_lowrank_t(const uint16_t* __restrict__ H,
+                                              const int8_t* __restrict__ Bc,
+                                              const float* __restrict__ sBc,
+                                              const int8_t* __restrict__ Bw,
+                                              const float* __restrict__ sBw, int r_c, int r_r,
+                                              int64_t N, int64_t D, int g, float* __restrict__ t,
+                                              int j) {
+  const int RR = r_c + r_r;
+  const int8_t* B = j < r_c ? Bc + (int64_t)j * D : Bw + (int64_t)(j - r_c) * D;
+  const float* sB = j < r_c ? sBc + (int64_t)j * (D / g) : sBw + (int64_t)(j - r_c) * (D / g);
+  float acc[16];
+#pragma unroll
+  for (int n = 0; n < 16; ++n) acc[n] = 0.f;
+  for (int64_t d0 = threadIdx.x * 8; d0 < D; d0 += 256 * 8) {
+    const uint2 braw = *reinterpret_cast<const uint2*>(B + d0);
+    const float sc = sB[d0 / g];
+    const int8_t* bq = reinterpret_cast<const int8_t*>(&braw);
+    float b[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) b[k] = __fmul_rn((float)bq[k], sc);
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+      if (n < N) {
+        const uint4 hv = *reinterpret_cast<const uint4*>(H + n * D + d0);
+        const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
+        float a = acc[n];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          a = fmaf(__uint_as_float(hw[k] << 16), b[2 * k], a);
+          a = fmaf(__uint_as_float(hw[k] & 0xFFFF0000u), b[2 * k + 1], a);
+        }
+        acc[n] = a;
+      }
+    }
+  }
+  __shared__ float red[8][16];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int n = 0; n < 16; ++n) {
+    float v = acc[n];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) red[warp][n] = v;
+  }
+  __syncthreads();
+  if ((int64_t)threadIdx.x < N) {
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) v += red[w][threadIdx.x];
+    t[(int64_t)threadIdx.x * RR + j] = v;
+  }
+}
+
+// The whole prologue of this path in one launch: blocks [0, nconv) build the H image, its
+// corrections and the zeroed counters; the next r_c + r_r blocks form t.
+__global__ void __launch_bounds__(256) dec_prologue_kernel(
+    const uint16_t* __restrict__ H, __half* __restrict__ img, int64_t N, int ntok, int64_t D,
+    int scale_b, unsigned* __restrict__ counters, int64_t n_counters, int nconv,
+    const int8_t* __restrict__ Bc, const float* __restrict__ sBc,
+    const int8_t* __restrict__ Bw, const float* __restrict__ sBw, int r_c, int r_r, int g,
+    float* __restrict__ t, unsigned* err) {
+  allow_dependent_launch();  // the main kernel may start streaming the packed head
+  if ((int)blockIdx.x < nconv)
+    dec_convert_h(H, img, N, ntok, D, scale_b, counters, n_counters, err, blockIdx.x, nconv);
+  else
+    dec_lowrank_t(H, Bc, sBc, Bw, sBw, r_c, r_r, N, D, g, t, (int)blockIdx.x - nconv);
 }
 
 constexpr int kDecMaxSP = 8;
@@ -213,7 +283,7 @@ __device__ __forceinline__ void mma_f16_16816_z(float d[4], const uint32_t a[4],
 }
 
 // Raw magic-number reads of the eight nibbles of a device-layout word (no FP16 math):
-// pairs 0 and 2 read 1032 + q, pairs 1 and 3 read 1152 + 16 q (see dec_convert_h_kernel).
+// pairs 0 and 2 read 1032 + q, pairs 1 and 3 read 1152 + 16 q (see dec_convert_h).
 __device__ __forceinline__ void nibble_reads(uint32_t w, uint32_t x[4]) {
   const uint32_t w2 = w >> 8;
   x[0] = and_xor(w, 0x000F000Fu, 0x64086408u);
@@ -335,14 +405,25 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
     if (lane == 0) {
       bool ok = true;
       const uint32_t hbytes = (uint32_t)(NTOK * D * 2 + (int64_t)nkb * NTOK * 4);
-      tc::mbar_arrive_expect_tx(h_full, hbytes);
-      tc::bulk_g2s(smem + m.h, p.Himg, hbytes, h_full);
+      // The H image comes from the prologue kernel, which may still be running (this
+      // kernel is a programmatic dependent launch): the packed stream starts at once, and
+      // the image is fetched after the prologue grid completes, before the first wait that
+      // needs consumers to make progress.
+      bool h_issued = false;
+      auto issue_h = [&]() {
+        if (h_issued) return;
+        h_issued = true;
+        grid_dependency_wait();
+        tc::mbar_arrive_expect_tx(h_full, hbytes);
+        tc::bulk_g2s(smem + m.h, p.Himg, hbytes, h_full);
+      };
       int k = 0, np = 0, nc = 0, s = 0;
       for (int64_t u = u0; ok && u < u1; ++s) {
         const int64_t T = u / nkb;
         const int kb0 = (int)(u - T * nkb);
         const int kb1 = (int)((int64_t)nkb < kb0 + (u1 - u) ? (int64_t)nkb : kb0 + (u1 - u));
         const int cs = s & 1;
+        if (s >= 2) issue_h();
         if (s >= 2 && !tc::mbar_wait(&c_empty[cs], ((s >> 1) - 1) & 1, p.err)) {
           ok = false;
           break;
@@ -361,6 +442,7 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
         for (int kb = kb0; kb < kb1; kb += 2, ++k) {
           const int st = k % SP;
           const uint32_t bytes = (uint32_t)(kb + 1 < kb1 ? 2 * kDecPk : kDecPk);
+          if (k >= SP) issue_h();
           if (k >= SP && !tc::mbar_wait(&p_empty[st], ((k / SP) - 1) & 1, p.err)) {
             ok = false;
             break;
@@ -373,6 +455,7 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
         }
         u += kb1 - kb0;
       }
+      issue_h();
       tc::mbar_wait(h_full, 0, p.err);
       if (!ok) {  // drain copies still in flight before the CTA exits
         for (int q = np - SP < 0 ? 0 : np - SP; q < np; ++q)
@@ -389,6 +472,7 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
   const int gid = lane >> 2, tq = lane & 3;
   const int par = warp / kDecRows;
   const int ctid = threadIdx.x;  // the first eight warps: 0 .. 255
+  grid_dependency_wait();  // t and the tile counters come from the prologue kernel
   bool ok = dec_wait(h_full, 0, p.err, true);
   for (int i = ctid; i < NTOK * RR; i += CONSUMERS * 32) {  // ts[j * NTOK + n]
     const int j = i / NTOK, n = i - j * NTOK;
@@ -743,8 +827,7 @@ cudaError_t launch_dec_cfg(const DecParams& p, int grid, cudaStream_t st) {
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   if (DecCfg<NT8>::PAR == 2 && p.sp % 2 != 0) return cudaErrorInvalidValue;
-  kern<<<(unsigned)grid, DecCfg<NT8>::THREADS, smem, st>>>(p);
-  return cudaGetLastError();
+  return launch_dependent(kern, grid, DecCfg<NT8>::THREADS, smem, st, p);
 }
 
 template <int NT8, int MODE>
@@ -800,18 +883,18 @@ cudaError_t launch_dec_prologue(const uint16_t* H, const archead_head* head, con
                                 unsigned* err, cudaStream_t st, int* launches) {
   const int64_t ntok = 8 * pl.nt8;
   const int64_t n_counters = (s.V + 127) / 128;
-  // one warp per (token, 128-column block); the counters ride on the same grid
+  // one warp per (token, 128-column block), the counters on the same blocks; then one
+  // block per factor index for t
   int64_t blocks = (ntok * (s.D / 128) * 32 + 255) / 256;
   const int64_t cb = (n_counters + 255) / 256;
   if (cb > blocks) blocks = cb;
   if (blocks > 148 * 8) blocks = 148 * 8;
-  dec_convert_h_kernel<<<(unsigned)blocks, 256, 0, st>>>(H, img, s.N, (int)ntok, s.D,
-                                                         s.g >= 128 ? 1 : 0, counters,
-                                                         n_counters, err);
+  const int RR = s.r_c + s.r_r;
+  dec_prologue_kernel<<<(unsigned)(blocks + RR), 256, 0, st>>>(
+      H, img, s.N, (int)ntok, s.D, s.g >= 128 ? 1 : 0, counters, n_counters, (int)blocks,
+      head->Bc, head->sBc, head->Bw, head->sBw, s.r_c, s.r_r, s.g, t, err);
   ++*launches;
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  return launch_lowrank_t(H, head, s, t, nullptr, 0, 0, err, st, launches);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_residual_dec(const __half* img, const float* t, const archead_head* head,

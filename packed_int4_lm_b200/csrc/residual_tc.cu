@@ -284,6 +284,9 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
           tc::mbar_wait(&c_full[q & 1], (q >> 1) & 1, p.err);
       }
     } else if (lane == 1) {
+      // the B image comes from the prologue kernels: this kernel is a programmatic
+      // dependent launch, so the packed stream (lane 0) starts while they finish
+      grid_dependency_wait();
       int k = 0, nb = 0;
       bool ok = true;
       Item it;
@@ -572,6 +575,7 @@ __global__ void __launch_bounds__(256) convert_h_blocked_kernel(const uint16_t* 
                                                                 int64_t N, int64_t Npad,
                                                                 int64_t D, int64_t nkbt, int nt,
                                                                 unsigned* err) {
+  allow_dependent_launch();
   const int64_t chunks_per_row = nkbt * 16;  // 8 FP16 per chunk
   const int64_t total = Npad * chunks_per_row;
   const int64_t hchunks = D / 8;
@@ -637,8 +641,7 @@ cudaError_t launch_tc_cfg(const TcParams& p, cudaStream_t st) {
   int64_t items = p.n_vtiles * p.n_tok_tiles;
   int64_t grid = (int64_t)sms * occ;
   if (grid > items) grid = items;
-  kern<<<(unsigned)grid, kTcThreads, smem, st>>>(p);
-  return cudaGetLastError();
+  return launch_dependent(kern, grid, kTcThreads, smem, st, p);
 }
 
 template <int NT, int MODE>

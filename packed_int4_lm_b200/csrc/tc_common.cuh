@@ -194,4 +194,36 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 }
 
 }  // namespace tc
+
+// ---- programmatic dependent launch ------------------------------------------------------
+// A kernel launched with launch_dependent may start while the previous kernel in the
+// stream still runs.  Before touching that kernel's outputs it calls grid_dependency_wait,
+// which returns once the previous grid has completed and its writes are visible (at once
+// for an ordinary launch).  The previous kernel calls allow_dependent_launch early so the
+// dependent grid can be scheduled while it runs; the dependent launches only after every
+// block of the previous grid has made that call or exited, so both are resident together
+// and neither waits on a grid that cannot be scheduled.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+}
+__device__ __forceinline__ void allow_dependent_launch() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
+template <typename Kern, typename Params>
+cudaError_t launch_dependent(Kern kern, int64_t grid, int threads, size_t smem,
+                             cudaStream_t st, const Params& p) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3((unsigned)threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
 }  // namespace archead

@@ -181,15 +181,18 @@ def test_host_entry_points_match_device(dev, rhead):
 
 
 def test_launch_counts(dev, rhead):
-    """Kernels per call: logits = FP16 H (row-major or blocked), t, contraction;
-    NLL = FP16 H, t, contraction, combine."""
+    """Kernels per call.  N <= 16 (decode kernel): one prologue (H image, corrections and t)
+    and the contraction, plus the combine for NLL.  Larger N (tcgen05 kernel): blocked H,
+    the rank pieces of t, the contraction."""
     head, dh = rhead
     H = _rand_H(4, 512, 1).to(dev)
     ah.logits(H, dh)
-    assert ah.last_launches() == 3
+    assert ah.last_launches() == 2
     ah.logits(_rand_H(40, 512, 2).to(dev), dh)
     assert ah.last_launches() == 3
     ah.nll(H, dh, make_targets(4, head["V"], 1).to(dev))
+    assert ah.last_launches() == 3
+    ah.nll(_rand_H(40, 512, 3).to(dev), dh, make_targets(40, head["V"], 2).to(dev))
     assert ah.last_launches() == 4
     torch.cuda.synchronize()
 
