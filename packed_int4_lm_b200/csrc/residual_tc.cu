@@ -65,6 +65,7 @@ struct TcParams {
   int a_words;     // factor rows readable as aligned 32-bit words
   int sb;          // B ring stages (<= kMaxSB)
   int n_tok_tiles;
+  int tt_band;  // token tiles per band (their B image stays in L2 while the head streams)
   int64_t n_vtiles;
   unsigned* err;
 };
@@ -109,10 +110,18 @@ __device__ __forceinline__ bool get_item(const TcParams& p, int k, Item& it) {
     if (it.vt >= t1) return false;
     it.tt = 0;
   } else {
+    // bands of tt_band token tiles; inside a band the token tile varies fastest, so CTAs
+    // reading the same vocabulary rows run together and the band's B image is reused
+    // from L2 across all vocabulary tiles
     const int64_t gi = blockIdx.x + (int64_t)k * gridDim.x;
     if (gi >= p.n_vtiles * p.n_tok_tiles) return false;
-    it.vt = gi / p.n_tok_tiles;
-    it.tt = (int)(gi - it.vt * p.n_tok_tiles);
+    const int64_t band_items = p.n_vtiles * p.tt_band;
+    const int64_t band = gi / band_items;
+    const int64_t local = gi - band * band_items;
+    const int64_t tt0 = band * p.tt_band;
+    const int64_t nb = p.n_tok_tiles - tt0 < p.tt_band ? p.n_tok_tiles - tt0 : p.tt_band;
+    it.vt = local / nb;
+    it.tt = (int)(tt0 + (local - it.vt * nb));
   }
   it.row0 = it.vt * 128;
   it.row_end = it.row0 + 128 < p.V ? it.row0 + 128 : p.V;
@@ -745,6 +754,14 @@ cudaError_t launch_residual_tc(const __half* Hb, const archead_head* head, const
   p.sb = plan.sb;
   p.err = err;
   p.n_tok_tiles = (int)((s.N + plan.nt - 1) / plan.nt);
+  {
+    // a band's B image within about 48 MB, well inside the 126 MB L2
+    const int64_t tile_bytes = (int64_t)plan.nt * (s.D + 128 * plan.nrb) * 2;
+    int64_t band = (48ll << 20) / tile_bytes;
+    if (band < 1) band = 1;
+    if (band > p.n_tok_tiles) band = p.n_tok_tiles;
+    p.tt_band = (int)band;
+  }
   p.n_vtiles = (s.V + 127) / 128;
   if (plan.nt == 0 || plan.sb < 2 || plan.sb > kMaxSB) return cudaErrorInvalidValue;
   cudaError_t e = Y ? launch_tc_mode<0>(p, plan.nt, s.g, st)
