@@ -255,35 +255,79 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
   const uint32_t acol = tbase + 2 * NT;  // A ring after the two accumulators (lane 0)
 
   if (warp == 8) {
-    // ---------------- producers: lane 0 codes + packed blocks, lane 1 B blocks ----------
-    // Two independent streams, so the packed prefetch is not held back by the B ring
-    // (whose stages free up only as MMAs retire).
+    // ---------------- producer: one thread, two streams ----------------
+    // The packed stream (group codes once per item, then the packed blocks) and the B
+    // stream (the token tile's image blocks) are polled without blocking, and whichever
+    // ring has a free stage is refilled, so neither waits behind the other (as two lanes of
+    // one warp, a lane blocked on its full ring held the other's refills back).  The B
+    // image comes from the prologue kernels (this kernel is a programmatic dependent
+    // launch): the B stream starts once the packed ring is full.  No progress for about a
+    // second sets the device error word; the copies in flight are then drained.
     if (lane == 0) {
-      int k = 0, np = 0, nc = 0;
-      bool ok = true;
-      Item it;
-      for (int i = 0; ok && get_item(p, i, it); ++i) {
-        const int cs = i & 1;
-        if (i >= 2 && !tc::mbar_wait(&c_empty[cs], ((i >> 1) - 1) & 1, p.err)) {
-          ok = false;
-          break;
-        }
-        tc::fence_proxy_async_smem();  // the stage was read with generic loads
-        tc::mbar_arrive_expect_tx(&c_full[cs], (uint32_t)code_bytes);
-        tc::bulk_g2s(cds + cs * round16(code_bytes), p.code + it.row0 * G, (uint32_t)code_bytes,
-                     &c_full[cs]);
-        ++nc;
-        const uint8_t* psrc = p.nib + ((it.vt * nkb) << 13);
-        for (int kb = 0; kb < nkb; ++kb, ++k) {
-          const int sp = k % C::SP;
-          if (k >= C::SP && !tc::mbar_wait(&p_empty[sp], ((k / C::SP) - 1) & 1, p.err)) {
-            ok = false;
-            break;
+      Item pit, hit;
+      bool p_have = get_item(p, 0, pit), h_have = get_item(p, 0, hit);
+      int ip = 0, pkb = -1, kpk = 0, np = 0, nc = 0;  // pkb = -1: the item's codes are next
+      int ih = 0, hkb = 0, kh = 0, nb = 0;
+      bool h_started = false, ok = true;
+      long long idle0 = clock64();
+      while (ok && (p_have || h_have)) {
+        bool progress = false;
+        if (p_have) {
+          if (pkb < 0) {
+            const int cs = ip & 1;
+            if (ip < 2 || tc::mbar_test(&c_empty[cs], ((ip >> 1) - 1) & 1)) {
+              tc::fence_proxy_async_smem();  // the slot was read with generic loads
+              tc::mbar_arrive_expect_tx(&c_full[cs], (uint32_t)code_bytes);
+              tc::bulk_g2s(cds + cs * round16(code_bytes), p.code + pit.row0 * G,
+                           (uint32_t)code_bytes, &c_full[cs]);
+              ++nc;
+              pkb = 0;
+              progress = true;
+            }
+          } else {
+            const int sp = kpk % C::SP;
+            if (kpk < C::SP || tc::mbar_test(&p_empty[sp], ((kpk / C::SP) - 1) & 1)) {
+              tc::fence_proxy_async_smem();  // the stage was read with generic loads
+              tc::mbar_arrive_expect_tx(&p_full[sp], kPkBytes);
+              tc::bulk_g2s(pk + sp * kPkBytes, p.nib + ((pit.vt * nkb + pkb) << 13), kPkBytes,
+                           &p_full[sp]);
+              ++np;
+              ++kpk;
+              progress = true;
+              if (++pkb == nkb) {
+                ++ip;
+                pkb = -1;
+                p_have = get_item(p, ip, pit);
+              }
+            }
           }
-          tc::fence_proxy_async_smem();  // the stage was read with generic loads
-          tc::mbar_arrive_expect_tx(&p_full[sp], kPkBytes);
-          tc::bulk_g2s(pk + sp * kPkBytes, psrc + ((int64_t)kb << 13), kPkBytes, &p_full[sp]);
-          ++np;
+        }
+        if (h_have && (h_started || !p_have || kpk >= C::SP)) {
+          if (!h_started) {
+            grid_dependency_wait();
+            h_started = true;
+          }
+          const int sb = kh % SB;
+          if (kh < SB || tc::mbar_test(&b_empty[sb], ((kh / SB) - 1) & 1)) {
+            const unsigned char* hsrc = reinterpret_cast<const unsigned char*>(p.Hb) +
+                                        ((int64_t)hit.tt * nkbt + hkb) * C::HSTAGE;
+            tc::mbar_arrive_expect_tx(&b_full[sb], C::HSTAGE);
+            tc::bulk_g2s(Hs + sb * C::HSTAGE, hsrc, C::HSTAGE, &b_full[sb]);
+            ++nb;
+            ++kh;
+            progress = true;
+            if (++hkb == nkbt) {
+              ++ih;
+              hkb = 0;
+              h_have = get_item(p, ih, hit);
+            }
+          }
+        }
+        if (progress) {
+          idle0 = clock64();
+        } else if (clock64() - idle0 > (1ll << 31)) {
+          atomicOr(p.err, kErrTimeout);
+          ok = false;
         }
       }
       if (!ok) {  // drain copies still in flight before the CTA exits
@@ -291,29 +335,6 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
           tc::mbar_wait(&p_full[q % C::SP], (q / C::SP) & 1, p.err);
         for (int q = nc - 2 < 0 ? 0 : nc - 2; q < nc; ++q)
           tc::mbar_wait(&c_full[q & 1], (q >> 1) & 1, p.err);
-      }
-    } else if (lane == 1) {
-      // the B image comes from the prologue kernels: this kernel is a programmatic
-      // dependent launch, so the packed stream (lane 0) starts while they finish
-      grid_dependency_wait();
-      int k = 0, nb = 0;
-      bool ok = true;
-      Item it;
-      for (int i = 0; ok && get_item(p, i, it); ++i) {
-        const unsigned char* hsrc =
-            reinterpret_cast<const unsigned char*>(p.Hb) + (int64_t)it.tt * nkbt * C::HSTAGE;
-        for (int kb = 0; kb < nkbt; ++kb, ++k) {
-          const int sb = k % SB;
-          if (k >= SB && !tc::mbar_wait(&b_empty[sb], ((k / SB) - 1) & 1, p.err)) {
-            ok = false;
-            break;
-          }
-          tc::mbar_arrive_expect_tx(&b_full[sb], C::HSTAGE);
-          tc::bulk_g2s(Hs + sb * C::HSTAGE, hsrc + (int64_t)kb * C::HSTAGE, C::HSTAGE, &b_full[sb]);
-          ++nb;
-        }
-      }
-      if (!ok) {
         for (int q = nb - SB < 0 ? 0 : nb - SB; q < nb; ++q)
           tc::mbar_wait(&b_full[q % SB], (q / SB) & 1, p.err);
       }
