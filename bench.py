@@ -152,15 +152,53 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------------------
-def build_head(w, device):
+def build_head(w, device, keep_dense=False):
+    """The packed head of workload w (and, with keep_dense, the dense head as BF16 for the
+    quality comparison of the fused-NLL workload)."""
     from packed_int4_lm_b200 import pack
     W = make_weight(w.V, w.D, w.rank, w.sigma0, w.noise, w.seed_w, device=device)
     s = make_channel_scales(w.D, w.sigma_s, w.n_outliers, w.outlier_mult, w.seed_scales)
     Hc = make_hidden(w.n_cal, s, w.seed_hcal).to(device)
     head = pack.build_head(W, Hc, w.r_c, w.r_r, w.g, w.p, w.lam, seed=w.seed_rsvd)
+    Wb = W.to(torch.bfloat16) if keep_dense else None
     del W, Hc
     torch.cuda.empty_cache()
-    return head, s
+    return (head, s, Wb) if keep_dense else (head, s)
+
+
+def nll_quality(head, Wb, Hcpu, tg, ours, sample=16):
+    """Quality context for the fused-NLL workload: mean NLL of the packed head (the timed
+    path's output), of the dense head in BF16 on the same tokens (torch.matmul +
+    cross_entropy, a comparator only), and of the fp64 oracle on the first `sample` tokens
+    next to the packed head's values for them."""
+    import oracle
+    dev = Wb.device
+    H = Hcpu.to(dev)
+    tgt = tg.to(dev).long()
+    dense = []
+    for i in range(0, H.shape[0], 512):
+        logits = torch.matmul(H[i:i + 512], Wb.t()).float()
+        dense.append(torch.nn.functional.cross_entropy(logits, tgt[i:i + 512], reduction="none"))
+    dense = torch.cat(dense)
+    ref = oracle.nll(head, bf16_bits(Hcpu[:sample]), tg[:sample].numpy())
+    mine = ours[:sample].double().cpu().numpy()
+    return {"mean_nll_packed": float(ours.double().mean()),
+            "mean_nll_dense_bf16": float(dense.double().mean()),
+            "oracle_sample_tokens": sample,
+            "mean_nll_oracle_sample": float(np.mean(ref)),
+            "mean_nll_packed_sample": float(np.mean(mine)),
+            "max_abs_nll_diff_vs_oracle": float(np.max(np.abs(mine - ref)))}
+
+
+def job_throughput(local_ms, tokens_per_rank, world, device):
+    """Whole-job tokens/s of `world` ranks that each ran the same steps: the job takes as long
+    as its slowest rank, so the local device times are reduced with MAX.  Returns
+    (tokens/s, job ms)."""
+    t = torch.tensor([float(local_ms)], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms = float(t.item())
+    return tokens_per_rank * world / (ms / 1e3), ms
 
 
 def main_kernel_bytes(head, N):
@@ -258,7 +296,11 @@ def main():
             device_id=torch.device("cuda", local))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    head, s = build_head(w, dev)
+    Wb = None
+    if nll_mode and rank == 0:
+        head, s, Wb = build_head(w, dev, keep_dense=True)
+    else:
+        head, s = build_head(w, dev)
     dh = ah.DeviceHead.from_canonical(head, dev)
     # each rank evaluates its own tokens
     Hcpu = {N: make_hidden(N, s, w.seed_heval + 7919 * rank) for N in Ns}
@@ -312,12 +354,7 @@ def main():
     ah.profile(False)
     ah.check()
     main_ms, main_n = ah.profile_read()
-    t = torch.tensor([elapsed_ms], device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    elapsed_ms = float(t.item())
-    tokens = sum(Ns) * K * world
-    value = tokens / (elapsed_ms / 1e3)
+    value, elapsed_ms = job_throughput(elapsed_ms, sum(Ns) * K, world, dev)
     peaks = load_peaks()
 
     # roofline of the residual kernel over the timed launches
@@ -398,12 +435,18 @@ def main():
     g1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    te = torch.tensor([g0.elapsed_time(g1)], device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
-    e2e_value = sum(Ns) * KE * world / (float(te.item()) / 1e3)
+    e2e_value, _ = job_throughput(g0.elapsed_time(g1), sum(Ns) * KE, world, dev)
     h2d = sum(N * w.D * 2 + (4 * N if nll_mode else 0) for N in Ns)
     d2h = sum(4 * N if nll_mode else 4 * N * w.V for N in Ns)
+
+    quality = None
+    if nll_mode and rank == 0:
+        Nq = Ns[0]
+        ah.nll(H[Nq], dh, tgd[Nq], out=out[Nq])
+        torch.cuda.synchronize()
+        quality = nll_quality(head, Wb, Hcpu[Nq], tg[Nq], out[Nq].clone())
+        del Wb
+        torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
@@ -429,6 +472,8 @@ def main():
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": KE},
             "gpu_launches": launches, "clocks": ck, "per_n": per_n}
+    if quality is not None:
+        line["quality"] = quality
     print(json.dumps(line), flush=True)
 
 

@@ -113,6 +113,21 @@ def test_logits_extreme_scale_ratios(dev, sup_exp, fac_exp):
         _assert_logits(Y.cpu().numpy(), oracle.logits(head, bf16_bits(H)), f"{sup_exp} {N}")
 
 
+@pytest.mark.parametrize("g,N,launches", [(128, 3, 3), (128, 12, 3), (128, 100, 3), (32, 12, 3)])
+def test_fallback_kernels_for_wide_rows(dev, g, N, launches):
+    """D = 16384: the decode kernel's resident H does not fit shared memory, so N <= 8 runs
+    on the token-block warp-MMA kernel; with g = 32 the tcgen05 kernel's code ring does not
+    fit either and N = 12 also takes the warp-MMA kernel (three launches each path)."""
+    V, D = 300, 16384
+    head = random_canonical_head(V, D, 8, 8, g, seed=N + g, zero_rows=2)
+    dh = ah.DeviceHead.from_canonical(head, dev)
+    H = _rand_H(N, D, 900 + N)
+    Y = ah.logits(H.to(dev), dh)
+    ah.check()
+    assert ah.last_launches() == launches
+    _assert_logits(Y.cpu().numpy(), oracle.logits(head, bf16_bits(H)), f"D={D} g={g} N={N}")
+
+
 @pytest.fixture(scope="module")
 def nhead(dev):
     """Random packed bytes scaled so that rms(Y) is a few units, the regime of language-model

@@ -204,3 +204,48 @@ def test_int8_dequant_is_single_precision_product():
     ref = torch.tensor(q, dtype=torch.float32) * torch.tensor(s)[:, None]
     assert np.array_equal(out, ref.double().numpy())
     assert out[0, 0] != 127 * 0.1  # not the exact real product
+
+
+def test_brute_force_loops_on_a_tiny_head():
+    """The oracle against explicit scalar loops over the canonical bytes (V=8, D=128, g=64,
+    N=3, r_c=r_r=2): each logit is sum_d h_d (q c S + sum_j Ac Bc + sum_j Aw Bw), every
+    factor entry the single-precision product of its INT8 value and scale (ARCHead Sec. 3,
+    the packed head and the logit formula)."""
+    import struct
+
+    V, D, g, N, rc, rr = 8, 128, 64, 3, 2, 2
+    head = random_canonical_head(V, D, rc, rr, g, seed=99, zero_rows=1, zero_groups=1)
+    rng = np.random.default_rng(7)
+    Hf = rng.standard_normal((N, D)).astype(np.float32)
+    Hb = (Hf.view(np.uint32) >> 16).astype(np.uint16)  # truncate to BF16 bit patterns
+
+    def bf16(b):
+        return struct.unpack("<f", struct.pack("<I", int(b) << 16))[0]
+
+    def f32(x):
+        return struct.unpack("<f", struct.pack("<f", x))[0]
+
+    def int4(v, d):
+        byte = int(head["r_nib"][v, d // 2])
+        nib = (byte >> (4 * (d % 2))) & 0xF
+        return nib - 16 if nib >= 8 else nib
+
+    def factor(a, s):  # one IEEE-single product
+        return f32(float(a) * float(s))
+
+    Y = np.zeros((N, V))
+    for n in range(N):
+        for v in range(V):
+            acc = 0.0
+            for d in range(D):
+                w = float(int4(v, d)) * float(head["r_code"][v, d // g]) * bf16(head["r_super"][v])
+                for j in range(rc):
+                    w += factor(head["Ac"][v, j], head["sAc"][v]) * \
+                        factor(head["Bc"][j, d], head["sBc"][j, d // g])
+                for j in range(rr):
+                    w += factor(head["Aw"][v, j], head["sAw"][v]) * \
+                        factor(head["Bw"][j, d], head["sBw"][j, d // g])
+                acc += bf16(Hb[n, d]) * w
+            Y[n, v] = acc
+    Yo = oracle.logits(head, Hb)
+    assert np.max(np.abs(Yo - Y)) <= 1e-12 * max(1.0, np.max(np.abs(Y)))
