@@ -22,15 +22,20 @@
  *    detected on the host before anything is enqueued.  Errors detected by a kernel
  *    (ARCHEAD_ERR_RANGE_H, ARCHEAD_ERR_TARGET) set a per-device error word; the affected
  *    outputs are non-finite; archead_check() reports and clears the word.
- *  - Temporary device memory (the N x (r_c + r_r) prologue product t, the FP16 copy of H,
- *    the NLL partials) is taken with cudaMallocAsync from a library-owned pool on
- *    `stream` and returned with cudaFreeAsync on the same stream.
+ *  - Temporary device memory (the N x (r_c + r_r) prologue product t, the FP16 image of H,
+ *    the split-tile partials and counters, the NLL partials) is taken with
+ *    cudaMallocAsync from a library-owned pool on `stream` and returned with
+ *    cudaFreeAsync on the same stream.
  *  - Limits: g in {32, 64, 128, 256}; D % 128 == 0 and D % g == 0; 0 <= r_c, r_r <= 128;
  *    1 <= V <= 8388480 (65535 blocks of 128 rows); 0 <= N < 2^31; N == 0 is a successful
  *    no-op.  V needs no multiple of
  *    any tile: the vocabulary tail is predicated.
  *  - |H| must stay within the FP16 range (|h| <= 65504); larger or non-finite entries
- *    raise ARCHEAD_ERR_RANGE_H (see archead_logits).
+ *    raise ARCHEAD_ERR_RANGE_H (see archead_logits).  Where the rank terms run on the
+ *    tensor cores (r_c and r_r multiples of 16 for N <= 16; every shape for N > 16) the
+ *    same holds for the prologue products t = H [Q8(B_c) | Q8(B_w)]^T, and with one group
+ *    code per 128 columns (g >= 128, N <= 16) for H / 16 on half of the columns (values
+ *    below the FP16 normal range lose bits, like H's own FP16 rounding).
  */
 #ifndef ARCHEAD_H_
 #define ARCHEAD_H_
@@ -94,10 +99,16 @@ typedef struct archead_head {
  * archead_logits -- Y = H W_d^T + (H B_w^T) A_w^T   (ARCHead Sec. 3, logit formula).
  *   H  bf16 N x D (device), Y float N x V (device, fully overwritten).
  *   N, V, D, r_c, r_r, g must equal the head's metadata (ARCHEAD_ERR_SHAPE otherwise).
- *   N <= 64 runs the memory-bound decode kernel (each packed byte read once per call);
- *   larger N runs the dense-contraction kernel.  Asynchronous on `stream`.
- *   Precision: residual operands q*c are exact in FP16, H is rounded to FP16, products
- *   accumulate in FP32; the low-rank terms run in FP32.
+ *   N <= 16 runs the persistent decode kernel (warp MMAs; each packed byte read once per
+ *   call), larger N the tcgen05 kernel (tensor-memory accumulators); shapes whose shared-
+ *   memory plans do not fit take a token-block warp-MMA kernel.  The main kernel starts
+ *   while the prologue still runs (programmatic dependent launch).  Asynchronous on
+ *   `stream`.
+ *   Precision: H is rounded to FP16 and products accumulate in FP32.  Residual operands:
+ *   exact q*c*2^-k in FP16 (N > 16), or raw nibble reads with a per-block offset
+ *   correction and the group code applied to the FP32 block sum (N <= 16, g >= 128),
+ *   else exact q*c.  Low-rank terms: FP32 (r not a multiple of 16, N <= 16) or FP16
+ *   hi/lo pieces of the factor entries and of t on the tensor cores (about 22 bits).
  */
 int archead_logits(const uint16_t* H, const archead_head* head, float* Y, int64_t N,
                    int64_t V, int64_t D, int r_c, int r_r, int g, void* stream);
