@@ -33,9 +33,10 @@
  *  - |H| must stay within the FP16 range (|h| <= 65504); larger or non-finite entries
  *    raise ARCHEAD_ERR_RANGE_H (see archead_logits).  Where the rank terms run on the
  *    tensor cores (r_c and r_r multiples of 16 for N <= 16; every shape for N > 16) the
- *    same holds for the prologue products t = H [Q8(B_c) | Q8(B_w)]^T, and with one group
- *    code per 128 columns (g >= 128, N <= 16) for H / 16 on half of the columns (values
- *    below the FP16 normal range lose bits, like H's own FP16 rounding).
+ *    same holds for the prologue products t = H [Q8(B_c) | Q8(B_w)]^T.  With one group code
+ *    per 128 columns (g >= 128, N <= 16) half of the columns of H are stored as H / 16;
+ *    such values that fall below the FP16 normal range keep fewer bits, as H's own
+ *    rounding to FP16 does.
  */
 #ifndef ARCHEAD_H_
 #define ARCHEAD_H_
