@@ -165,7 +165,7 @@ int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* ta
   // N <= 16: the persistent decode kernel with H resident in shared memory, when it fits
   const DecPlan dplan = dec_plan(s, nll_mode);
   if (dplan.nt8 > 0) return run_dec(H, head, Y, targets, nll, s, dplan, ds, st);
-  const TcPlan plan = s.N > 8 ? tc_plan(s, nll_mode) : TcPlan{0, 0, 0};
+  const TcPlan plan = s.N > 8 ? tc_plan(s, nll_mode) : TcPlan{0, 0, 0, 0};
   const bool use_tc = plan.nt > 0;
   const int64_t tb = use_tc ? plan.nt : residual_token_block(s.N);
   const int64_t Npad = (s.N + tb - 1) / tb * tb;

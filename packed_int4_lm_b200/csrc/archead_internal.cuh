@@ -175,6 +175,7 @@ struct TcPlan {
   int nt;   // token tile: 16, 32, 64 or 128 (0: the shape does not fit this kernel)
   int sb;   // stages of the shared-memory ring of B blocks
   int nrb;  // rank blocks after the nkb blocks of H
+  int sp;   // stages of the shared-memory ring of packed blocks
 };
 TcPlan tc_plan(const Shapes& s, bool nll);
 // FP16 element offset of (token nn of token tile tt, column kk < 128 of block kb) in the

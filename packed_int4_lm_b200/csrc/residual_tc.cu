@@ -44,6 +44,7 @@ namespace {
 constexpr int kTcThreads = 320;  // warps 0-3 dequant, 4-7 epilogue, 8 producer, 9 MMA
 constexpr int kPkBytes = 8192;   // packed block of one 128-row tile (128 columns)
 constexpr int kMaxSB = 8;        // deepest B ring
+constexpr int kMaxSP = 8;        // deepest packed ring
 
 struct TcParams {
   const __half* Hb;  // B image: [token tile][nkb + nrb blocks][NT x 128]
@@ -64,6 +65,7 @@ struct TcParams {
   int rank_steps;  // K=16 steps holding rank columns: ceil(4 (r_c + r_r) / 16)
   int a_words;     // factor rows readable as aligned 32-bit words
   int sb;          // B ring stages (<= kMaxSB)
+  int spk;         // packed ring stages (<= kMaxSP)
   int n_tok_tiles;
   int tt_band;  // token tiles per band (their B image stays in L2 while the head streams)
   int64_t n_vtiles;
@@ -72,12 +74,18 @@ struct TcParams {
 
 template <int NT>
 struct TcCfg {
-  static constexpr int SP = NT <= 32 ? 6 : 4;  // packed ring stages
   static constexpr int HSTAGE = NT * 256;      // bytes of one 128-column B block
-  static constexpr int TMEM_COLS = NT <= 64 ? 256 : 512;
-  // A-ring stages (64 columns each) in what the two accumulators leave, at most 4
-  static constexpr int SA = (TMEM_COLS - 2 * NT) / 64 < 4 ? (TMEM_COLS - 2 * NT) / 64 : 4;
-  static_assert(SA >= 2 && 2 * NT + 64 * SA <= TMEM_COLS, "tensor memory budget");
+  // Two CTAs per SM (256 TMEM columns each) for every tile: a single MMA issuer per SM
+  // sustains only about one 8-MMA stage per ~950 cycles (stage handshakes ride on commit
+  // and mbarrier latencies), two issuers fill each other's gaps.  The 128-token tile then
+  // keeps one accumulator (the next item's MMAs wait for the epilogue while the other CTA
+  // uses the tensor core); smaller tiles double-buffer it.
+  static constexpr int TMEM_COLS = 256;
+  static constexpr int NACC = NT == 128 ? 1 : 2;
+  // A-ring stages (64 columns each) in what the accumulators leave, at most 4
+  static constexpr int SA =
+      (TMEM_COLS - NACC * NT) / 64 < 4 ? (TMEM_COLS - NACC * NT) / 64 : 4;
+  static_assert(SA >= 2 && NACC * NT + 64 * SA <= TMEM_COLS, "tensor memory budget");
   static_assert(NT % 16 == 0 && NT >= 16 && NT <= 256, "M=128 MMA needs N in 16..256");
 };
 
@@ -90,9 +98,9 @@ constexpr size_t nll_scratch_bytes() {
 }
 
 template <int NT>
-size_t tc_smem_bytes(int sb, int G, bool nll) {
+size_t tc_smem_bytes(int sb, int sp, int G, bool nll) {
   using C = TcCfg<NT>;
-  return (size_t)sb * C::HSTAGE + (size_t)C::SP * kPkBytes + 2 * round16((size_t)128 * G) +
+  return (size_t)sb * C::HSTAGE + (size_t)sp * kPkBytes + 2 * round16((size_t)128 * G) +
          (nll ? nll_scratch_bytes<NT>() : 0) + 512;
 }
 
@@ -204,7 +212,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
   const int SB = p.sb;
   unsigned char* Hs = smem;
   unsigned char* pk = Hs + SB * C::HSTAGE;
-  unsigned char* cds = pk + C::SP * kPkBytes;  // [2][128 x G]
+  const int SPK = p.spk;
+  unsigned char* cds = pk + SPK * kPkBytes;  // [2][128 x G]
   unsigned char* after_codes = cds + 2 * round16(code_bytes);
   float* nll_y = reinterpret_cast<float*>(after_codes);  // [16][128]
   int32_t* tgt_s = reinterpret_cast<int32_t*>(nll_y + 16 * 128);  // [NT]
@@ -213,8 +222,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
   uint64_t* b_full = bars;
   uint64_t* b_empty = b_full + kMaxSB;
   uint64_t* p_full = b_empty + kMaxSB;
-  uint64_t* p_empty = p_full + C::SP;
-  uint64_t* c_full = p_empty + C::SP;   // [2]
+  uint64_t* p_empty = p_full + kMaxSP;
+  uint64_t* c_full = p_empty + kMaxSP;  // [2]
   uint64_t* c_empty = c_full + 2;       // [2]
   uint64_t* a_full = c_empty + 2;
   uint64_t* a_empty = a_full + C::SA;
@@ -230,7 +239,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
       tc::mbar_init(&b_full[s], 1);
       tc::mbar_init(&b_empty[s], 1);
     }
-    for (int s = 0; s < C::SP; ++s) {
+    for (int s = 0; s < SPK; ++s) {
       tc::mbar_init(&p_full[s], 1);
       tc::mbar_init(&p_empty[s], 4);  // one arrival per dequant warp
     }
@@ -252,7 +261,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tbase = *tmem_slot;
-  const uint32_t acol = tbase + 2 * NT;  // A ring after the two accumulators (lane 0)
+  const uint32_t acol = tbase + C::NACC * NT;  // A ring after the accumulators (lane 0)
 
   if (warp == 8) {
     // ---------------- producer: one thread, two streams ----------------
@@ -285,8 +294,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
               progress = true;
             }
           } else {
-            const int sp = kpk % C::SP;
-            if (kpk < C::SP || tc::mbar_test(&p_empty[sp], ((kpk / C::SP) - 1) & 1)) {
+            const int sp = kpk % SPK;
+            if (kpk < SPK || tc::mbar_test(&p_empty[sp], ((kpk / SPK) - 1) & 1)) {
               tc::fence_proxy_async_smem();  // the stage was read with generic loads
               tc::mbar_arrive_expect_tx(&p_full[sp], kPkBytes);
               tc::bulk_g2s(pk + sp * kPkBytes, p.nib + ((pit.vt * nkb + pkb) << 13), kPkBytes,
@@ -302,7 +311,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
             }
           }
         }
-        if (h_have && (h_started || !p_have || kpk >= C::SP)) {
+        if (h_have && (h_started || !p_have || kpk >= SPK)) {
           if (!h_started) {
             grid_dependency_wait();
             h_started = true;
@@ -331,8 +340,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
         }
       }
       if (!ok) {  // drain copies still in flight before the CTA exits
-        for (int q = np - C::SP < 0 ? 0 : np - C::SP; q < np; ++q)
-          tc::mbar_wait(&p_full[q % C::SP], (q / C::SP) & 1, p.err);
+        for (int q = np - SPK < 0 ? 0 : np - SPK; q < np; ++q)
+          tc::mbar_wait(&p_full[q % SPK], (q / SPK) & 1, p.err);
         for (int q = nc - 2 < 0 ? 0 : nc - 2; q < nc; ++q)
           tc::mbar_wait(&c_full[q & 1], (q >> 1) & 1, p.err);
         for (int q = nb - SB < 0 ? 0 : nb - SB; q < nb; ++q)
@@ -347,8 +356,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
       bool ok = true;
       Item it;
       for (int i = 0; ok && get_item(p, i, it); ++i) {
-        const int ab = i & 1;
-        if (i >= 2 && !tc::mbar_wait(&acc_empty[ab], ((i >> 1) - 1) & 1, p.err)) break;
+        const int ab = i % C::NACC, use = i / C::NACC;
+        if (i >= C::NACC && !tc::mbar_wait(&acc_empty[ab], (use - 1) & 1, p.err)) break;
         tc::fence_after_sync();
         const uint32_t dcol = tbase + ab * NT;
         for (int kb = 0; kb < nkbt; ++kb, ++k) {
@@ -411,8 +420,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
       }
       const unsigned char* crow = cds + cs * round16(code_bytes) + tid * G;
       for (int kb = 0; kb < nkb; ++kb, ++k, ++kp) {
-        const int sp = kp % C::SP, sa = k % C::SA;
-        if (!__all_sync(0xffffffffu, tc::mbar_wait(&p_full[sp], (kp / C::SP) & 1, p.err))) {
+        const int sp = kp % SPK, sa = k % C::SA;
+        if (!__all_sync(0xffffffffu, tc::mbar_wait(&p_full[sp], (kp / SPK) & 1, p.err))) {
           ok = false;
           break;
         }
@@ -519,7 +528,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
     int cur_tt = -1;
     Item it;
     for (int i = 0; get_item(p, i, it); ++i) {
-      const int ab = i & 1;
+      const int ab = i % C::NACC, use = i / C::NACC;
       const int64_t tok0 = (int64_t)it.tt * NT;
       if (MODE == 1 && it.tt != cur_tt) {  // the token tile's targets
         asm volatile("bar.sync 1, 128;\n" ::: "memory");
@@ -532,7 +541,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
       const bool live = v < it.row_end;
       const float sp = row_scale(load_row(p, v)).sp;  // loads overlap the wait below
       // one outcome for all four epilogue warps: they share named barriers below
-      if (!tc::bar_and(1, 128, tc::mbar_wait(&acc_full[ab], (i >> 1) & 1, p.err))) break;
+      if (!tc::bar_and(1, 128, tc::mbar_wait(&acc_full[ab], use & 1, p.err))) break;
       tc::fence_after_sync();
 #pragma unroll 1
       for (int c = 0; c < NT / 16; ++c) {
@@ -651,7 +660,7 @@ int tc_residency(const cudaFuncAttributes& fa, size_t smem, int tmem_cols, int r
 
 template <int NT, int CPC, int DQ, int MODE>
 cudaError_t launch_tc_cfg(const TcParams& p, cudaStream_t st) {
-  const size_t smem = tc_smem_bytes<NT>(p.sb, (int)(p.D >> p.g_shift), MODE == 1);
+  const size_t smem = tc_smem_bytes<NT>(p.sb, p.spk, (int)(p.D >> p.g_shift), MODE == 1);
   auto kern = residual_tc_kernel<NT, CPC, DQ, MODE>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -691,39 +700,36 @@ cudaError_t launch_tc_mode(const TcParams& p, int nt, int g, cudaStream_t st) {
   }
 }
 
-// Deepest B ring (2 .. max_sb stages) whose shared memory fits the budget, or 0.
+// First (B stages, packed stages) pair whose shared memory fits the budget; nt = 0 if none.
 template <int NT>
-int fit_sb(int max_sb, int G, bool nll, size_t budget) {
-  for (int sb = max_sb; sb >= 2; --sb)
-    if (tc_smem_bytes<NT>(sb, G, nll) <= budget) return sb;
-  return 0;
+TcPlan fit_rings(const int (*pairs)[2], int npairs, int G, bool nll, size_t budget) {
+  for (int i = 0; i < npairs; ++i)
+    if (tc_smem_bytes<NT>(pairs[i][0], pairs[i][1], G, nll) <= budget)
+      return TcPlan{NT, pairs[i][0], 0, pairs[i][1]};
+  return TcPlan{0, 0, 0, 0};
 }
 
 }  // namespace
 
 TcPlan tc_plan(const Shapes& s, bool nll) {
-  // Shared memory per SM is 228 KB with 1 KB reserved per CTA; a CTA may take 227 KB.
-  // Token tiles up to 64 use 256 TMEM columns and keep two CTAs per SM within budget.
-  const size_t two_per_sm = 228 * 1024 / 2 - 1024, one_per_sm = 227 * 1024;
+  // Shared memory per SM is 228 KB with 1 KB reserved per CTA: two CTAs per SM take at
+  // most 113 KB each.
+  const size_t two_per_sm = 228 * 1024 / 2 - 1024;
   const int G = (int)(s.D / s.g);
-  TcPlan pl = {0, 0, (s.r_c + s.r_r + 31) / 32};
+  TcPlan pl = {0, 0, 0, 0};
   if (s.N > 64) {
-    if ((pl.sb = fit_sb<128>(4, G, nll, one_per_sm))) pl.nt = 128;
+    static const int p128[][2] = {{2, 4}, {2, 3}, {2, 2}};
+    pl = fit_rings<128>(p128, 3, G, nll, two_per_sm);
   }
   if (!pl.nt) {
-    const int nt = s.N <= 16 ? 16 : (s.N <= 32 ? 32 : 64);
-    const int max_sb = nt == 16 ? 8 : (nt == 32 ? 6 : 4);
-    int sb = 0;
-    switch (nt) {
-      case 16: sb = fit_sb<16>(max_sb, G, nll, two_per_sm); break;
-      case 32: sb = fit_sb<32>(max_sb, G, nll, two_per_sm); break;
-      default: sb = fit_sb<64>(max_sb, G, nll, two_per_sm); break;
-    }
-    if (sb) {
-      pl.nt = nt;
-      pl.sb = sb;
-    }
+    static const int p16[][2] = {{8, 6}, {7, 6}, {6, 6}, {5, 6}, {4, 6}, {3, 6}, {2, 6}, {2, 4}};
+    static const int p32[][2] = {{6, 6}, {5, 6}, {4, 6}, {3, 6}, {2, 6}, {2, 4}};
+    static const int p64[][2] = {{4, 4}, {3, 4}, {2, 4}};
+    if (s.N <= 16) pl = fit_rings<16>(p16, 8, G, nll, two_per_sm);
+    else if (s.N <= 32) pl = fit_rings<32>(p32, 6, G, nll, two_per_sm);
+    else pl = fit_rings<64>(p64, 3, G, nll, two_per_sm);
   }
+  pl.nrb = (s.r_c + s.r_r + 31) / 32;
   return pl;
 }
 
@@ -773,6 +779,7 @@ cudaError_t launch_residual_tc(const __half* Hb, const archead_head* head, const
   // factor rows as aligned words: both ranks multiples of 4 (bases are 16-byte aligned)
   p.a_words = (s.r_c % 4 == 0 && s.r_r % 4 == 0) ? 1 : 0;
   p.sb = plan.sb;
+  p.spk = plan.sp;
   p.err = err;
   p.n_tok_tiles = (int)((s.N + plan.nt - 1) / plan.nt);
   {
@@ -784,7 +791,8 @@ cudaError_t launch_residual_tc(const __half* Hb, const archead_head* head, const
     p.tt_band = (int)band;
   }
   p.n_vtiles = (s.V + 127) / 128;
-  if (plan.nt == 0 || plan.sb < 2 || plan.sb > kMaxSB) return cudaErrorInvalidValue;
+  if (plan.nt == 0 || plan.sb < 2 || plan.sb > kMaxSB || plan.sp < 2 || plan.sp > kMaxSP)
+    return cudaErrorInvalidValue;
   cudaError_t e = Y ? launch_tc_mode<0>(p, plan.nt, s.g, st)
                     : launch_tc_mode<1>(p, plan.nt, s.g, st);
   ++*launches;
