@@ -394,6 +394,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
     int k = 0;   // A-ring sequence: residual and rank blocks
     int kp = 0;  // packed-ring sequence: residual blocks only
+    int sp = 0;  // its slot (kp % SPK) and phase parity ((kp / SPK) & 1), kept incrementally
+    uint32_t spar = 0;
     bool ok = true;
     Item it;
     bool have = get_item(p, 0, it);
@@ -420,8 +422,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
       }
       const unsigned char* crow = cds + cs * round16(code_bytes) + tid * G;
       for (int kb = 0; kb < nkb; ++kb, ++k, ++kp) {
-        const int sp = kp % SPK, sa = k % C::SA;
-        if (!__all_sync(0xffffffffu, tc::mbar_wait(&p_full[sp], (kp / SPK) & 1, p.err))) {
+        const int sa = k % C::SA;
+        if (!__all_sync(0xffffffffu, tc::mbar_wait(&p_full[sp], spar, p.err))) {
           ok = false;
           break;
         }
@@ -447,6 +449,10 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
         }
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&p_empty[sp]);
+        if (++sp == SPK) {
+          sp = 0;
+          spar ^= 1u;
+        }
         if (k >= C::SA) {
           if (!__all_sync(0xffffffffu,
                           tc::mbar_wait(&a_empty[sa], ((k / C::SA) - 1) & 1, p.err))) {
