@@ -77,11 +77,14 @@ struct TcCfg {
   static constexpr int HSTAGE = NT * 256;      // bytes of one 128-column B block
   // Two CTAs per SM (256 TMEM columns each) for every tile: a single MMA issuer per SM
   // sustains only about one 8-MMA stage per ~950 cycles (stage handshakes ride on commit
-  // and mbarrier latencies), two issuers fill each other's gaps.  The 128-token tile then
-  // keeps one accumulator (the next item's MMAs wait for the epilogue while the other CTA
-  // uses the tensor core); smaller tiles double-buffer it.
+  // and mbarrier latencies), two issuers fill each other's gaps.  Tiles of 64 and 128
+  // tokens keep one accumulator, which the epilogue frees as soon as it holds the values in
+  // registers, so three (NT = 64) or two (NT = 128) A stages fit; smaller tiles
+  // double-buffer the accumulator and keep three A stages.  An A stage is reused only
+  // after the MMAs reading it have completed (about a thousand cycles after their issue),
+  // so the A-ring depth bounds the stage rate.
   static constexpr int TMEM_COLS = 256;
-  static constexpr int NACC = NT == 128 ? 1 : 2;
+  static constexpr int NACC = NT >= 64 ? 1 : 2;
   // A-ring stages (64 columns each) in what the accumulators leave, at most 4
   static constexpr int SA =
       (TMEM_COLS - NACC * NT) / 64 < 4 ? (TMEM_COLS - NACC * NT) / 64 : 4;
@@ -266,71 +269,86 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
   if (warp == 8) {
     // ---------------- producer: one thread, two streams ----------------
     // The packed stream (group codes once per item, then the packed blocks) and the B
-    // stream (the token tile's image blocks) are polled without blocking, and whichever
-    // ring has a free stage is refilled, so neither waits behind the other (as two lanes of
-    // one warp, a lane blocked on its full ring held the other's refills back).  The B
+    // stream (the token tile's image blocks) are polled without blocking, and every free
+    // stage of either ring is refilled in the same pass, so neither waits behind the other
+    // (as two lanes of one warp, a lane blocked on its full ring held the other's refills
+    // back).  The thread is on the critical path of the whole pipeline: ring slots and
+    // phases advance incrementally and the source addresses by constant strides.  The B
     // image comes from the prologue kernels (this kernel is a programmatic dependent
     // launch): the B stream starts once the packed ring is full.  No progress for about a
     // second sets the device error word; the copies in flight are then drained.
     if (lane == 0) {
       Item pit, hit;
       bool p_have = get_item(p, 0, pit), h_have = get_item(p, 0, hit);
-      int ip = 0, pkb = -1, kpk = 0, np = 0, nc = 0;  // pkb = -1: the item's codes are next
-      int ih = 0, hkb = 0, kh = 0, nb = 0;
+      int ip = 0, pkb = -1;  // packed stream: item, block (-1: the item's codes are next)
+      int np = 0, nc = 0, ps = 0, cs = 0;
+      uint32_t pph = 0, cph = 0;  // phase parities of the next refill of slot ps / cs
+      const uint8_t* psrc = nullptr;
+      int ih = 0, hkb = 0, nb = 0, hs = 0;
+      uint32_t hph = 0;
+      const unsigned char* hsrc =
+          h_have ? reinterpret_cast<const unsigned char*>(p.Hb) + (int64_t)hit.tt * nkbt * C::HSTAGE
+                 : nullptr;
       bool h_started = false, ok = true;
       long long idle0 = clock64();
       while (ok && (p_have || h_have)) {
         bool progress = false;
-        if (p_have) {
+        // packed stream: codes, then blocks, while slots are free
+        while (p_have) {
           if (pkb < 0) {
-            const int cs = ip & 1;
-            if (ip < 2 || tc::mbar_test(&c_empty[cs], ((ip >> 1) - 1) & 1)) {
-              tc::fence_proxy_async_smem();  // the slot was read with generic loads
-              tc::mbar_arrive_expect_tx(&c_full[cs], (uint32_t)code_bytes);
-              tc::bulk_g2s(cds + cs * round16(code_bytes), p.code + pit.row0 * G,
-                           (uint32_t)code_bytes, &c_full[cs]);
-              ++nc;
-              pkb = 0;
-              progress = true;
+            if (nc >= 2 && !tc::mbar_test(&c_empty[cs], cph ^ 1u)) break;
+            tc::fence_proxy_async_smem();  // the slot was read with generic loads
+            tc::mbar_arrive_expect_tx(&c_full[cs], (uint32_t)code_bytes);
+            tc::bulk_g2s(cds + cs * round16(code_bytes), p.code + pit.row0 * G,
+                         (uint32_t)code_bytes, &c_full[cs]);
+            ++nc;
+            if (++cs == 2) {
+              cs = 0;
+              cph ^= 1u;
             }
+            pkb = 0;
+            psrc = p.nib + ((pit.vt * nkb) << 13);
           } else {
-            const int sp = kpk % SPK;
-            if (kpk < SPK || tc::mbar_test(&p_empty[sp], ((kpk / SPK) - 1) & 1)) {
-              tc::fence_proxy_async_smem();  // the stage was read with generic loads
-              tc::mbar_arrive_expect_tx(&p_full[sp], kPkBytes);
-              tc::bulk_g2s(pk + sp * kPkBytes, p.nib + ((pit.vt * nkb + pkb) << 13), kPkBytes,
-                           &p_full[sp]);
-              ++np;
-              ++kpk;
-              progress = true;
-              if (++pkb == nkb) {
-                ++ip;
-                pkb = -1;
-                p_have = get_item(p, ip, pit);
-              }
+            if (np >= SPK && !tc::mbar_test(&p_empty[ps], pph ^ 1u)) break;
+            tc::fence_proxy_async_smem();  // the stage was read with generic loads
+            tc::mbar_arrive_expect_tx(&p_full[ps], kPkBytes);
+            tc::bulk_g2s(pk + ps * kPkBytes, psrc, kPkBytes, &p_full[ps]);
+            psrc += kPkBytes;
+            ++np;
+            if (++ps == SPK) {
+              ps = 0;
+              pph ^= 1u;
+            }
+            if (++pkb == nkb) {
+              pkb = -1;
+              p_have = get_item(p, ++ip, pit);
             }
           }
+          progress = true;
         }
-        if (h_have && (h_started || !p_have || kpk >= SPK)) {
+        // B stream: every free stage
+        while (h_have && (h_started || !p_have || np >= SPK)) {
           if (!h_started) {
             grid_dependency_wait();
             h_started = true;
           }
-          const int sb = kh % SB;
-          if (kh < SB || tc::mbar_test(&b_empty[sb], ((kh / SB) - 1) & 1)) {
-            const unsigned char* hsrc = reinterpret_cast<const unsigned char*>(p.Hb) +
-                                        ((int64_t)hit.tt * nkbt + hkb) * C::HSTAGE;
-            tc::mbar_arrive_expect_tx(&b_full[sb], C::HSTAGE);
-            tc::bulk_g2s(Hs + sb * C::HSTAGE, hsrc, C::HSTAGE, &b_full[sb]);
-            ++nb;
-            ++kh;
-            progress = true;
-            if (++hkb == nkbt) {
-              ++ih;
-              hkb = 0;
-              h_have = get_item(p, ih, hit);
-            }
+          if (nb >= SB && !tc::mbar_test(&b_empty[hs], hph ^ 1u)) break;
+          tc::mbar_arrive_expect_tx(&b_full[hs], C::HSTAGE);
+          tc::bulk_g2s(Hs + hs * C::HSTAGE, hsrc, C::HSTAGE, &b_full[hs]);
+          hsrc += C::HSTAGE;
+          ++nb;
+          if (++hs == SB) {
+            hs = 0;
+            hph ^= 1u;
           }
+          if (++hkb == nkbt) {
+            hkb = 0;
+            h_have = get_item(p, ++ih, hit);
+            if (h_have)
+              hsrc = reinterpret_cast<const unsigned char*>(p.Hb) +
+                     (int64_t)hit.tt * nkbt * C::HSTAGE;
+          }
+          progress = true;
         }
         if (progress) {
           idle0 = clock64();
@@ -350,9 +368,17 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
     }
   } else if (warp == 9) {
     // ---------------- MMA issuer ----------------
+    // A single thread whose every step is on the critical path of the stage ring: ring
+    // slots and phases advance incrementally (no division), the B descriptor of a stage is
+    // one add to a base descriptor (start address field in 16-byte units; shared-memory
+    // addresses stay below 2^18, so the field never carries), the K steps of a residual
+    // block are unrolled with constant offsets, and the A and B barriers are probed
+    // together before any blocking wait.
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_f16_m128(NT);
-      int k = 0;
+      const uint64_t bdesc0 = tc::smem_desc_kmajor_sw128(tc::smem_u32(Hs));
+      int sa = 0, sb = 0;
+      uint32_t pa = 0, pb = 0;
       bool ok = true;
       Item it;
       for (int i = 0; ok && get_item(p, i, it); ++i) {
@@ -360,28 +386,42 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
         if (i >= C::NACC && !tc::mbar_wait(&acc_empty[ab], (use - 1) & 1, p.err)) break;
         tc::fence_after_sync();
         const uint32_t dcol = tbase + ab * NT;
-        for (int kb = 0; kb < nkbt; ++kb, ++k) {
-          const int sa = k % C::SA, sb = k % SB;
-          // residual blocks: 8 K steps; rank blocks: the steps that hold factor columns
-          const int steps = kb < nkb ? 8 : min(8, p.rank_steps - 8 * (kb - nkb));
-          if (!tc::mbar_wait(&a_full[sa], (k / C::SA) & 1, p.err) ||
-              !tc::mbar_wait(&b_full[sb], (k / SB) & 1, p.err)) {
+        for (int kb = 0; kb < nkbt; ++kb) {
+          const bool a_rdy = tc::mbar_try_wait(&a_full[sa], pa);
+          const bool b_rdy = tc::mbar_try_wait(&b_full[sb], pb);
+          if (!(a_rdy && b_rdy) && (!tc::mbar_wait(&a_full[sa], pa, p.err) ||
+                                    !tc::mbar_wait(&b_full[sb], pb, p.err))) {
             ok = false;
             break;
           }
           tc::fence_after_sync();
-          const uint32_t hb = tc::smem_u32(Hs + sb * C::HSTAGE);
+          // K step j: 64-column half j / 4 (NT x 128 bytes each), 32-byte offset j % 4
+          const uint64_t bd = bdesc0 + (uint64_t)((sb * C::HSTAGE) >> 4);
+          const uint32_t ad = acol + 64 * sa;
+          if (kb < nkb) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            if (j < steps) {
-              // K step j: 64-column half j / 4 (NT x 128 bytes each), 32-byte offset j % 4
-              const uint64_t bd =
-                  tc::smem_desc_kmajor_sw128(hb + (j >> 2) * NT * 128 + (j & 3) * 32);
-              tc::mma_f16_ts(dcol, acol + 64 * sa + 8 * j, bd, idesc, (kb | j) != 0);
-            }
+            for (int j = 0; j < 8; ++j)
+              tc::mma_f16_ts(dcol, ad + 8 * j, bd + (((j >> 2) * NT * 128 + (j & 3) * 32) >> 4),
+                             idesc, (kb | j) != 0);
+          } else {
+            // rank blocks: the K steps that hold factor columns
+            const int steps = min(8, p.rank_steps - 8 * (kb - nkb));
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              if (j < steps)
+                tc::mma_f16_ts(dcol, ad + 8 * j,
+                               bd + (((j >> 2) * NT * 128 + (j & 3) * 32) >> 4), idesc, 1u);
           }
           tc::mma_commit(&a_empty[sa]);
           tc::mma_commit(&b_empty[sb]);
+          if (++sa == C::SA) {
+            sa = 0;
+            pa ^= 1u;
+          }
+          if (++sb == SB) {
+            sb = 0;
+            pb ^= 1u;
+          }
         }
         if (ok) tc::mma_commit(&acc_full[ab]);
       }
@@ -549,56 +589,71 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
       // one outcome for all four epilogue warps: they share named barriers below
       if (!tc::bar_and(1, 128, tc::mbar_wait(&acc_full[ab], use & 1, p.err))) break;
       tc::fence_after_sync();
+      // The accumulator is read in batches of up to 32 columns into registers (all loads of
+      // a batch in flight together); it is released as soon as the last batch is in
+      // registers, before that batch is scaled and stored.
+      constexpr int HC = NT < 32 ? NT : 32;
 #pragma unroll 1
-      for (int c = 0; c < NT / 16; ++c) {
-        float y[16];
-        tc::tmem_ld16(tbase + ab * NT + lane_off + 16 * c, y);
+      for (int h = 0; h < NT / HC; ++h) {
+        uint32_t r[HC / 16][16];
 #pragma unroll
-        for (int q = 0; q < 16; ++q) y[q] *= sp;
-        if (MODE == 0) {
-          if (live) {
+        for (int c = 0; c < HC / 16; ++c)
+          tc::tmem_ld16_nowait(tbase + ab * NT + lane_off + h * HC + 16 * c, r[c]);
+#pragma unroll
+        for (int c = 0; c < HC / 16; ++c) tc::tmem_wait_ld(r[c]);
+        if (h == NT / HC - 1) {
+          tc::fence_before_sync();
+          tc::mbar_arrive(&acc_empty[ab]);
+        }
+#pragma unroll
+        for (int c = 0; c < HC / 16; ++c) {
+          const int c16 = h * (HC / 16) + c;  // 16-token chunk of the tile
+          float y[16];
+#pragma unroll
+          for (int q = 0; q < 16; ++q) y[q] = __uint_as_float(r[c][q]) * sp;
+          if (MODE == 0) {
+            if (live) {
+#pragma unroll
+              for (int q = 0; q < 16; ++q) {
+                const int64_t tok = tok0 + 16 * c16 + q;
+                if (tok < p.N) p.Y[tok * p.V + v] = y[q];
+              }
+            }
+          } else {
+            // ---- fused NLL: per token of the chunk, (max, sum exp) over the tile's rows ----
+            const float NEG_INF = __int_as_float(0xff800000);
 #pragma unroll
             for (int q = 0; q < 16; ++q) {
-              const int64_t tok = tok0 + 16 * c + q;
-              if (tok < p.N) p.Y[tok * p.V + v] = y[q];
+              nll_y[q * 128 + e] = live ? y[q] : NEG_INF;
+              const int tg = tgt_s[16 * c16 + q];
+              if (live && tg == v) p.tlogit[tok0 + 16 * c16 + q] = y[q];
             }
-          }
-        } else {
-          // ---- fused NLL: per token of the chunk, (max, sum exp) over the tile's rows ----
-          const float NEG_INF = __int_as_float(0xff800000);
+            asm volatile("bar.sync 1, 128;\n" ::: "memory");
+            // thread e: token q = e / 8 of the chunk, rows 16 * (e % 8) .. +15
+            const int q = e >> 3, seg = e & 7;
+            const float* yr = nll_y + q * 128 + 16 * seg;
+            float m = NEG_INF;
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            nll_y[q * 128 + e] = live ? y[q] : NEG_INF;
-            const int tg = tgt_s[16 * c + q];
-            if (live && tg == v) p.tlogit[tok0 + 16 * c + q] = y[q];
-          }
-          asm volatile("bar.sync 1, 128;\n" ::: "memory");
-          // thread e: token q = e / 8 of the chunk, rows 16 * (e % 8) .. +15
-          const int q = e >> 3, seg = e & 7;
-          const float* yr = nll_y + q * 128 + 16 * seg;
-          float m = NEG_INF;
+            for (int i = 0; i < 16; ++i) m = fmaxf(m, yr[i]);
+            float sm = 0.f;
+            if (m != NEG_INF) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) m = fmaxf(m, yr[i]);
-          float sm = 0.f;
-          if (m != NEG_INF) {
+              for (int i = 0; i < 16; ++i) sm += __expf(yr[i] - m);
+            }
 #pragma unroll
-            for (int i = 0; i < 16; ++i) sm += __expf(yr[i] - m);
+            for (int o = 1; o < 8; o <<= 1) {  // combine the 8 segments of the token
+              const float mo = __shfl_xor_sync(0xffffffffu, m, o);
+              const float so = __shfl_xor_sync(0xffffffffu, sm, o);
+              const float mn = fmaxf(m, mo);
+              sm = (m == NEG_INF ? 0.f : sm * __expf(m - mn)) + (mo == NEG_INF ? 0.f : so * __expf(mo - mn));
+              m = mn;
+            }
+            const int64_t tok = tok0 + 16 * c16 + q;
+            if (seg == 0 && tok < p.N) p.part[tok * p.n_vtiles + it.vt] = make_float2(m, sm);
+            asm volatile("bar.sync 1, 128;\n" ::: "memory");
           }
-#pragma unroll
-          for (int o = 1; o < 8; o <<= 1) {  // combine the 8 segments of the token
-            const float mo = __shfl_xor_sync(0xffffffffu, m, o);
-            const float so = __shfl_xor_sync(0xffffffffu, sm, o);
-            const float mn = fmaxf(m, mo);
-            sm = (m == NEG_INF ? 0.f : sm * __expf(m - mn)) + (mo == NEG_INF ? 0.f : so * __expf(mo - mn));
-            m = mn;
-          }
-          const int64_t tok = tok0 + 16 * c + q;
-          if (seg == 0 && tok < p.N) p.part[tok * p.n_vtiles + it.vt] = make_float2(m, sm);
-          asm volatile("bar.sync 1, 128;\n" ::: "memory");
         }
       }
-      tc::fence_before_sync();
-      tc::mbar_arrive(&acc_empty[ab]);
     }
   }
 
