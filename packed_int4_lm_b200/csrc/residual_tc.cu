@@ -41,7 +41,7 @@
 namespace archead {
 namespace {
 
-constexpr int kTcThreads = 320;  // warps 0-3 dequant, 4-7 epilogue, 8 producer, 9 MMA
+constexpr int kTcThreads = 352;  // warps 0-3 dequant, 4-7 epilogue, 8 and 10 producers, 9 MMA
 constexpr int kPkBytes = 8192;   // packed block of one 128-row tile (128 columns)
 constexpr int kMaxSB = 8;        // deepest B ring
 constexpr int kMaxSP = 8;        // deepest packed ring
@@ -77,14 +77,14 @@ struct TcCfg {
   static constexpr int HSTAGE = NT * 256;      // bytes of one 128-column B block
   // Two CTAs per SM (256 TMEM columns each) for every tile: a single MMA issuer per SM
   // sustains only about one 8-MMA stage per ~950 cycles (stage handshakes ride on commit
-  // and mbarrier latencies), two issuers fill each other's gaps.  Tiles of 64 and 128
-  // tokens keep one accumulator, which the epilogue frees as soon as it holds the values in
-  // registers, so three (NT = 64) or two (NT = 128) A stages fit; smaller tiles
-  // double-buffer the accumulator and keep three A stages.  An A stage is reused only
-  // after the MMAs reading it have completed (about a thousand cycles after their issue),
-  // so the A-ring depth bounds the stage rate.
+  // and mbarrier latencies), two issuers fill each other's gaps.  The 128-token tile keeps
+  // one accumulator, which the epilogue frees once its last 32-column batch is in
+  // registers (two A stages fit beside it); smaller tiles double-buffer the accumulator, so the
+  // next item's MMAs never wait for the epilogue, and keep two (NT = 64) or three A
+  // stages.  An A stage is reused only after the MMAs reading it have completed (about a
+  // thousand cycles after their issue), so the A-ring depth bounds the stage rate.
   static constexpr int TMEM_COLS = 256;
-  static constexpr int NACC = NT >= 64 ? 1 : 2;
+  static constexpr int NACC = NT == 128 ? 1 : 2;
   // A-ring stages (64 columns each) in what the accumulators leave, at most 4
   static constexpr int SA =
       (TMEM_COLS - NACC * NT) / 64 < 4 ? (TMEM_COLS - NACC * NT) / 64 : 4;
@@ -267,72 +267,77 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
   const uint32_t acol = tbase + C::NACC * NT;  // A ring after the accumulators (lane 0)
 
   if (warp == 8) {
-    // ---------------- producer: one thread, two streams ----------------
-    // The packed stream (group codes once per item, then the packed blocks) and the B
-    // stream (the token tile's image blocks) are polled without blocking, and every free
-    // stage of either ring is refilled in the same pass, so neither waits behind the other
-    // (as two lanes of one warp, a lane blocked on its full ring held the other's refills
-    // back).  The thread is on the critical path of the whole pipeline: ring slots and
-    // phases advance incrementally and the source addresses by constant strides.  The B
-    // image comes from the prologue kernels (this kernel is a programmatic dependent
-    // launch): the B stream starts once the packed ring is full.  No progress for about a
-    // second sets the device error word; the copies in flight are then drained.
+    // ---------------- packed producer (one thread) ----------------
+    // Each item's group codes, then its packed blocks, each copy as soon as its slot is
+    // released (blocking waits: the thread sleeps instead of taking issue slots from the
+    // dequant warps).  Ring slots and phases advance incrementally and the source address
+    // by a constant stride: the thread is on the critical path of the pipeline.  A wait
+    // that gives up drains the copies in flight.
     if (lane == 0) {
-      Item pit, hit;
-      bool p_have = get_item(p, 0, pit), h_have = get_item(p, 0, hit);
-      int ip = 0, pkb = -1;  // packed stream: item, block (-1: the item's codes are next)
-      int np = 0, nc = 0, ps = 0, cs = 0;
+      Item pit;
+      bool p_have = get_item(p, 0, pit);
+      int ip = 0, np = 0, nc = 0, ps = 0, cs = 0;
       uint32_t pph = 0, cph = 0;  // phase parities of the next refill of slot ps / cs
-      const uint8_t* psrc = nullptr;
-      int ih = 0, hkb = 0, nb = 0, hs = 0;
-      uint32_t hph = 0;
-      const unsigned char* hsrc =
-          h_have ? reinterpret_cast<const unsigned char*>(p.Hb) + (int64_t)hit.tt * nkbt * C::HSTAGE
-                 : nullptr;
-      bool h_started = false, ok = true;
-      long long idle0 = clock64();
-      while (ok && (p_have || h_have)) {
-        bool progress = false;
-        // packed stream: codes, then blocks, while slots are free
-        while (p_have) {
-          if (pkb < 0) {
-            if (nc >= 2 && !tc::mbar_test(&c_empty[cs], cph ^ 1u)) break;
-            tc::fence_proxy_async_smem();  // the slot was read with generic loads
-            tc::mbar_arrive_expect_tx(&c_full[cs], (uint32_t)code_bytes);
-            tc::bulk_g2s(cds + cs * round16(code_bytes), p.code + pit.row0 * G,
-                         (uint32_t)code_bytes, &c_full[cs]);
-            ++nc;
-            if (++cs == 2) {
-              cs = 0;
-              cph ^= 1u;
-            }
-            pkb = 0;
-            psrc = p.nib + ((pit.vt * nkb) << 13);
-          } else {
-            if (np >= SPK && !tc::mbar_test(&p_empty[ps], pph ^ 1u)) break;
-            tc::fence_proxy_async_smem();  // the stage was read with generic loads
-            tc::mbar_arrive_expect_tx(&p_full[ps], kPkBytes);
-            tc::bulk_g2s(pk + ps * kPkBytes, psrc, kPkBytes, &p_full[ps]);
-            psrc += kPkBytes;
-            ++np;
-            if (++ps == SPK) {
-              ps = 0;
-              pph ^= 1u;
-            }
-            if (++pkb == nkb) {
-              pkb = -1;
-              p_have = get_item(p, ++ip, pit);
-            }
-          }
-          progress = true;
+      bool ok = true;
+      while (ok && p_have) {
+        if (nc >= 2 && !tc::mbar_wait(&c_empty[cs], cph ^ 1u, p.err)) {
+          ok = false;
+          break;
         }
-        // B stream: every free stage
-        while (h_have && (h_started || !p_have || np >= SPK)) {
-          if (!h_started) {
-            grid_dependency_wait();
-            h_started = true;
+        tc::fence_proxy_async_smem();  // the slot was read with generic loads
+        tc::mbar_arrive_expect_tx(&c_full[cs], (uint32_t)code_bytes);
+        tc::bulk_g2s(cds + cs * round16(code_bytes), p.code + pit.row0 * G,
+                     (uint32_t)code_bytes, &c_full[cs]);
+        ++nc;
+        if (++cs == 2) {
+          cs = 0;
+          cph ^= 1u;
+        }
+        const uint8_t* psrc = p.nib + ((pit.vt * nkb) << 13);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (np >= SPK && !tc::mbar_wait(&p_empty[ps], pph ^ 1u, p.err)) {
+            ok = false;
+            break;
           }
-          if (nb >= SB && !tc::mbar_test(&b_empty[hs], hph ^ 1u)) break;
+          tc::fence_proxy_async_smem();  // the stage was read with generic loads
+          tc::mbar_arrive_expect_tx(&p_full[ps], kPkBytes);
+          tc::bulk_g2s(pk + ps * kPkBytes, psrc, kPkBytes, &p_full[ps]);
+          psrc += kPkBytes;
+          ++np;
+          if (++ps == SPK) {
+            ps = 0;
+            pph ^= 1u;
+          }
+        }
+        p_have = get_item(p, ++ip, pit);
+      }
+      if (!ok) {  // drain copies still in flight before the CTA exits
+        for (int q = np - SPK < 0 ? 0 : np - SPK; q < np; ++q)
+          tc::mbar_wait(&p_full[q % SPK], (q / SPK) & 1, p.err);
+        for (int q = nc - 2 < 0 ? 0 : nc - 2; q < nc; ++q)
+          tc::mbar_wait(&c_full[q & 1], (q >> 1) & 1, p.err);
+      }
+    }
+  } else if (warp == 10) {
+    // ---------------- B producer (one thread) ----------------
+    // The token tile's image blocks, one per stage, each as soon as the MMAs that read its
+    // slot have completed.  The image comes from the prologue kernels (this kernel is a
+    // programmatic dependent launch), so the stream starts after the dependency wait.
+    if (lane == 0) {
+      grid_dependency_wait();
+      Item hit;
+      bool h_have = get_item(p, 0, hit);
+      int ih = 0, nb = 0, hs = 0;
+      uint32_t hph = 0;
+      bool ok = true;
+      while (ok && h_have) {
+        const unsigned char* hsrc =
+            reinterpret_cast<const unsigned char*>(p.Hb) + (int64_t)hit.tt * nkbt * C::HSTAGE;
+        for (int kb = 0; kb < nkbt; ++kb) {
+          if (nb >= SB && !tc::mbar_wait(&b_empty[hs], hph ^ 1u, p.err)) {
+            ok = false;
+            break;
+          }
           tc::mbar_arrive_expect_tx(&b_full[hs], C::HSTAGE);
           tc::bulk_g2s(Hs + hs * C::HSTAGE, hsrc, C::HSTAGE, &b_full[hs]);
           hsrc += C::HSTAGE;
@@ -341,40 +346,24 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
             hs = 0;
             hph ^= 1u;
           }
-          if (++hkb == nkbt) {
-            hkb = 0;
-            h_have = get_item(p, ++ih, hit);
-            if (h_have)
-              hsrc = reinterpret_cast<const unsigned char*>(p.Hb) +
-                     (int64_t)hit.tt * nkbt * C::HSTAGE;
-          }
-          progress = true;
         }
-        if (progress) {
-          idle0 = clock64();
-        } else if (clock64() - idle0 > (1ll << 31)) {
-          atomicOr(p.err, kErrTimeout);
-          ok = false;
-        }
+        h_have = get_item(p, ++ih, hit);
       }
-      if (!ok) {  // drain copies still in flight before the CTA exits
-        for (int q = np - SPK < 0 ? 0 : np - SPK; q < np; ++q)
-          tc::mbar_wait(&p_full[q % SPK], (q / SPK) & 1, p.err);
-        for (int q = nc - 2 < 0 ? 0 : nc - 2; q < nc; ++q)
-          tc::mbar_wait(&c_full[q & 1], (q >> 1) & 1, p.err);
+      if (!ok) {
         for (int q = nb - SB < 0 ? 0 : nb - SB; q < nb; ++q)
           tc::mbar_wait(&b_full[q % SB], (q / SB) & 1, p.err);
       }
     }
   } else if (warp == 9) {
-    // ---------------- MMA issuer ----------------
-    // A single thread whose every step is on the critical path of the stage ring: ring
-    // slots and phases advance incrementally (no division), the B descriptor of a stage is
-    // one add to a base descriptor (start address field in 16-byte units; shared-memory
-    // addresses stay below 2^18, so the field never carries), the K steps of a residual
-    // block are unrolled with constant offsets, and the A and B barriers are probed
-    // together before any blocking wait.
-    if (lane == 0) {
+    // ---------------- MMA issuer: the whole warp, one elected lane issues ----------------
+    // The issuing thread is on the critical path of the stage ring, so its stream is kept
+    // short: ring slots and phases advance incrementally (no division), the B descriptor
+    // of a stage is one add to a base descriptor (start address field in 16-byte units;
+    // shared-memory addresses stay below 2^18, so the field never carries), the K steps of
+    // a residual block are unrolled with constant offsets, and the whole warp runs the
+    // loop converged so those values stay warp-uniform; one elected lane issues the MMAs
+    // and commits.
+    {
       const uint32_t idesc = tc::idesc_f16_m128(NT);
       const uint64_t bdesc0 = tc::smem_desc_kmajor_sw128(tc::smem_u32(Hs));
       int sa = 0, sb = 0;
@@ -383,14 +372,17 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
       Item it;
       for (int i = 0; ok && get_item(p, i, it); ++i) {
         const int ab = i % C::NACC, use = i / C::NACC;
-        if (i >= C::NACC && !tc::mbar_wait(&acc_empty[ab], (use - 1) & 1, p.err)) break;
+        if (i >= C::NACC &&
+            !__all_sync(0xffffffffu, tc::mbar_wait(&acc_empty[ab], (use - 1) & 1, p.err)))
+          break;
         tc::fence_after_sync();
         const uint32_t dcol = tbase + ab * NT;
         for (int kb = 0; kb < nkbt; ++kb) {
           const bool a_rdy = tc::mbar_try_wait(&a_full[sa], pa);
           const bool b_rdy = tc::mbar_try_wait(&b_full[sb], pb);
-          if (!(a_rdy && b_rdy) && (!tc::mbar_wait(&a_full[sa], pa, p.err) ||
-                                    !tc::mbar_wait(&b_full[sb], pb, p.err))) {
+          if (!__all_sync(0xffffffffu, (a_rdy && b_rdy) ||
+                                           (tc::mbar_wait(&a_full[sa], pa, p.err) &&
+                                            tc::mbar_wait(&b_full[sb], pb, p.err)))) {
             ok = false;
             break;
           }
@@ -398,22 +390,26 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
           // K step j: 64-column half j / 4 (NT x 128 bytes each), 32-byte offset j % 4
           const uint64_t bd = bdesc0 + (uint64_t)((sb * C::HSTAGE) >> 4);
           const uint32_t ad = acol + 64 * sa;
-          if (kb < nkb) {
+          if (tc::elect_one()) {
+            if (kb < nkb) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              tc::mma_f16_ts(dcol, ad + 8 * j, bd + (((j >> 2) * NT * 128 + (j & 3) * 32) >> 4),
-                             idesc, (kb | j) != 0);
-          } else {
-            // rank blocks: the K steps that hold factor columns
-            const int steps = min(8, p.rank_steps - 8 * (kb - nkb));
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              if (j < steps)
+              for (int j = 0; j < 8; ++j)
                 tc::mma_f16_ts(dcol, ad + 8 * j,
-                               bd + (((j >> 2) * NT * 128 + (j & 3) * 32) >> 4), idesc, 1u);
+                               bd + (((j >> 2) * NT * 128 + (j & 3) * 32) >> 4), idesc,
+                               (kb | j) != 0);
+            } else {
+              // rank blocks: the K steps that hold factor columns
+              const int steps = min(8, p.rank_steps - 8 * (kb - nkb));
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                if (j < steps)
+                  tc::mma_f16_ts(dcol, ad + 8 * j,
+                                 bd + (((j >> 2) * NT * 128 + (j & 3) * 32) >> 4), idesc, 1u);
+            }
+            tc::mma_commit(&a_empty[sa]);
+            tc::mma_commit(&b_empty[sb]);
           }
-          tc::mma_commit(&a_empty[sa]);
-          tc::mma_commit(&b_empty[sb]);
+          __syncwarp();
           if (++sa == C::SA) {
             sa = 0;
             pa ^= 1u;
@@ -423,10 +419,14 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
             pb ^= 1u;
           }
         }
-        if (ok) tc::mma_commit(&acc_full[ab]);
+        if (ok && tc::elect_one()) tc::mma_commit(&acc_full[ab]);
+        __syncwarp();
       }
-      tc::mma_commit(mma_done);
-      tc::mbar_wait(mma_done, 0, p.err);  // every MMA issued here has retired
+      if (tc::elect_one()) {
+        tc::mma_commit(mma_done);
+        tc::mbar_wait(mma_done, 0, p.err);  // every MMA issued here has retired
+      }
+      __syncwarp();
     }
   } else if (warp < 4) {
     // ---------------- dequant: thread = tile row = TMEM lane ----------------
@@ -613,10 +613,14 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
           for (int q = 0; q < 16; ++q) y[q] = __uint_as_float(r[c][q]) * sp;
           if (MODE == 0) {
             if (live) {
+              // token rows of the chunk below N, one pointer stepped by a row of Y
+              const int64_t t16 = tok0 + 16 * c16;
+              const int64_t nq = p.N - t16;
+              float* yp = p.Y + t16 * p.V + v;
 #pragma unroll
               for (int q = 0; q < 16; ++q) {
-                const int64_t tok = tok0 + 16 * c16 + q;
-                if (tok < p.N) p.Y[tok * p.V + v] = y[q];
+                if (q < nq) *yp = y[q];
+                yp += p.V;
               }
             }
           } else {

@@ -200,6 +200,20 @@ __device__ __forceinline__ uint64_t smem_desc_kmajor_sw128(uint32_t saddr) {
   return d;
 }
 
+// True in exactly one lane of a converged warp (elect.sync over the full mask).  Code that
+// keeps a whole warp converged around single-thread tensor-core issue lets the compiler
+// hold the warp-uniform operands (descriptors, addresses, ring counters) in uniform
+// registers.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "elect.sync _|P, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}\n"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // D[tmem] (+)= A[tmem] * B[smem]^T, one M=128 x N x K=16 step, issued by one thread.
 __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                            uint32_t idesc, uint32_t accumulate) {
