@@ -176,6 +176,10 @@ int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* ta
   const size_t o_t = cv.take(use_tc ? 0 : (size_t)s.N * RR * 4);
   const size_t o_part = nll_mode ? cv.take((size_t)s.N * nvblk * 8) : 0;
   const size_t o_tl = nll_mode ? cv.take((size_t)s.N * 4) : 0;
+  // a single token tile is split evenly over the CTAs (partials + per-tile counters)
+  const size_t split_bytes = use_tc ? tc_split_scratch_bytes(s, plan) : 0;
+  const size_t o_scr = split_bytes ? cv.take(split_bytes) : 0;
+  const size_t o_cnt = split_bytes ? cv.take((size_t)((s.V + 127) / 128) * 4) : 0;
   void* base = nullptr;
   if (cudaMallocFromPoolAsync(&base, cv.off, ds->pool, st) != cudaSuccess) {
     cudaGetLastError();
@@ -183,16 +187,18 @@ int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* ta
   }
   char* b = static_cast<char*>(base);
   __half* Hh = reinterpret_cast<__half*>(b + o_hh);
+  float* scr = split_bytes ? reinterpret_cast<float*>(b + o_scr) : nullptr;
+  unsigned* cnt = split_bytes ? reinterpret_cast<unsigned*>(b + o_cnt) : nullptr;
   float* t = reinterpret_cast<float*>(b + o_t);
-  cudaError_t e = use_tc ? launch_prologue_blocked(H, head, s, plan, Hh, ds->err, st, &launches)
+  cudaError_t e = use_tc ? launch_prologue_blocked(H, head, s, plan, Hh, cnt, ds->err, st, &launches)
                          : launch_prologue(H, head, s, Npad, Hh, t, ds->err, st, &launches);
   if (e == cudaSuccess) {
     if (use_tc) {
       float2* part = nll_mode ? reinterpret_cast<float2*>(b + o_part) : nullptr;
       float* tl = nll_mode ? reinterpret_cast<float*>(b + o_tl) : nullptr;
       prof_mark(0, st);
-      e = launch_residual_tc(Hh, head, s, plan, nll_mode ? nullptr : Y, targets, part, tl,
-                             ds->err, st, &launches);
+      e = launch_residual_tc(Hh, head, s, plan, nll_mode ? nullptr : Y, targets, part, tl, scr,
+                             cnt, ds->err, st, &launches);
       prof_mark(1, st);
       if (e == cudaSuccess && nll_mode)
         e = launch_nll_combine(part, tl, targets, s, nll, ds->err, st, &launches);

@@ -189,15 +189,23 @@ __host__ __device__ __forceinline__ int64_t tc_image_offset(int64_t tt, int64_t 
          ((((kk >> 3) & 7) ^ (int)(nn & 7)) << 3) + (kk & 7);
 }
 // Blocked image of H (zero rows up to the token tile) and its rank blocks.
+// counters: the per-tile counters of a split launch (ceil(V/128) words, zeroed here), or
+// nullptr.
 cudaError_t launch_prologue_blocked(const uint16_t* H, const archead_head* head,
                                     const Shapes& s, const TcPlan& plan, __half* Hb,
-                                    unsigned* err, cudaStream_t st, int* launches);
+                                    unsigned* counters, unsigned* err, cudaStream_t st,
+                                    int* launches);
+// Bytes of scratch for a launch whose single token tile is split evenly over the CTAs
+// (0 when the shape has more than one token tile).
+size_t tc_split_scratch_bytes(const Shapes& s, const TcPlan& plan);
 // Y != nullptr: write logits.  Y == nullptr: fused NLL, writing (max, sum exp) partials
 // into part[N x ceil(V/128)] and target logits into tlogit[N] (see launch_nll_combine).
+// scratch / counters (tc_split_scratch_bytes, launch_prologue_blocked): the split of a
+// single token tile over the CTAs, or nullptr for whole tiles per CTA.
 cudaError_t launch_residual_tc(const __half* Hb, const archead_head* head, const Shapes& s,
                                const TcPlan& plan, float* Y, const int32_t* targets,
-                               float2* part, float* tlogit, unsigned* err, cudaStream_t st,
-                               int* launches);
+                               float2* part, float* tlogit, float* scratch, unsigned* counters,
+                               unsigned* err, cudaStream_t st, int* launches);
 
 // Decode path (N <= 16): persistent bulk-copy-fed warp-MMA kernel with H resident in
 // shared memory.  nt8 = 0 when the shape does not fit (then the token-block kernel runs).

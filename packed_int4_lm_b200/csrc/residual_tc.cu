@@ -69,6 +69,14 @@ struct TcParams {
   int n_tok_tiles;
   int tt_band;  // token tiles per band (their B image stays in L2 while the head streams)
   int64_t n_vtiles;
+  // One token tile: the (tile, K block) units are split evenly over the CTAs, so a tile
+  // at the edge of a CTA's range is shared with the neighbouring CTA (its "head" blocks
+  // in one, its "tail" blocks in the next).  Each part's raw accumulator goes to scratch
+  // ([CTA][slot 0: first item, 1: last item][NT][128] FP32); the part that arrives second
+  // at the tile's counter (zeroed by the prologue) adds the two and finishes the tile.
+  int split;
+  float* scratch;
+  unsigned* counters;
   unsigned* err;
 };
 
@@ -111,10 +119,29 @@ size_t tc_smem_bytes(int sb, int sp, int G, bool nll) {
 struct Item {
   int64_t vt, row0, row_end;
   int tt;
+  int kb0, kb1;  // the item's K blocks [kb0, kb1) of the tile's nkb + nrb
+  int part;      // 0: whole tile; 1: head part (blocks from 0); 2: tail part (to the end)
 };
 
 __device__ __forceinline__ bool get_item(const TcParams& p, int k, Item& it) {
-  if (p.n_tok_tiles == 1) {
+  const int nkbt = (int)(p.D >> 7) + p.nrb;
+  it.kb0 = 0;
+  it.kb1 = nkbt;
+  it.part = 0;
+  if (p.split) {
+    // units u = tile * nkbt + block, [u0, u1) per CTA; every range spans at least one
+    // tile (the grid has at most one CTA per tile), so a tile has at most two parts
+    const int64_t U = p.n_vtiles * nkbt;
+    const int64_t u0 = U * blockIdx.x / gridDim.x;
+    const int64_t u1 = U * (blockIdx.x + 1) / gridDim.x;
+    it.vt = u0 / nkbt + k;
+    const int64_t ts = it.vt * nkbt;
+    if (ts >= u1) return false;
+    it.kb0 = u0 > ts ? (int)(u0 - ts) : 0;
+    it.kb1 = u1 < ts + nkbt ? (int)(u1 - ts) : nkbt;
+    it.part = it.kb0 > 0 ? 2 : (it.kb1 < nkbt ? 1 : 0);
+    it.tt = 0;
+  } else if (p.n_tok_tiles == 1) {
     const int64_t t0 = p.n_vtiles * blockIdx.x / gridDim.x;
     const int64_t t1 = p.n_vtiles * (blockIdx.x + 1) / gridDim.x;
     it.vt = t0 + k;
@@ -234,6 +261,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
   uint64_t* acc_empty = acc_full + 2;    // [2]
   uint64_t* mma_done = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  int* ep_flag = reinterpret_cast<int*>(tmem_slot + 1);  // epilogue: a tile counter's value
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -293,8 +321,9 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
           cs = 0;
           cph ^= 1u;
         }
-        const uint8_t* psrc = p.nib + ((pit.vt * nkb) << 13);
-        for (int kb = 0; kb < nkb; ++kb) {
+        const int pk1 = pit.kb1 < nkb ? pit.kb1 : nkb;
+        const uint8_t* psrc = p.nib + ((pit.vt * nkb + pit.kb0) << 13);
+        for (int kb = pit.kb0; kb < pk1; ++kb) {
           if (np >= SPK && !tc::mbar_wait(&p_empty[ps], pph ^ 1u, p.err)) {
             ok = false;
             break;
@@ -331,9 +360,9 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
       uint32_t hph = 0;
       bool ok = true;
       while (ok && h_have) {
-        const unsigned char* hsrc =
-            reinterpret_cast<const unsigned char*>(p.Hb) + (int64_t)hit.tt * nkbt * C::HSTAGE;
-        for (int kb = 0; kb < nkbt; ++kb) {
+        const unsigned char* hsrc = reinterpret_cast<const unsigned char*>(p.Hb) +
+                                    ((int64_t)hit.tt * nkbt + hit.kb0) * C::HSTAGE;
+        for (int kb = hit.kb0; kb < hit.kb1; ++kb) {
           if (nb >= SB && !tc::mbar_wait(&b_empty[hs], hph ^ 1u, p.err)) {
             ok = false;
             break;
@@ -377,7 +406,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
           break;
         tc::fence_after_sync();
         const uint32_t dcol = tbase + ab * NT;
-        for (int kb = 0; kb < nkbt; ++kb) {
+        for (int kb = it.kb0; kb < it.kb1; ++kb) {
           const bool a_rdy = tc::mbar_try_wait(&a_full[sa], pa);
           const bool b_rdy = tc::mbar_try_wait(&b_full[sb], pb);
           if (!__all_sync(0xffffffffu, (a_rdy && b_rdy) ||
@@ -396,7 +425,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
               for (int j = 0; j < 8; ++j)
                 tc::mma_f16_ts(dcol, ad + 8 * j,
                                bd + (((j >> 2) * NT * 128 + (j & 3) * 32) >> 4), idesc,
-                               (kb | j) != 0);
+                               (kb != it.kb0) | (j != 0));
             } else {
               // rank blocks: the K steps that hold factor columns
               const int steps = min(8, p.rank_steps - 8 * (kb - nkb));
@@ -404,7 +433,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
               for (int j = 0; j < 8; ++j)
                 if (j < steps)
                   tc::mma_f16_ts(dcol, ad + 8 * j,
-                                 bd + (((j >> 2) * NT * 128 + (j & 3) * 32) >> 4), idesc, 1u);
+                                 bd + (((j >> 2) * NT * 128 + (j & 3) * 32) >> 4), idesc,
+                                 (kb != it.kb0) | (j != 0));
             }
             tc::mma_commit(&a_empty[sa]);
             tc::mma_commit(&b_empty[sb]);
@@ -461,7 +491,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
         break;
       }
       const unsigned char* crow = cds + cs * round16(code_bytes) + tid * G;
-      for (int kb = 0; kb < nkb; ++kb, ++k, ++kp) {
+      const int kr1 = it.kb1 < nkb ? it.kb1 : nkb;
+      for (int kb = it.kb0; kb < kr1; ++kb, ++k, ++kp) {
         const int sa = k % C::SA;
         if (!__all_sync(0xffffffffu, tc::mbar_wait(&p_full[sp], spar, p.err))) {
           ok = false;
@@ -530,7 +561,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
       // rank blocks: factor index j = 32 rb + i takes TMEM columns 2i (x1, x1) and
       // 2i + 1 (x2, x2), x = fl32(A[v, j] s_v) / S' split into FP16 hi and remainder
       const float rcp = 1.f / rs.sp;
-      for (int rb = 0; ok && rb < p.nrb; ++rb, ++k) {
+      const int rb1 = it.kb1 - nkb;
+      for (int rb = it.kb0 > nkb ? it.kb0 - nkb : 0; ok && rb < rb1; ++rb, ++k) {
         const int sa = k % C::SA;
         uint32_t fw[8];
 #pragma unroll
@@ -593,17 +625,66 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
       // a batch in flight together); it is released as soon as the last batch is in
       // registers, before that batch is scaled and stored.
       constexpr int HC = NT < 32 ? NT : 32;
+      // A part of a shared tile: the raw accumulator goes to this CTA's scratch slot, then
+      // the tile's counter tells whether the other part is already there; the second part
+      // finishes the tile from the two slots (their sum does not depend on the order).
+      const float* mine = nullptr;
+      const float* other = nullptr;
+      if (it.part) {
+        float* slot = p.scratch + (size_t)(blockIdx.x * 2 + (it.part == 1 ? 1 : 0)) * NT * 128 + e;
+#pragma unroll 1
+        for (int h = 0; h < NT / HC; ++h) {
+          uint32_t r[HC / 16][16];
+#pragma unroll
+          for (int c = 0; c < HC / 16; ++c)
+            tc::tmem_ld16_nowait(tbase + ab * NT + lane_off + h * HC + 16 * c, r[c]);
+#pragma unroll
+          for (int c = 0; c < HC / 16; ++c) tc::tmem_wait_ld(r[c]);
+          if (h == NT / HC - 1) {
+            tc::fence_before_sync();
+            tc::mbar_arrive(&acc_empty[ab]);
+          }
+#pragma unroll
+          for (int c = 0; c < HC / 16; ++c)
+#pragma unroll
+            for (int q = 0; q < 16; ++q) slot[(h * HC + 16 * c + q) * 128] = __uint_as_float(r[c][q]);
+        }
+        __threadfence();
+        asm volatile("bar.sync 1, 128;\n" ::: "memory");
+        if (e == 0) {
+          grid_dependency_wait();  // the counters are zeroed by the prologue kernels
+          *ep_flag = (int)atomicAdd(p.counters + it.vt, 1u);
+        }
+        asm volatile("bar.sync 1, 128;\n" ::: "memory");
+        const bool second = *reinterpret_cast<volatile int*>(ep_flag) != 0;
+        asm volatile("bar.sync 1, 128;\n" ::: "memory");  // the flag is reused
+        if (!second) continue;
+        __threadfence();
+        mine = slot;
+        other = p.scratch +
+                (size_t)((blockIdx.x + (it.part == 1 ? 1 : -1)) * 2 + (it.part == 1 ? 0 : 1)) * NT * 128 + e;
+      }
 #pragma unroll 1
       for (int h = 0; h < NT / HC; ++h) {
         uint32_t r[HC / 16][16];
+        if (mine) {
 #pragma unroll
-        for (int c = 0; c < HC / 16; ++c)
-          tc::tmem_ld16_nowait(tbase + ab * NT + lane_off + h * HC + 16 * c, r[c]);
+          for (int c = 0; c < HC / 16; ++c)
 #pragma unroll
-        for (int c = 0; c < HC / 16; ++c) tc::tmem_wait_ld(r[c]);
-        if (h == NT / HC - 1) {
-          tc::fence_before_sync();
-          tc::mbar_arrive(&acc_empty[ab]);
+            for (int q = 0; q < 16; ++q) {
+              const int col = (h * HC + 16 * c + q) * 128;
+              r[c][q] = __float_as_uint(__ldcg(mine + col) + __ldcg(other + col));
+            }
+        } else {
+#pragma unroll
+          for (int c = 0; c < HC / 16; ++c)
+            tc::tmem_ld16_nowait(tbase + ab * NT + lane_off + h * HC + 16 * c, r[c]);
+#pragma unroll
+          for (int c = 0; c < HC / 16; ++c) tc::tmem_wait_ld(r[c]);
+          if (h == NT / HC - 1) {
+            tc::fence_before_sync();
+            tc::mbar_arrive(&acc_empty[ab]);
+          }
         }
 #pragma unroll
         for (int c = 0; c < HC / 16; ++c) {
@@ -678,8 +759,12 @@ __global__ void __launch_bounds__(256) convert_h_blocked_kernel(const uint16_t* 
                                                                 __half* __restrict__ Hb,
                                                                 int64_t N, int64_t Npad,
                                                                 int64_t D, int64_t nkbt, int nt,
+                                                                unsigned* counters, int64_t ncnt,
                                                                 unsigned* err) {
   allow_dependent_launch();
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < ncnt;
+       i += (int64_t)gridDim.x * blockDim.x)
+    counters[i] = 0u;
   const int64_t chunks_per_row = nkbt * 16;  // 8 FP16 per chunk
   const int64_t total = Npad * chunks_per_row;
   const int64_t hchunks = D / 8;
@@ -798,16 +883,27 @@ TcPlan tc_plan(const Shapes& s, bool nll) {
   return pl;
 }
 
+size_t tc_split_scratch_bytes(const Shapes& s, const TcPlan& plan) {
+  if (plan.nt == 0 || s.N > plan.nt) return 0;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  // two CTAs per SM at most (tensor memory), two slots each
+  return (size_t)2 * sms * 2 * plan.nt * 128 * 4;
+}
+
 cudaError_t launch_prologue_blocked(const uint16_t* H, const archead_head* head,
                                     const Shapes& s, const TcPlan& plan, __half* Hb,
-                                    unsigned* err, cudaStream_t st, int* launches) {
+                                    unsigned* counters, unsigned* err, cudaStream_t st,
+                                    int* launches) {
   const int nt = plan.nt;
   const int64_t Npad = (s.N + nt - 1) / nt * nt;
   const int64_t nkbt = s.D / 128 + plan.nrb;
   int64_t blocks = (Npad * nkbt * 16 + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
   convert_h_blocked_kernel<<<(unsigned)(blocks < 1 ? 1 : blocks), 256, 0, st>>>(
-      H, Hb, s.N, Npad, s.D, nkbt, nt, err);
+      H, Hb, s.N, Npad, s.D, nkbt, nt, counters, counters ? (s.V + 127) / 128 : 0, err);
   ++*launches;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -816,8 +912,8 @@ cudaError_t launch_prologue_blocked(const uint16_t* H, const archead_head* head,
 
 cudaError_t launch_residual_tc(const __half* Hb, const archead_head* head, const Shapes& s,
                                const TcPlan& plan, float* Y, const int32_t* targets,
-                               float2* part, float* tlogit, unsigned* err, cudaStream_t st,
-                               int* launches) {
+                               float2* part, float* tlogit, float* scratch, unsigned* counters,
+                               unsigned* err, cudaStream_t st, int* launches) {
   TcParams p;
   p.Hb = Hb;
   p.nib = head->r_nib;
@@ -856,6 +952,9 @@ cudaError_t launch_residual_tc(const __half* Hb, const archead_head* head, const
     p.tt_band = (int)band;
   }
   p.n_vtiles = (s.V + 127) / 128;
+  p.split = (p.n_tok_tiles == 1 && scratch && counters) ? 1 : 0;
+  p.scratch = scratch;
+  p.counters = counters;
   if (plan.nt == 0 || plan.sb < 2 || plan.sb > kMaxSB || plan.sp < 2 || plan.sp > kMaxSP)
     return cudaErrorInvalidValue;
   cudaError_t e = Y ? launch_tc_mode<0>(p, plan.nt, s.g, st)

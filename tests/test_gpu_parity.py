@@ -183,6 +183,34 @@ def test_many_items_per_cta_consistent(dev):
             assert diff <= tol, (rep, N, diff, tol)
 
 
+@pytest.mark.parametrize("N", [20, 64])
+def test_split_tiles_match_oracle(dev, N):
+    """One token tile over more 128-row tiles than resident CTAs: the (tile, K block) units
+    are split evenly, so the tiles at the edges of the CTAs' ranges are computed in two
+    parts (raw accumulators through scratch, finished by the part that arrives second).
+    Every row of the logits and the NLL must match the oracle, and repeated calls must be
+    bit-identical (the two parts are added in an order-independent way)."""
+    V, D = 40000, 256
+    # scaled into the logit regime (rms of a few units), where an NLL bound in nats means
+    # something (as the NLL head above)
+    head = random_canonical_head(V, D, 16, 16, 64, seed=50, zero_rows=5,
+                                 super_exp_range=(-17, -13), factor_exp_range=(-13, -10))
+    dh = ah.DeviceHead.from_canonical(head, dev)
+    H = _rand_H(N, D, 51 + N)
+    Hd = H.to(dev)
+    Y = ah.logits(Hd, dh)
+    ah.check()
+    _assert_logits(Y.cpu().numpy(), oracle.logits(head, bf16_bits(H)), f"split N={N}")
+    for _ in range(3):
+        assert torch.equal(ah.logits(Hd, dh), Y)
+    tg = make_targets(N, V, 52 + N)
+    out = ah.nll(Hd, dh, tg.to(dev))
+    ah.check()
+    ref = oracle.nll(head, bf16_bits(H), tg.numpy())
+    err = np.max(np.abs(out.cpu().double().numpy() - ref))
+    assert err <= NLL_TOL, err
+
+
 def test_host_entry_points_match_device(dev, rhead):
     head, dh = rhead
     H = _rand_H(20, 512, 5)
