@@ -59,44 +59,6 @@ __device__ __forceinline__ void dequant_word(uint32_t w, __half2 c2, __half2 nc2
   out[3] = __hfma2(*reinterpret_cast<__half2*>(&p3), c2, nc24);
 }
 
-// Same result as dequant_word with fewer integer-pipe instructions (one shift, four
-// LOP3) and more FP16 ones.  A nibble in bits 0-3 of a half under exponent 1024 (pattern
-// 0x6400, unit 1) reads 1024 + n; in bits 4-7 it reads 1024 + 16n.  With the top bit
-// flipped (offset binary n = q + 8), x - 1032 and x / 16 - 72 both give q exactly, and
-// q * c is exact in FP16 (|q * c| <= 2040).
-__device__ __forceinline__ void dequant_word_lite(uint32_t w, __half2 c2, __half2 out[4]) {
-  const uint32_t w2 = w >> 8;
-  uint32_t x0 = and_xor(w, 0x000F000Fu, 0x64086408u);
-  uint32_t x1 = and_xor(w, 0x00F000F0u, 0x64806480u);
-  uint32_t x2 = and_xor(w2, 0x000F000Fu, 0x64086408u);
-  uint32_t x3 = and_xor(w2, 0x00F000F0u, 0x64806480u);
-  const __half2 k1032 = __float2half2_rn(1032.f);
-  const __half2 k16 = __float2half2_rn(0.0625f);
-  const __half2 k72 = __float2half2_rn(-72.f);
-  out[0] = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&x0), k1032), c2);
-  out[1] = __hmul2(__hfma2(*reinterpret_cast<__half2*>(&x1), k16, k72), c2);
-  out[2] = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&x2), k1032), c2);
-  out[3] = __hmul2(__hfma2(*reinterpret_cast<__half2*>(&x3), k16, k72), c2);
-}
-
-// Exact FP16 q of the eight nibbles of one device-layout word, without a group scale
-// (for kernels that apply the scale to FP32 partial sums): the magic-number reads of
-// dequant_word_lite minus their offsets.
-__device__ __forceinline__ void dequant_word_q(uint32_t w, __half2 out[4]) {
-  const uint32_t w2 = w >> 8;
-  uint32_t x0 = and_xor(w, 0x000F000Fu, 0x64086408u);
-  uint32_t x1 = and_xor(w, 0x00F000F0u, 0x64806480u);
-  uint32_t x2 = and_xor(w2, 0x000F000Fu, 0x64086408u);
-  uint32_t x3 = and_xor(w2, 0x00F000F0u, 0x64806480u);
-  const __half2 k1032 = __float2half2_rn(1032.f);
-  const __half2 k16 = __float2half2_rn(0.0625f);
-  const __half2 k72 = __float2half2_rn(-72.f);
-  out[0] = __hsub2(*reinterpret_cast<__half2*>(&x0), k1032);
-  out[1] = __hfma2(*reinterpret_cast<__half2*>(&x1), k16, k72);
-  out[2] = __hsub2(*reinterpret_cast<__half2*>(&x2), k1032);
-  out[3] = __hfma2(*reinterpret_cast<__half2*>(&x3), k16, k72);
-}
-
 // Device nibble layout, tiled: rows are padded to a multiple of 128 and every 128-row
 // tile's 128-column block (64 bytes per row) is one contiguous 8 KB region, so each tile
 // streams sequentially from HBM.  Inside the region, 16-byte chunk i (i = 0..3) of row s

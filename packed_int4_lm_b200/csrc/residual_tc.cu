@@ -230,7 +230,7 @@ __device__ __forceinline__ void prefetch_l2(const void* ptr) {
   asm volatile("prefetch.global.L2 [%0];\n" ::"l"(ptr));
 }
 
-template <int NT, int CPC, int DQ, int MODE>
+template <int NT, int CPC, int MODE>
 __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcParams p) {
   using C = TcCfg<NT>;
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -538,15 +538,12 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
         for (int w = 0; w < 4; ++w) {
           // c 2^-k is exact in FP16 (8 significant bits, k <= 24)
           const __half2 c2 = __float2half2_rn((float)cw[w] * rs.cs);
+          const __half2 nc24 = __hmul2(c2, __float2half2_rn(-24.f));  // exact: 3 c 2^(3-k)
           uint32_t a16[16];
 #pragma unroll
           for (int t4 = 0; t4 < 4; ++t4) {
             __half2 pr[4];
-            if (DQ == 0) {
-              dequant_word(wd[4 * t4 + w], c2, __hmul2(c2, __float2half2_rn(-24.f)), pr);
-            } else {
-              dequant_word_lite(wd[4 * t4 + w], c2, pr);
-            }
+            dequant_word(wd[4 * t4 + w], c2, nc24, pr);
 #pragma unroll
             for (int q = 0; q < 4; ++q) a16[4 * t4 + q] = h2_bits(pr[q]);
           }
@@ -808,10 +805,10 @@ int tc_residency(const cudaFuncAttributes& fa, size_t smem, int tmem_cols, int r
   return occ;
 }
 
-template <int NT, int CPC, int DQ, int MODE>
+template <int NT, int CPC, int MODE>
 cudaError_t launch_tc_cfg(const TcParams& p, cudaStream_t st) {
   const size_t smem = tc_smem_bytes<NT>(p.sb, p.spk, (int)(p.D >> p.g_shift), MODE == 1);
-  auto kern = residual_tc_kernel<NT, CPC, DQ, MODE>;
+  auto kern = residual_tc_kernel<NT, CPC, MODE>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -835,9 +832,9 @@ cudaError_t launch_tc_cfg(const TcParams& p, cudaStream_t st) {
 
 template <int NT, int MODE>
 cudaError_t launch_tc_nt(const TcParams& p, int g, cudaStream_t st) {
-  if (g == 32) return launch_tc_cfg<NT, 4, 1, MODE>(p, st);
-  if (g == 64) return launch_tc_cfg<NT, 2, 1, MODE>(p, st);
-  return launch_tc_cfg<NT, 1, 1, MODE>(p, st);
+  if (g == 32) return launch_tc_cfg<NT, 4, MODE>(p, st);
+  if (g == 64) return launch_tc_cfg<NT, 2, MODE>(p, st);
+  return launch_tc_cfg<NT, 1, MODE>(p, st);
 }
 
 template <int MODE>
