@@ -145,7 +145,8 @@ __device__ __forceinline__ bool dec_wait(uint64_t* bar, uint32_t parity, unsigne
 // magic-number reads of the nibbles: 1032 + q for columns with (d & 2) == 0 and
 // 1152 + 16 q for the others, whose H values are stored divided by 16 (exact: a power of
 // two).  Each k-block sum then carries the constant 1032 sum_A b + 1152 sum_B b over the
-// stored values b, which corr holds and the kernel subtracts before scaling by the code.
+// stored values b; corr holds its negation, from which the kernel's MMA chain of the block
+// starts, so the chain ends at the block's dot product.
 // Non-finite or out-of-range FP16 values set kErrRangeH.
 // Runs on blocks blk of nblk.
 __device__ __forceinline__ void dec_convert_h(const uint16_t* __restrict__ H,
@@ -186,7 +187,7 @@ __device__ __forceinline__ void dec_convert_h(const uint16_t* __restrict__ H,
     *reinterpret_cast<uint2*>(img + dec_h_offset(n, d, D)) = make_uint2(lo, hi);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    if (lane == 0) corr[kb * ntok + n] = scale_b ? sum : 0.f;
+    if (lane == 0) corr[kb * ntok + n] = scale_b ? -sum : 0.f;
   }
   for (int64_t i = blk * (int64_t)blockDim.x + threadIdx.x; i < n_counters;
        i += nblk * (int64_t)blockDim.x)
@@ -272,14 +273,14 @@ __host__ __device__ __forceinline__ bool dec_arow_copy(int64_t rows, int r_c, in
   return ((rows * r_c) % 16) == 0 && ((rows * r_r) % 16) == 0;
 }
 
-// m16n8k16 FP16 MMA with a zero accumulator input: d = a * b.
-__device__ __forceinline__ void mma_f16_16816_z(float d[4], const uint32_t a[4], uint32_t b0,
-                                                uint32_t b1) {
+// m16n8k16 FP16 MMA, D = A * B + (c0, c1, c0, c1): the chain's start value per accumulator column pair.
+__device__ __forceinline__ void mma_f16_16816_c(float d[4], const uint32_t a[4], uint32_t b0,
+                                                uint32_t b1, float c0, float c1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-      "{%8, %9}, {%10, %10, %10, %10};\n"
+      "{%8, %9}, {%10, %11, %10, %11};\n"
       : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(c0), "f"(c1));
 }
 
 // Raw magic-number reads of the eight nibbles of a device-layout word (no FP16 math):
@@ -293,9 +294,11 @@ __device__ __forceinline__ void nibble_reads(uint32_t w, uint32_t x[4]) {
 }
 
 // NB (1 or 2) consecutive blocks with one group code each (g >= 128): raw nibble reads
-// (nibble_reads) times the resident B image, one independent two-MMA chain per (block,
-// chunk), then acc += code * (sum of the chains - corr).  The chains are summed in a fixed
-// order.
+// (nibble_reads) times the resident B image, one chain of eight MMAs per block, plus the
+// block's negated offset constant (corr: the chain's start value for one token block,
+// added after the chain for two), then acc += code * (chain + offset).  The blocks'
+// chains are independent; one chain per block needs no adds to combine partial chains,
+// which costs less than the longer MMA dependency.
 template <int NT8, int NB>
 __device__ __forceinline__ void dec_blocks_q(const uint32_t (&wlo)[2][4],
                                              const uint32_t (&whi)[2][4],
@@ -304,7 +307,14 @@ __device__ __forceinline__ void dec_blocks_q(const uint32_t (&wlo)[2][4],
                                              const int (&hoff)[4], const float* corr, int kb2,
                                              int tq, float (&acc)[NT8][4]) {
   constexpr int NTOK = 8 * NT8;
-  float t[NB][4][NT8][4];
+  float t[NB][NT8][4];
+  float2 ncr[NB][NT8];
+#pragma unroll
+  for (int b = 0; b < NB; ++b)
+#pragma unroll
+    for (int j = 0; j < NT8; ++j)
+      if (NT8 == 1)
+        ncr[b][j] = *reinterpret_cast<const float2*>(corr + (kb2 + b) * NTOK + 8 * j + 2 * tq);
 #pragma unroll
   for (int c = 0; c < 4; ++c)
 #pragma unroll
@@ -318,8 +328,11 @@ __device__ __forceinline__ void dec_blocks_q(const uint32_t (&wlo)[2][4],
       for (int j = 0; j < NT8; ++j) {
         const uint4 hv =
             *reinterpret_cast<const uint4*>(Hb + hrow[j] + (kb2 + b) * 256 + hoff[c]);
-        mma_f16_16816_z(t[b][c][j], a0, hv.x, hv.y);
-        mma_f16_16816(t[b][c][j], a1, hv.z, hv.w);
+        if (c == 0)  // chain start: the negated offset (one token block), or zero
+          mma_f16_16816_c(t[b][j], a0, hv.x, hv.y, NT8 == 1 ? ncr[b][j].x : 0.f,
+                          NT8 == 1 ? ncr[b][j].y : 0.f);
+        else mma_f16_16816(t[b][j], a0, hv.x, hv.y);
+        mma_f16_16816(t[b][j], a1, hv.z, hv.w);
       }
     }
 #pragma unroll
@@ -327,16 +340,14 @@ __device__ __forceinline__ void dec_blocks_q(const uint32_t (&wlo)[2][4],
     const float fl = (float)clo[b], fh = (float)chi[b];
 #pragma unroll
     for (int j = 0; j < NT8; ++j) {
-      const float2 cr =
-          *reinterpret_cast<const float2*>(corr + (kb2 + b) * NTOK + 8 * j + 2 * tq);
-      float sm[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        sm[e] = (t[b][0][j][e] + t[b][1][j][e]) + (t[b][2][j][e] + t[b][3][j][e]);
-      acc[j][0] = fmaf(fl, sm[0] - cr.x, acc[j][0]);
-      acc[j][1] = fmaf(fl, sm[1] - cr.y, acc[j][1]);
-      acc[j][2] = fmaf(fh, sm[2] - cr.x, acc[j][2]);
-      acc[j][3] = fmaf(fh, sm[3] - cr.y, acc[j][3]);
+      if (NT8 != 1)
+        ncr[b][j] = *reinterpret_cast<const float2*>(corr + (kb2 + b) * NTOK + 8 * j + 2 * tq);
+      // two token blocks: the offset is added here (fewer registers live across the chain)
+      const float ox = NT8 == 1 ? 0.f : ncr[b][j].x, oy = NT8 == 1 ? 0.f : ncr[b][j].y;
+      acc[j][0] = fmaf(fl, t[b][j][0] + ox, acc[j][0]);
+      acc[j][1] = fmaf(fl, t[b][j][1] + oy, acc[j][1]);
+      acc[j][2] = fmaf(fh, t[b][j][2] + ox, acc[j][2]);
+      acc[j][3] = fmaf(fh, t[b][j][3] + oy, acc[j][3]);
     }
   }
 }

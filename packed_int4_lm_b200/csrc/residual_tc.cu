@@ -182,8 +182,10 @@ __device__ __forceinline__ RowIn load_row(const TcParams& p, int64_t v) {
 // Accumulator scale S' = S 2^k of a row and the factor 2^-k applied to its group codes
 // (0 when S = 0: the residual row is zero and is dropped).  With M = 128 max(|sAc|, |sAw|)
 // bounding every factor entry, k = ilogb(M) - ilogb(S) - 13 puts M / S' in (2^12, 2^14);
-// k is clamped to [-5, 40] (q c 2^5 <= 65280 stays finite in FP16; q c 2^-k is exact for
-// k <= 24 and below that the residual is under 2^-30 of the factor terms).
+// k is clamped to [-3, 40]: the dequant's fused multiply-add takes -24 c 2^-k as an FP16
+// operand, and 24 * 255 * 2^3 = 48960 stays finite (a larger k only shrinks M / S'); q c
+// 2^-k is exact for k <= 24, and below that the residual is under 2^-30 of the factor
+// terms.
 struct RowScale {
   float sp, cs;
 };
@@ -194,7 +196,7 @@ __device__ __forceinline__ RowScale row_scale(const RowIn& in) {
     int k = 0;
     if (M > 0.f) {
       k = ilogbf(M) - ilogbf(in.S) - 13;
-      k = k < -5 ? -5 : (k > 40 ? 40 : k);
+      k = k < -3 ? -3 : (k > 40 ? 40 : k);
     }
     r.sp = ldexpf(in.S, k);
     r.cs = ldexpf(1.f, -k);
