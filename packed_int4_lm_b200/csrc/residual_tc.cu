@@ -468,6 +468,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
     int kp = 0;  // packed-ring sequence: residual blocks only
     int sp = 0;  // its slot (kp % SPK) and phase parity ((kp / SPK) & 1), kept incrementally
     uint32_t spar = 0;
+    bool p_ready = false, a_ready = false;  // the next stage's barriers, probed early
     bool ok = true;
     Item it;
     bool have = get_item(p, 0, it);
@@ -496,7 +497,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
       const int kr1 = it.kb1 < nkb ? it.kb1 : nkb;
       for (int kb = it.kb0; kb < kr1; ++kb, ++k, ++kp) {
         const int sa = k % C::SA;
-        if (!__all_sync(0xffffffffu, tc::mbar_wait(&p_full[sp], spar, p.err))) {
+        if (!__all_sync(0xffffffffu, p_ready) &&
+            !__all_sync(0xffffffffu, tc::mbar_wait(&p_full[sp], spar, p.err))) {
           ok = false;
           break;
         }
@@ -527,13 +529,19 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
           spar ^= 1u;
         }
         if (k >= C::SA) {
-          if (!__all_sync(0xffffffffu,
+          if (!__all_sync(0xffffffffu, a_ready) &&
+              !__all_sync(0xffffffffu,
                           tc::mbar_wait(&a_empty[sa], ((k / C::SA) - 1) & 1, p.err))) {
             ok = false;
             break;
           }
           tc::fence_after_sync();
         }
+        // The next stage's barriers are probed now and their answers used only after this
+        // stage's arithmetic, which hides the shared-memory round trip of the probe; a
+        // phase seen complete stays complete until this thread releases the slot.
+        p_ready = tc::mbar_test(&p_full[sp], spar);
+        a_ready = k + 1 < C::SA || tc::mbar_test(&a_empty[(k + 1) % C::SA], (((k + 1) / C::SA) - 1) & 1);
         const uint32_t ta = acol + 64 * sa + lane_off;
         // window w (32 block columns) = TMEM columns 16w..16w+15: words w, 4+w, 8+w, 12+w
 #pragma unroll
@@ -555,6 +563,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
         tc::fence_before_sync();
         tc::mbar_arrive(&a_full[sa]);
       }
+      a_ready = false;  // probed for the next A stage, which the rank blocks wait for themselves
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&c_empty[cs]);
       // rank blocks: factor index j = 32 rb + i takes TMEM columns 2i (x1, x1) and
