@@ -13,27 +13,31 @@
 // k_v is chosen from the row's scales alone: every factor entry obeys |a| <= 128 max(sAc,
 // sAw), and k puts that bound between 2^12 and 2^14 after division by S', far inside FP16.
 //
-// Persistent, warp-specialised kernel.  A work item is one 128-row vocabulary tile for one
-// tile of NT tokens (NT = 16..128):
-//  * warp 8 (two threads, independent streams) feeds three shared-memory rings with bulk
-//    copies (TMA engine, no tensor map, no multicast): the tile's 8 KB packed-nibble block
-//    per 128 columns (one contiguous region in the tiled device layout), the tile's
-//    group-scale codes once per item, and the token tile's FP16 B blocks (pre-arranged by
-//    the prologue as the 128-byte-swizzled K-major image the MMA reads);
+// Persistent, warp-specialised kernel, two CTAs per SM.  A work item is one 128-row
+// vocabulary tile for one tile of NT tokens (NT = 16..128), or a K range of it:
+//  * warp 8 (one thread) feeds the packed ring with bulk copies (TMA engine, no tensor
+//    map, no multicast): the tile's group-scale codes once per item, then its 8 KB
+//    packed-nibble block per 128 columns (one contiguous region in the tiled device
+//    layout); warp 10 (one thread) feeds the B ring with the token tile's FP16 blocks
+//    (pre-arranged by the prologue as the 128-byte-swizzled K-major image the MMA reads).
+//    Each waits (blocking) for the slot it refills, so neither stream waits behind the
+//    other and neither takes issue slots from the dequant warps while it waits;
 //  * warps 0-3 (dequant): one vocabulary row per thread (= one TMEM lane).  A thread reads
 //    its row's four 16-byte chunks of a block (conflict free: chunk i of row s sits at
 //    (i * 128 + s) * 16), dequantises them to exact FP16 q c 2^-k, and after the residual
 //    blocks converts its row's factor entries into the rank blocks; it stores both with
-//    tcgen05.st into an A ring of 2-4 stages in tensor memory (128 x 128 FP16 = 64
+//    tcgen05.st into an A ring of 2-3 stages in tensor memory (128 x 128 FP16 = 64
 //    columns per stage);
-//  * warp 9 (one thread): issues tcgen05.mma kind::f16, A from tensor memory, B from
-//    shared memory, K=16 steps, into one of two M=128 x N=NT FP32 accumulators, so the
-//    next item's MMAs overlap the previous item's epilogue;
-//  * warps 4-7 (epilogue): tcgen05.ld of an accumulator row, times S'_v, stored coalesced
-//    into Y, or reduced on chip into split-vocabulary log-sum-exp partials (fused NLL).
-// Scheduling: with a single token tile (decode) every CTA owns a contiguous run of tiles;
-// otherwise items are dealt round-robin with the token tile varying fastest, so CTAs
-// working on the same rows run together and re-read them from L2.
+//  * warp 9 (the whole warp, one elected lane issues): tcgen05.mma kind::f16, A from
+//    tensor memory, B from shared memory, K=16 steps, into an M=128 x N=NT FP32
+//    accumulator (two of them below NT = 128, so the next item's MMAs overlap the
+//    previous item's epilogue);
+//  * warps 4-7 (epilogue): tcgen05.ld of an accumulator row, times S'_v, stored into Y, or
+//    reduced on chip into split-vocabulary log-sum-exp partials (fused NLL).
+// Scheduling: with a single token tile (decode) the (tile, K block) units are split evenly
+// over the CTAs and a tile at the edge of two ranges is finished from two partial
+// accumulators; otherwise items are dealt round-robin with the token tile varying
+// fastest, so CTAs working on the same rows run together and re-read them from L2.
 // Every mbarrier wait is bounded (about a second of SM cycles); a wait that gives up sets
 // the device error word, the CTA drains what it issued and frees its tensor memory.
 #include "tc_common.cuh"
@@ -87,10 +91,11 @@ struct TcCfg {
   // sustains only about one 8-MMA stage per ~950 cycles (stage handshakes ride on commit
   // and mbarrier latencies), two issuers fill each other's gaps.  The 128-token tile keeps
   // one accumulator, which the epilogue frees once its last 32-column batch is in
-  // registers (two A stages fit beside it); smaller tiles double-buffer the accumulator, so the
-  // next item's MMAs never wait for the epilogue, and keep two (NT = 64) or three A
-  // stages.  An A stage is reused only after the MMAs reading it have completed (about a
-  // thousand cycles after their issue), so the A-ring depth bounds the stage rate.
+  // registers (two A stages fit beside it); smaller tiles double-buffer the accumulator,
+  // so the next item's MMAs never wait for the epilogue, and keep two (NT = 64) or three
+  // A stages.  An A stage is reused only after the MMAs reading it have completed (about
+  // a thousand cycles after their issue); at these depths the dequant warps, not the
+  // ring, set the stage rate.
   static constexpr int TMEM_COLS = 256;
   static constexpr int NACC = NT == 128 ? 1 : 2;
   // A-ring stages (64 columns each) in what the accumulators leave, at most 4
