@@ -470,8 +470,9 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
     const int tid = threadIdx.x;
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
     int k = 0;   // A-ring sequence: residual and rank blocks
-    int kp = 0;  // packed-ring sequence: residual blocks only
-    int sp = 0;  // its slot (kp % SPK) and phase parity ((kp / SPK) & 1), kept incrementally
+    // packed-ring position of the next residual block (the ring carries residual blocks
+    // only): slot and phase parity, kept incrementally
+    int sp = 0;
     uint32_t spar = 0;
     bool p_ready = false, a_ready = false;  // the next stage's barriers, probed early
     bool ok = true;
@@ -500,7 +501,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
       }
       const unsigned char* crow = cds + cs * round16(code_bytes) + tid * G;
       const int kr1 = it.kb1 < nkb ? it.kb1 : nkb;
-      for (int kb = it.kb0; kb < kr1; ++kb, ++k, ++kp) {
+      for (int kb = it.kb0; kb < kr1; ++kb, ++k) {
         const int sa = k % C::SA;
         if (!__all_sync(0xffffffffu, p_ready) &&
             !__all_sync(0xffffffffu, tc::mbar_wait(&p_full[sp], spar, p.err))) {
