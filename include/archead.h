@@ -125,6 +125,31 @@ int archead_nll(const uint16_t* H, const archead_head* head, const int32_t* targ
                 void* stream);
 
 /*
+ * archead_nll_partials -- one vocabulary shard's share of archead_nll (cross-entropy of
+ *   Sec. 5, evaluated vocabulary-parallel).  `head` holds rows [v_begin, v_begin + V) of a
+ *   head with v_total rows (its V-indexed components sliced, B_c and B_w whole); targets
+ *   are global ids in [0, v_total).  For every token it writes partials[n] = (m, s, y)
+ *   (float N x 3, device): m = max_v Y[n, v] and s = sum_v exp(Y[n, v] - m) over the
+ *   shard's rows, and y = Y[n, target] if the shard owns the target row, else 0.  The
+ *   logits are not written.  Requires 0 <= v_begin, v_begin + V <= v_total < 2^31
+ *   (ARCHEAD_ERR_SHAPE otherwise); a target outside [0, v_total) sets ARCHEAD_ERR_TARGET.
+ *   Asynchronous on `stream`.
+ */
+int archead_nll_partials(const uint16_t* H, const archead_head* head, const int32_t* targets,
+                         int64_t v_begin, int64_t v_total, float* partials, int64_t N,
+                         int64_t V, int64_t D, int r_c, int r_r, int g, void* stream);
+
+/*
+ * archead_nll_merge -- nll[n] from G shards' partials (float G x N x 3, device, as
+ *   archead_nll_partials writes them, shard k at [k]): M = max_k m_k,
+ *   nll = M + log(sum_k s_k exp(m_k - M)) - sum_k y_k, combined in shard order.  Together
+ *   with an all-gather of the partials between the GPUs that hold the shards this equals
+ *   archead_nll on the whole head (up to rounding).  1 <= G <= 65536.  Asynchronous on
+ *   `stream`.
+ */
+int archead_nll_merge(const float* partials, int G, int64_t N, float* nll_out, void* stream);
+
+/*
  * archead_logits_host -- archead_logits with HOST buffers: copies H_host (bf16 N x D) to
  * the device, evaluates, copies Y back into Y_host (float N x V), and synchronises
  * `stream` before returning.  Pinned host memory gives asynchronous copies.  The device

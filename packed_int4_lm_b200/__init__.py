@@ -122,6 +122,53 @@ def nll(H: torch.Tensor, dh: DeviceHead, targets: torch.Tensor,
     return out
 
 
+def nll_partials(H: torch.Tensor, dh: DeviceHead, targets: torch.Tensor, v_begin: int,
+                 v_total: int, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """archead_nll_partials: this vocabulary shard's (max, sum exp, target logit) per token
+    (N x 3 float32).  dh holds rows [v_begin, v_begin + dh.V) of a v_total-row head."""
+    _check_H(H, dh)
+    N = H.shape[0]
+    if targets.dtype != torch.int32 or targets.shape != (N,) or not targets.is_cuda:
+        raise ValueError("targets must be an int32 CUDA tensor of shape (N,)")
+    if out is None:
+        out = torch.empty(N, 3, device=H.device, dtype=torch.float32)
+    _lib.check(_lib.lib().archead_nll_partials(H.data_ptr(), ctypes.byref(dh.struct),
+                                               targets.contiguous().data_ptr(), int(v_begin),
+                                               int(v_total), out.data_ptr() if N else None, N,
+                                               *dh.shape_args, _stream_handle(stream)),
+               "archead_nll_partials")
+    return out
+
+
+def nll_merge(partials: torch.Tensor, out: Optional[torch.Tensor] = None,
+              stream=None) -> torch.Tensor:
+    """archead_nll_merge: per-token NLL from G shards' partials (G x N x 3 float32 CUDA)."""
+    if (partials.dtype != torch.float32 or partials.dim() != 3 or partials.shape[2] != 3
+            or not partials.is_cuda):
+        raise ValueError("partials must be a float32 CUDA tensor of shape (G, N, 3)")
+    G, N = int(partials.shape[0]), int(partials.shape[1])
+    p = partials.contiguous()
+    if out is None:
+        out = torch.empty(N, device=partials.device, dtype=torch.float32)
+    _lib.check(_lib.lib().archead_nll_merge(p.data_ptr(), G, N, out.data_ptr() if N else None,
+                                            _stream_handle(stream)), "archead_nll_merge")
+    return out
+
+
+def vocab_parallel_nll(H: torch.Tensor, dh: DeviceHead, targets: torch.Tensor, v_begin: int,
+                       v_total: int, group=None) -> torch.Tensor:
+    """Per-token NLL of a head whose vocabulary rows are sharded over the ranks of `group`
+    (rank k holds dh = rows [v_begin, v_begin + dh.V)): each rank reduces its shard to
+    (max, sum exp, target logit) per token, one all-gather exchanges the N x 3 partials,
+    and every rank merges them in rank order.  H and targets are the same on every rank."""
+    import torch.distributed as dist
+    part = nll_partials(H, dh, targets, v_begin, v_total)
+    G = dist.get_world_size(group)
+    gathered = [torch.empty_like(part) for _ in range(G)]
+    dist.all_gather(gathered, part, group=group)
+    return nll_merge(torch.stack(gathered))
+
+
 def logits_host(H: torch.Tensor, dh: DeviceHead, out: Optional[torch.Tensor] = None,
                 stream=None) -> torch.Tensor:
     """archead_logits_host: host H in, host Y out (copies inside the call, synchronous)."""

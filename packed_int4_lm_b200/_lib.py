@@ -51,6 +51,9 @@ _SIGS = {
     "archead_last_launches": (c_int, []),
     "archead_logits_noalloc": (c_int, [c_vp, ctypes.POINTER(ArcheadHead), c_vp, c_i64, c_i64,
                                        c_i64, c_int, c_int, c_int, c_vp]),
+    "archead_nll_partials": (c_int, [c_vp, ctypes.POINTER(ArcheadHead), c_vp, c_i64, c_i64,
+                                     c_vp, c_i64, c_i64, c_i64, c_int, c_int, c_int, c_vp]),
+    "archead_nll_merge": (c_int, [c_vp, c_int, c_i64, c_vp, c_vp]),
     "archead_profile": (c_int, [c_int]),
     "archead_profile_read": (c_int, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(c_int)]),
 }

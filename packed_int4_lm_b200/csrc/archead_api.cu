@@ -111,11 +111,20 @@ struct Carve {
   }
 };
 
+// A vocabulary shard of a larger head (archead_nll_partials): rows [v_begin, v_begin + V)
+// of v_total; the NLL path then writes the per-token (max, sum exp, target logit) triples
+// into partials instead of the NLL.
+struct NllShard {
+  int64_t v_begin, v_total;
+  float* partials;
+};
+
 int run_dec(const uint16_t* H, const archead_head* head, float* Y, const int32_t* targets,
-            float* nll, const Shapes& s, const DecPlan& pl, DeviceState* ds, cudaStream_t st) {
+            float* nll, const Shapes& s, const DecPlan& pl, DeviceState* ds, cudaStream_t st,
+            const NllShard* shard) {
   int launches = 0;
   const int RR = s.r_c + s.r_r;
-  const bool nll_mode = nll != nullptr;
+  const bool nll_mode = nll != nullptr || shard != nullptr;
   const int64_t nvt = (s.V + 127) / 128;
   Carve cv;
   const size_t o_img = cv.take(dec_image_bytes(s, pl));
@@ -124,6 +133,7 @@ int run_dec(const uint16_t* H, const archead_head* head, float* Y, const int32_t
   const size_t o_scr = cv.take(dec_partial_bytes(pl));
   const size_t o_part = nll_mode ? cv.take((size_t)s.N * nvt * 8) : 0;
   const size_t o_tl = nll_mode ? cv.take((size_t)s.N * 4) : 0;
+  const size_t o_tloc = shard ? cv.take((size_t)s.N * 4) : 0;
   void* base = nullptr;
   if (cudaMallocFromPoolAsync(&base, cv.off, ds->pool, st) != cudaSuccess) {
     cudaGetLastError();
@@ -136,14 +146,22 @@ int run_dec(const uint16_t* H, const archead_head* head, float* Y, const int32_t
   float4* scr = reinterpret_cast<float4*>(b + o_scr);
   float2* part = nll_mode ? reinterpret_cast<float2*>(b + o_part) : nullptr;
   float* tl = nll_mode ? reinterpret_cast<float*>(b + o_tl) : nullptr;
-  cudaError_t e = launch_dec_prologue(H, head, s, pl, img, t, cnt, ds->err, st, &launches);
+  int32_t* tloc = shard ? reinterpret_cast<int32_t*>(b + o_tloc) : nullptr;
+  cudaError_t e = cudaSuccess;
+  if (shard)  // shard-local targets and zeroed target logits, before the prologue
+    e = launch_nll_shard_prep(targets, s.N, shard->v_begin, s.V, shard->v_total, tloc, tl,
+                              ds->err, st, &launches);
+  const int32_t* tg = shard ? tloc : targets;
+  if (e == cudaSuccess)
+    e = launch_dec_prologue(H, head, s, pl, img, t, cnt, ds->err, st, &launches);
   if (e == cudaSuccess) {
     prof_mark(0, st);
-    e = launch_residual_dec(img, t, head, s, pl, nll_mode ? nullptr : Y, targets, part, tl, scr,
+    e = launch_residual_dec(img, t, head, s, pl, nll_mode ? nullptr : Y, tg, part, tl, scr,
                             cnt, ds->err, st, &launches);
     prof_mark(1, st);
     if (e == cudaSuccess && nll_mode)
-      e = launch_nll_combine(part, tl, targets, s, nll, ds->err, st, &launches);
+      e = shard ? launch_nll_partials(part, tl, s, shard->partials, st, &launches)
+                : launch_nll_combine(part, tl, targets, s, nll, ds->err, st, &launches);
   }
   cudaFreeAsync(base, st);
   if (e != cudaSuccess) return ARCHEAD_ERR_CUDA;
@@ -152,19 +170,19 @@ int run_dec(const uint16_t* H, const archead_head* head, float* Y, const int32_t
 }
 
 int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* targets,
-        float* nll, const Shapes& s, cudaStream_t st) {
+        float* nll, const Shapes& s, cudaStream_t st, const NllShard* shard = nullptr) {
   DeviceState* ds;
   int rc = current_state(&ds);
   if (rc) return rc;
   int launches = 0;
   const int RR = s.r_c + s.r_r;
-  const bool nll_mode = nll != nullptr;
+  const bool nll_mode = nll != nullptr || shard != nullptr;
   // N <= 8 on the warp-MMA kernel (one token block), larger N on the tensor-memory
   // (tcgen05) kernel when its shared-memory rings fit the shape; both have a fused
   // split-vocabulary NLL epilogue
   // N <= 16: the persistent decode kernel with H resident in shared memory, when it fits
   const DecPlan dplan = dec_plan(s, nll_mode);
-  if (dplan.nt8 > 0) return run_dec(H, head, Y, targets, nll, s, dplan, ds, st);
+  if (dplan.nt8 > 0) return run_dec(H, head, Y, targets, nll, s, dplan, ds, st, shard);
   const TcPlan plan = s.N > 8 ? tc_plan(s, nll_mode) : TcPlan{0, 0, 0, 0};
   const bool use_tc = plan.nt > 0;
   const int64_t tb = use_tc ? plan.nt : residual_token_block(s.N);
@@ -180,6 +198,7 @@ int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* ta
   const size_t split_bytes = use_tc ? tc_split_scratch_bytes(s, plan) : 0;
   const size_t o_scr = split_bytes ? cv.take(split_bytes) : 0;
   const size_t o_cnt = split_bytes ? cv.take((size_t)((s.V + 127) / 128) * 4) : 0;
+  const size_t o_tloc = shard ? cv.take((size_t)s.N * 4) : 0;
   void* base = nullptr;
   if (cudaMallocFromPoolAsync(&base, cv.off, ds->pool, st) != cudaSuccess) {
     cudaGetLastError();
@@ -190,18 +209,26 @@ int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* ta
   float* scr = split_bytes ? reinterpret_cast<float*>(b + o_scr) : nullptr;
   unsigned* cnt = split_bytes ? reinterpret_cast<unsigned*>(b + o_cnt) : nullptr;
   float* t = reinterpret_cast<float*>(b + o_t);
-  cudaError_t e = use_tc ? launch_prologue_blocked(H, head, s, plan, Hh, cnt, ds->err, st, &launches)
-                         : launch_prologue(H, head, s, Npad, Hh, t, ds->err, st, &launches);
+  int32_t* tloc = shard ? reinterpret_cast<int32_t*>(b + o_tloc) : nullptr;
+  cudaError_t e = cudaSuccess;
+  if (shard)  // shard-local targets and zeroed target logits, before the prologue
+    e = launch_nll_shard_prep(targets, s.N, shard->v_begin, s.V, shard->v_total, tloc,
+                              reinterpret_cast<float*>(b + o_tl), ds->err, st, &launches);
+  const int32_t* tg = shard ? tloc : targets;
+  if (e == cudaSuccess)
+    e = use_tc ? launch_prologue_blocked(H, head, s, plan, Hh, cnt, ds->err, st, &launches)
+               : launch_prologue(H, head, s, Npad, Hh, t, ds->err, st, &launches);
   if (e == cudaSuccess) {
     if (use_tc) {
       float2* part = nll_mode ? reinterpret_cast<float2*>(b + o_part) : nullptr;
       float* tl = nll_mode ? reinterpret_cast<float*>(b + o_tl) : nullptr;
       prof_mark(0, st);
-      e = launch_residual_tc(Hh, head, s, plan, nll_mode ? nullptr : Y, targets, part, tl, scr,
-                             cnt, ds->err, st, &launches);
+      e = launch_residual_tc(Hh, head, s, plan, nll_mode ? nullptr : Y, tg, part, tl, scr, cnt,
+                             ds->err, st, &launches);
       prof_mark(1, st);
       if (e == cudaSuccess && nll_mode)
-        e = launch_nll_combine(part, tl, targets, s, nll, ds->err, st, &launches);
+        e = shard ? launch_nll_partials(part, tl, s, shard->partials, st, &launches)
+                  : launch_nll_combine(part, tl, targets, s, nll, ds->err, st, &launches);
     } else if (!nll_mode) {
       prof_mark(0, st);
       e = launch_residual_gemm(Hh, t, head, s, Y, nullptr, nullptr, nullptr, st, &launches, 0);
@@ -210,9 +237,11 @@ int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* ta
       float2* part = reinterpret_cast<float2*>(b + o_part);
       float* tl = reinterpret_cast<float*>(b + o_tl);
       prof_mark(0, st);
-      e = launch_residual_gemm(Hh, t, head, s, nullptr, targets, part, tl, st, &launches, 1);
+      e = launch_residual_gemm(Hh, t, head, s, nullptr, tg, part, tl, st, &launches, 1);
       prof_mark(1, st);
-      if (e == cudaSuccess) e = launch_nll_combine(part, tl, targets, s, nll, ds->err, st, &launches);
+      if (e == cudaSuccess)
+        e = shard ? launch_nll_partials(part, tl, s, shard->partials, st, &launches)
+                  : launch_nll_combine(part, tl, targets, s, nll, ds->err, st, &launches);
     }
   }
   cudaFreeAsync(base, st);
@@ -289,6 +318,39 @@ int archead_nll(const uint16_t* H, const archead_head* head, const int32_t* targ
   if (!aligned(H, 16) || !aligned(targets, 4) || !aligned(nll_out, 4)) return ARCHEAD_ERR_ALIGN;
   return run(H, head, nullptr, targets, nll_out, make_shapes(N, V, D, r_c, r_r, g),
              static_cast<cudaStream_t>(stream));
+}
+
+int archead_nll_partials(const uint16_t* H, const archead_head* head, const int32_t* targets,
+                         int64_t v_begin, int64_t v_total, float* partials, int64_t N,
+                         int64_t V, int64_t D, int r_c, int r_r, int g, void* stream) {
+  int rc = check_head(head, N, V, D, r_c, r_r, g);
+  if (rc) return rc;
+  if (v_begin < 0 || v_total < V || v_begin > v_total - V || v_total > 0x7fffffffLL)
+    return ARCHEAD_ERR_SHAPE;
+  if (N == 0) {
+    t_last_launches = 0;
+    return ARCHEAD_OK;
+  }
+  if (!H || !targets || !partials) return ARCHEAD_ERR_NULLPTR;
+  if (!aligned(H, 16) || !aligned(targets, 4) || !aligned(partials, 4)) return ARCHEAD_ERR_ALIGN;
+  const NllShard shard = {v_begin, v_total, partials};
+  return run(H, head, nullptr, targets, nullptr, make_shapes(N, V, D, r_c, r_r, g),
+             static_cast<cudaStream_t>(stream), &shard);
+}
+
+int archead_nll_merge(const float* partials, int G, int64_t N, float* nll_out, void* stream) {
+  if (N < 0 || N > 0x7fffffffLL || G < 1 || G > 65536) return ARCHEAD_ERR_SHAPE;
+  if (N == 0) {
+    t_last_launches = 0;
+    return ARCHEAD_OK;
+  }
+  if (!partials || !nll_out) return ARCHEAD_ERR_NULLPTR;
+  if (!aligned(partials, 4) || !aligned(nll_out, 4)) return ARCHEAD_ERR_ALIGN;
+  if (launch_nll_merge(partials, G, N, nll_out, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return ARCHEAD_ERR_CUDA;
+  t_last_launches = 1;
+  return ARCHEAD_OK;
 }
 
 int archead_logits_host(const uint16_t* H_host, const archead_head* head, float* Y_host,

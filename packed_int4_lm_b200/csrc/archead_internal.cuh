@@ -205,6 +205,19 @@ cudaError_t launch_nll_combine(const float2* part, const float* tlogit,
                                const int32_t* targets, const Shapes& s, float* nll,
                                unsigned* err, cudaStream_t st, int* launches);
 
+// Vocabulary-parallel NLL (csrc/nll_shard.cu).  A shard holds rows [v_begin, v_begin + V)
+// of a head with v_total rows.  prep: shard-local targets (t - v_begin, or -1 when another
+// shard owns the row) into tloc[N] and zeroed target logits; targets outside [0, v_total)
+// set kErrTarget.  partials: the shard's (max, sum exp, target logit) per token, out[N][3].
+// merge: nll[n] from G shard triples [G][N][3], combined in shard order.
+cudaError_t launch_nll_shard_prep(const int32_t* targets, int64_t N, int64_t v_begin,
+                                  int64_t V, int64_t v_total, int32_t* tloc, float* tlogit,
+                                  unsigned* err, cudaStream_t st, int* launches);
+cudaError_t launch_nll_partials(const float2* part, const float* tlogit, const Shapes& s,
+                                float* out, cudaStream_t st, int* launches);
+cudaError_t launch_nll_merge(const float* partials, int G, int64_t N, float* nll,
+                             cudaStream_t st);
+
 cudaError_t launch_repack(const uint8_t* canon, uint8_t* dev, int64_t V, int64_t D,
                           cudaStream_t st);
 

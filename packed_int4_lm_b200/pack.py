@@ -239,3 +239,22 @@ def storage_ratio(head: dict) -> float:
     nb = sum(np.asarray(head[k]).nbytes for k in
              ("r_nib", "r_code", "r_super", "Ac", "sAc", "Bc", "sBc", "Aw", "sAw", "Bw", "sBw"))
     return nb / (2.0 * head["V"] * head["D"])
+
+
+# V-indexed arrays of the canonical head (rows of the vocabulary); the B factors and their
+# scales are indexed by factor and column and are shared by every row.
+_ROW_KEYS = ("r_nib", "r_code", "r_super", "Ac", "sAc", "Aw", "sAw")
+
+
+def shard_rows(head: dict, v0: int, v1: int) -> dict:
+    """Rows [v0, v1) of a canonical packed head: the vocabulary shard one GPU holds when
+    the logits or the NLL are evaluated vocabulary-parallel.  The row-indexed arrays are
+    sliced and the B factors shared; the result is a canonical head with V = v1 - v0."""
+    V = int(head["V"])
+    if not 0 <= v0 < v1 <= V:
+        raise ValueError(f"row range [{v0}, {v1}) outside [0, {V})")
+    out = dict(head)
+    out["V"] = v1 - v0
+    for k in _ROW_KEYS:
+        out[k] = np.ascontiguousarray(head[k][v0:v1])
+    return out

@@ -32,7 +32,7 @@ def _rank(rank, world, port, local_ms, out):
 def test_two_gloo_ranks_report_the_slowest_rank():
     world, port = 2, _free_port()
     local_ms = [120.0, 150.0]
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_rank, args=(world, port, local_ms, out), nprocs=world, join=True)
         res = dict(out)
