@@ -90,3 +90,25 @@ def test_nll_and_other_entry_validation(L):
                              None) == E["ARCHEAD_ERR_SHAPE"]
     assert L.archead_logits_host(0x9000000, ctypes.byref(h), 0xA000000, 4, 1000, 512, 4, 4, 16,
                                  None) == E["ARCHEAD_ERR_SHAPE"]
+
+
+def test_vocab_parallel_entry_validation(L):
+    h = _fake_head()  # a 1000-row shard
+
+    def part(v_begin, v_total, N=4, targets=0xB000000, out=0xC000000):
+        return L.archead_nll_partials(0x9000000, ctypes.byref(h), targets, v_begin, v_total,
+                                      out, N, 1000, 512, 4, 4, 64, None)
+
+    assert part(-1, 5000) == E["ARCHEAD_ERR_SHAPE"]          # v_begin < 0
+    assert part(0, 999) == E["ARCHEAD_ERR_SHAPE"]            # shard larger than the head
+    assert part(4001, 5000) == E["ARCHEAD_ERR_SHAPE"]        # shard past the end
+    assert part(0, 1 << 31) == E["ARCHEAD_ERR_SHAPE"]        # ids beyond int32
+    assert part(4000, 5000, N=0) == E["ARCHEAD_OK"]          # N = 0: no-op
+    assert part(0, 5000, targets=0) == E["ARCHEAD_ERR_NULLPTR"]
+    assert part(0, 5000, out=0xC000002) == E["ARCHEAD_ERR_ALIGN"]
+    assert L.archead_nll_merge(0xC000000, 0, 4, 0xD000000, None) == E["ARCHEAD_ERR_SHAPE"]
+    assert L.archead_nll_merge(0xC000000, 70000, 4, 0xD000000, None) == E["ARCHEAD_ERR_SHAPE"]
+    assert L.archead_nll_merge(0xC000000, 2, -1, 0xD000000, None) == E["ARCHEAD_ERR_SHAPE"]
+    assert L.archead_nll_merge(0xC000000, 2, 0, 0xD000000, None) == E["ARCHEAD_OK"]
+    assert L.archead_nll_merge(None, 2, 4, 0xD000000, None) == E["ARCHEAD_ERR_NULLPTR"]
+    assert L.archead_nll_merge(0xC000001, 2, 4, 0xD000000, None) == E["ARCHEAD_ERR_ALIGN"]
