@@ -178,3 +178,34 @@ def test_storage_matched_baselines_on_tiny_head():
     e_full, e_naive, e_core = rel_err(full), rel_err(naive), rel_err(core)
     assert e_full < 0.6 * e_naive, (e_full, e_naive)
     assert e_full < 0.6 * e_core, (e_full, e_core)
+
+
+def test_agreement_with_the_dense_head_on_tiny_head():
+    """Top-k agreement and KL(dense || packed) of the next-token distributions on held-out
+    activations of the tiny synthetic head, the pages' agreement measures, for the full
+    construction and the two storage-matched baselines (fp64 oracle logits).  Measured:
+    KL 0.0018 / 0.0074 / 0.0096 nats, top-5 agreement 0.91 / 0.85 / 0.84."""
+    w = WORKLOADS["tiny"]
+    W = make_weight(w.V, w.D, w.rank, w.sigma0, w.noise, w.seed_w)
+    s = make_channel_scales(w.D, w.sigma_s, w.n_outliers, w.outlier_mult, w.seed_scales)
+    Hc = make_hidden(w.n_cal, s, w.seed_hcal)
+    Hb = bf16_bits(make_hidden(128, s, 99))
+    Yd = oracle.bf16_bits_to_f64(Hb) @ W.double().numpy().T
+
+    def log_softmax(Z):
+        Z = Z - Z.max(axis=1, keepdims=True)
+        return Z - np.log(np.exp(Z).sum(axis=1, keepdims=True))
+
+    def measures(head):
+        Y = oracle.logits(head, Hb)
+        pd, pp = log_softmax(Yd), log_softmax(Y)
+        kl = float(np.mean((np.exp(pd) * (pd - pp)).sum(axis=1)))
+        a, b = np.argsort(-Y, axis=1)[:, :5], np.argsort(-Yd, axis=1)[:, :5]
+        top5 = float(np.mean([len(set(a[i]) & set(b[i])) / 5 for i in range(len(a))]))
+        return kl, top5
+
+    kl_f, t5_f = measures(pack.build_head(W, Hc, w.r_c, w.r_r, w.g, w.p, w.lam, seed=w.seed_rsvd))
+    kl_n, t5_n = measures(pack.build_head(W, Hc, 0, 0, 32, w.p, w.lam, seed=w.seed_rsvd))
+    kl_c, t5_c = measures(pack.build_head(W, Hc, w.r_c, 0, w.g, w.p, w.lam, seed=w.seed_rsvd))
+    assert kl_f < 0.5 * kl_n and kl_f < 0.5 * kl_c, (kl_f, kl_n, kl_c)
+    assert t5_f > t5_n and t5_f > t5_c, (t5_f, t5_n, t5_c)
