@@ -26,10 +26,10 @@
  *    the split-tile partials and counters, the NLL partials) is taken with
  *    cudaMallocAsync from a library-owned pool on `stream` and returned with
  *    cudaFreeAsync on the same stream.
- *  - Limits: g in {32, 64, 128, 256}; D % 128 == 0 and D % g == 0; 0 <= r_c, r_r <= 128;
- *    1 <= V <= 8388480 (65535 blocks of 128 rows); 0 <= N < 2^31; N == 0 is a successful
- *    no-op.  V needs no multiple of
- *    any tile: the vocabulary tail is predicated.
+ *  - Limits: g in {32, 64, 128, 256}; 128 <= D <= 2^20, D % 128 == 0 and D % g == 0;
+ *    0 <= r_c, r_r <= 128; 1 <= V <= 8388480 (65535 blocks of 128 rows); 0 <= N < 2^31;
+ *    N == 0 is a successful no-op.  V needs no multiple of any tile: the vocabulary tail
+ *    is predicated.
  *  - |H| must stay within the FP16 range (|h| <= 65504); larger or non-finite entries
  *    raise ARCHEAD_ERR_RANGE_H (see archead_logits).  Where the rank terms run on the
  *    tensor cores (r_c and r_r multiples of 16 for N <= 16; every shape for N > 16) the
@@ -224,7 +224,9 @@ int archead_last_launches(void);
  *   until the process exits; larger requests return ARCHEAD_ERR_SHAPE before anything is
  *   enqueued (e.g. D = 4096 allows N <= 192 with r_c + r_r = 64).
  *   The first call on a device looks up that array's device address (cudaGetSymbolAddress)
- *   with the device current; make that first call before any stream capture.
+ *   with the device current; make that first call before any stream capture.  The address
+ *   is kept for the life of the process: after cudaDeviceReset on a device, do not call
+ *   this entry point (or any other of this library) on that device again.
  *   All calls share the one array: calls whose kernels overlap on the GPU (different
  *   streams, or several host threads) race on it and must be serialised by the caller.
  *   Each call writes every scratch byte before reading it, so no clearing is needed.

@@ -75,7 +75,8 @@ int check_head(const archead_head* h, int64_t N, int64_t V, int64_t D, int r_c, 
   if (h->V != V || h->D != D || h->r_c != r_c || h->r_r != r_r || h->g != g)
     return ARCHEAD_ERR_SHAPE;
   // V: the residual kernel's grid.y holds one 128-row vocabulary block each (<= 65535)
-  if (N < 0 || N > 0x7fffffffLL || V < 1 || V > 65535LL * 128 || D < 128 || D % 128 != 0)
+  if (N < 0 || N > 0x7fffffffLL || V < 1 || V > 65535LL * 128 || D < 128 || D % 128 != 0 ||
+      D > (1LL << 20))
     return ARCHEAD_ERR_SHAPE;
   if (!(g == 32 || g == 64 || g == 128 || g == 256) || D % g != 0) return ARCHEAD_ERR_SHAPE;
   if (r_c < 0 || r_c > 128 || r_r < 0 || r_r > 128) return ARCHEAD_ERR_SHAPE;
@@ -177,10 +178,10 @@ int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* ta
   int launches = 0;
   const int RR = s.r_c + s.r_r;
   const bool nll_mode = nll != nullptr || shard != nullptr;
-  // N <= 8 on the warp-MMA kernel (one token block), larger N on the tensor-memory
-  // (tcgen05) kernel when its shared-memory rings fit the shape; both have a fused
-  // split-vocabulary NLL epilogue
-  // N <= 16: the persistent decode kernel with H resident in shared memory, when it fits
+  // N <= 16: the persistent decode kernel with H resident in shared memory, when its plan
+  // fits; larger N: the tensor-memory (tcgen05) kernel when its shared-memory rings fit;
+  // other shapes: the token-block warp-MMA kernel.  All three have a fused
+  // split-vocabulary NLL epilogue.
   const DecPlan dplan = dec_plan(s, nll_mode);
   if (dplan.nt8 > 0) return run_dec(H, head, Y, targets, nll, s, dplan, ds, st, shard);
   const TcPlan plan = s.N > 8 ? tc_plan(s, nll_mode) : TcPlan{0, 0, 0, 0};

@@ -38,9 +38,15 @@ int device_setup(NoAllocDevice** out) {
   NoAllocDevice& d = g_devs[dev];
   if (!d.ready) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return ARCHEAD_ERR_CUDA;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
+      cudaGetLastError();  // do not leave the failure for the caller's next error check
+      return ARCHEAD_ERR_CUDA;
+    }
     unsigned* e = error_word_address();
-    if (!e) return ARCHEAD_ERR_CUDA;
+    if (!e) {
+      cudaGetLastError();
+      return ARCHEAD_ERR_CUDA;
+    }
     d.scratch = static_cast<unsigned char*>(p);
     d.err = e;
     d.ready = true;
@@ -67,9 +73,13 @@ extern "C" int archead_logits_noalloc(const uint16_t* H, const archead_head* hea
     return ARCHEAD_ERR_ALIGN;
   const int64_t tb = residual_token_block(N);
   const int64_t Npad = (N + tb - 1) / tb * tb;
+  // beyond the fixed scratch: rejected before any product is formed, so no size wraps
+  const int64_t cap = (int64_t)kScratchBytes;
+  if (D > cap / 2 || Npad > cap / 2 / D || N > cap / 4 / (r_c + r_r + 1))
+    return ARCHEAD_ERR_SHAPE;
   const size_t hh_bytes = round256((size_t)Npad * D * 2);
   const size_t t_bytes = round256((size_t)N * (r_c + r_r) * 4 + 16);
-  if (hh_bytes + t_bytes > kScratchBytes) return ARCHEAD_ERR_SHAPE;  // beyond the fixed scratch
+  if (hh_bytes + t_bytes > kScratchBytes) return ARCHEAD_ERR_SHAPE;
   NoAllocDevice* d = nullptr;
   rc = device_setup(&d);
   if (rc) return rc;

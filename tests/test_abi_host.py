@@ -71,6 +71,7 @@ def test_validation_errors(L):
     nul = _fake_head()
     nul.Bw = 0
     assert _logits(L, nul) == E["ARCHEAD_ERR_NULLPTR"]
+    assert _logits(L, _fake_head(D=(1 << 20) + 128)) == E["ARCHEAD_ERR_SHAPE"]  # D > 2^20
     zero_rank = _fake_head(r_r=0)
     zero_rank.Aw = zero_rank.sAw = zero_rank.Bw = zero_rank.sBw = 0
     assert _logits(L, zero_rank, N=0) == E["ARCHEAD_OK"]            # N = 0: no-op
@@ -112,3 +113,16 @@ def test_vocab_parallel_entry_validation(L):
     assert L.archead_nll_merge(0xC000000, 2, 0, 0xD000000, None) == E["ARCHEAD_OK"]
     assert L.archead_nll_merge(None, 2, 4, 0xD000000, None) == E["ARCHEAD_ERR_NULLPTR"]
     assert L.archead_nll_merge(0xC000001, 2, 4, 0xD000000, None) == E["ARCHEAD_ERR_ALIGN"]
+
+
+def test_noalloc_rejects_sizes_beyond_its_scratch_before_any_product(L):
+    """archead_logits_noalloc checks the request against its fixed 2 MiB array before it
+    forms any byte count, so a huge D or N cannot wrap a size and pass the check."""
+    def na(h, N):
+        return L.archead_logits_noalloc(0x9000000, ctypes.byref(h), 0xA000000, N, h.V, h.D,
+                                        h.r_c, h.r_r, h.g, None)
+    assert na(_fake_head(D=1 << 62), 4) == E["ARCHEAD_ERR_SHAPE"]
+    assert na(_fake_head(D=1 << 20), 4) == E["ARCHEAD_ERR_SHAPE"]     # 8 x 2^20 x 2 B > 2 MiB
+    assert na(_fake_head(D=4096), (1 << 31) - 1) == E["ARCHEAD_ERR_SHAPE"]
+    assert na(_fake_head(D=4096, r_c=32, r_r=32), 256) == E["ARCHEAD_ERR_SHAPE"]
+    assert na(_fake_head(), 0) == E["ARCHEAD_OK"]

@@ -157,6 +157,44 @@ def test_nll_random_head(dev, nhead, N):
     assert err <= NLL_TOL, err
 
 
+_WIDE_GROUP_HEADS = {}
+
+
+def _wide_group_head(dev, g, r_c, r_r):
+    """A logit-regime head with one group code per 128 columns or fewer (g >= 128): the
+    decode kernel's raw-nibble path (H / 16 on half of the columns, the per-block offset
+    taken off through the chain's start value, the code applied to the FP32 block sum)."""
+    key = (g, r_c, r_r)
+    if key not in _WIDE_GROUP_HEADS:
+        head = random_canonical_head(1000, 1024, r_c, r_r, g, seed=60 + g + r_c, zero_rows=3,
+                                     zero_groups=20, super_exp_range=(-17, -13),
+                                     factor_exp_range=(-13, -10))
+        _WIDE_GROUP_HEADS[key] = (head, ah.DeviceHead.from_canonical(head, dev))
+    return _WIDE_GROUP_HEADS[key]
+
+
+@pytest.mark.parametrize("g,r_c,r_r", [(128, 16, 16), (256, 16, 16), (128, 5, 3)])
+@pytest.mark.parametrize("N", [1, 4, 8, 9, 16])
+def test_nll_decode_kernel_one_code_per_block(dev, g, r_c, r_r, N):
+    """Fused NLL on the decode kernel (N <= 16) with g >= 128, element by element against
+    the oracle at 1e-3 nats; rank terms on warp MMAs (ranks multiples of 16) and in FP32
+    (5 and 3).  The logits of the same calls are checked too."""
+    head, dh = _wide_group_head(dev, g, r_c, r_r)
+    H = _rand_H(N, 1024, 700 + N + g)
+    Yref = oracle.logits(head, bf16_bits(H))
+    rms = np.sqrt(np.mean(Yref ** 2))
+    assert 0.5 < rms < 20, rms  # the language-model logit regime
+    tg = make_targets(N, head["V"], 800 + N)
+    out = ah.nll(H.to(dev), dh, tg.to(dev))
+    ah.check()
+    ref = oracle.nll_from_logits(Yref, tg.numpy())
+    err = np.max(np.abs(out.cpu().double().numpy() - ref))
+    assert err <= NLL_TOL, (g, N, err)
+    Y = ah.logits(H.to(dev), dh)
+    ah.check()
+    _assert_logits(Y.cpu().numpy(), Yref, f"g={g} N={N}")
+
+
 def test_many_items_per_cta_consistent(dev):
     """A vocabulary large enough that every persistent CTA of the tensor-memory kernel runs
     several 128-row tiles, repeated: the first 16 tokens of N = 64 and N = 32 calls must
@@ -328,11 +366,19 @@ def test_workload_qwen_decode_and_prefill(dev):
     Hfull = make_hidden(4096, s, w.seed_heval)           # prefill batch; decode uses its prefix
     sample = np.array([0, 1, 2, 3, 15, 63, 64, 1000, 2047, 4095])
     Yref = oracle.logits(head, bf16_bits(Hfull[sample]))
+    tg = make_targets(4096, w.V, w.seed_targets)
     for N in w.Ns:
         Y = ah.logits(Hfull[:N].to(dev), dh)
         ah.check()
         rows = [i for i, r in enumerate(sample) if r < N]
         _assert_logits(Y.cpu().numpy()[sample[rows]], Yref[rows], f"decode N={N}")
+        # fused NLL of the same batch (N <= 16: the decode kernel's g = 128 raw-nibble
+        # path), at the sampled tokens
+        out = ah.nll(Hfull[:N].to(dev), dh, tg[:N].to(dev))
+        ah.check()
+        ref = oracle.nll_from_logits(Yref[rows], tg.numpy()[sample[rows]])
+        err = np.max(np.abs(out.cpu().double().numpy()[sample[rows]] - ref))
+        assert err <= NLL_TOL, (N, err)
     Y = ah.logits(Hfull.to(dev), dh)
     ah.check()
     _assert_logits(Y[torch.from_numpy(sample).to(dev)].cpu().numpy(), Yref, "prefill N=4096")

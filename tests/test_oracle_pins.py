@@ -249,3 +249,18 @@ def test_brute_force_loops_on_a_tiny_head():
             Y[n, v] = acc
     Yo = oracle.logits(head, Hb)
     assert np.max(np.abs(Yo - Y)) <= 1e-12 * max(1.0, np.max(np.abs(Y)))
+
+
+@pytest.mark.parametrize("V,D,r_c,r_r,g", [(1000, 512, 8, 8, 64), (300, 1024, 0, 0, 128),
+                                           (257, 256, 3, 0, 32), (129, 512, 1, 7, 256)])
+def test_packed_nbytes_closed_form(V, D, r_c, r_r, g):
+    """Sec. 3 storage: the serialised module holds the INT4 residual (half a byte per
+    entry), one UINT8 code per g entries, one BF16 super-scale per row, the INT8 factors
+    (V + D)(r_c + r_r) bytes, an FP32 scale per factor row of A and per g entries of a row
+    of B -- and no dense head."""
+    head = random_canonical_head(V, D, r_c, r_r, g, seed=V)
+    closed = (V * D // 2 + V * D // g + 2 * V + (V + D) * (r_c + r_r)
+              + 4 * (2 * V + (r_c + r_r) * D // g))
+    assert oracle.packed_nbytes(head) == closed
+    # against the dense BF16 head: INT4 plus its code and super-scale overheads
+    assert oracle.packed_nbytes(head) < 2 * V * D
