@@ -196,62 +196,86 @@ __device__ __forceinline__ void dec_convert_h(const uint16_t* __restrict__ H,
 }
 
 // t[n, j] = sum_d h[n, d] fl32(B[j, d] s[j, d / g]) for the N <= 16 tokens of this path,
-// B = [Q8(B_c) | Q8(B_w)]: one block per factor index j, 256 threads striding over D.
+// B = [Q8(B_c) | Q8(B_w)], on warp MMAs: block f computes the factors 16 f .. 16 f + 15 for
+// all tokens, warp w the K range [w D / 8, (w + 1) D / 8).  Per 16-column step the INT8
+// factor bytes (exact in FP16) meet the FP16 hidden states in one m16n8k16 MMA per token
+// block, and the step's FP32 result is scaled by the factor's group scale s[j, d / g]: t is
+// sum over groups of s_jk sum_{d in k} q_jd h_nd, the product fl32(q s) h of the dequantised
+// factor up to the rounding of that one product.  The warps' sums are added in a fixed order.
 __device__ __forceinline__ void dec_lowrank_t(const uint16_t* __restrict__ H,
                                               const int8_t* __restrict__ Bc,
                                               const float* __restrict__ sBc,
                                               const int8_t* __restrict__ Bw,
                                               const float* __restrict__ sBw, int r_c, int r_r,
                                               int64_t N, int64_t D, int g, float* __restrict__ t,
-                                              int j) {
+                                              int fb) {
   const int RR = r_c + r_r;
-  const int8_t* B = j < r_c ? Bc + (int64_t)j * D : Bw + (int64_t)(j - r_c) * D;
-  const float* sB = j < r_c ? sBc + (int64_t)j * (D / g) : sBw + (int64_t)(j - r_c) * (D / g);
-  float acc[16];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gid = lane >> 2, tq = lane & 3;
+  const int64_t G = D / g;
+  const int8_t* qr[2];
+  const float* sr[2];
 #pragma unroll
-  for (int n = 0; n < 16; ++n) acc[n] = 0.f;
-  for (int64_t d0 = threadIdx.x * 8; d0 < D; d0 += 256 * 8) {
-    const uint2 braw = *reinterpret_cast<const uint2*>(B + d0);
-    const float sc = sB[d0 / g];
-    const int8_t* bq = reinterpret_cast<const int8_t*>(&braw);
-    float b[8];
+  for (int h = 0; h < 2; ++h) {
+    const int j = 16 * fb + gid + 8 * h;
+    qr[h] = j < r_c ? Bc + (int64_t)j * D : (j < RR ? Bw + (int64_t)(j - r_c) * D : nullptr);
+    sr[h] = j < r_c ? sBc + (int64_t)j * G : (j < RR ? sBw + (int64_t)(j - r_c) * G : nullptr);
+  }
+  const __half2 k1152 = __float2half2_rn(1152.f);
+  float acc[2][4];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) b[k] = __fmul_rn((float)bq[k], sc);
+  for (int b = 0; b < 2; ++b) acc[b][0] = acc[b][1] = acc[b][2] = acc[b][3] = 0.f;
+  const int64_t kw = D / 8;
+  for (int64_t k0 = warp * kw; k0 < (warp + 1) * kw; k0 += 16) {
+    // A: the factor rows gid (h = 0) and gid + 8 (h = 1), bytes k0 + 4 tq .. + 3 as the K
+    // slots 2 tq, 2 tq + 1 (bytes 0, 1) and 2 tq + 8, 2 tq + 9 (bytes 2, 3)
+    uint32_t a[4];
+    float sc[2];
 #pragma unroll
-    for (int n = 0; n < 16; ++n) {
-      if (n < N) {
-        const uint4 hv = *reinterpret_cast<const uint4*>(H + n * D + d0);
-        const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
-        float a = acc[n];
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t w =
+          qr[h] ? __ldg(reinterpret_cast<const unsigned int*>(qr[h] + k0 + 4 * tq)) ^ 0x80808080u
+                : 0x80808080u;
+      // bytes b + 128 under the FP16 pattern 0x6400 read 1024 + b + 128: minus 1152
+      uint32_t q0 = __byte_perm(w, 0x64646464u, 0x5140), q1 = __byte_perm(w, 0x64646464u, 0x7352);
+      a[h] = h2_bits(__hsub2(*reinterpret_cast<__half2*>(&q0), k1152));
+      a[2 + h] = h2_bits(__hsub2(*reinterpret_cast<__half2*>(&q1), k1152));
+      sc[h] = sr[h] ? __ldg(sr[h] + k0 / g) : 0.f;
+    }
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          a = fmaf(__uint_as_float(hw[k] << 16), b[2 * k], a);
-          a = fmaf(__uint_as_float(hw[k] & 0xFFFF0000u), b[2 * k + 1], a);
-        }
-        acc[n] = a;
-      }
+    for (int b = 0; b < 2; ++b) {  // token blocks 0..7, 8..15
+      const int64_t n = 8 * b + gid;
+      uint2 hb = make_uint2(0u, 0u);
+      if (n < N) hb = __ldg(reinterpret_cast<const uint2*>(H + n * D + k0 + 4 * tq));
+      const __half2 b0 = __floats2half2_rn(__uint_as_float(hb.x << 16), __uint_as_float(hb.x & 0xFFFF0000u));
+      const __half2 b1 = __floats2half2_rn(__uint_as_float(hb.y << 16), __uint_as_float(hb.y & 0xFFFF0000u));
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
+      mma_f16_16816(d, a, h2_bits(b0), h2_bits(b1));
+      acc[b][0] = fmaf(sc[0], d[0], acc[b][0]);
+      acc[b][1] = fmaf(sc[0], d[1], acc[b][1]);
+      acc[b][2] = fmaf(sc[1], d[2], acc[b][2]);
+      acc[b][3] = fmaf(sc[1], d[3], acc[b][3]);
     }
   }
-  __shared__ float red[8][16];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  // accumulator: row gid (+ 8) = factor, column 2 tq (+ 1) = token of the block
+  __shared__ float red[8][16][17];
 #pragma unroll
-  for (int n = 0; n < 16; ++n) {
-    float v = acc[n];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0) red[warp][n] = v;
+  for (int b = 0; b < 2; ++b) {
+    red[warp][gid][8 * b + 2 * tq] = acc[b][0];
+    red[warp][gid][8 * b + 2 * tq + 1] = acc[b][1];
+    red[warp][gid + 8][8 * b + 2 * tq] = acc[b][2];
+    red[warp][gid + 8][8 * b + 2 * tq + 1] = acc[b][3];
   }
   __syncthreads();
-  if ((int64_t)threadIdx.x < N) {
-    float v = 0.f;
+  const int row = threadIdx.x >> 4, n = threadIdx.x & 15;  // 256 = 16 factors x 16 tokens
+  float v = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) v += red[w][threadIdx.x];
-    t[(int64_t)threadIdx.x * RR + j] = v;
-  }
+  for (int w = 0; w < 8; ++w) v += red[w][row][n];
+  const int j = 16 * fb + row;
+  if (j < RR && n < N) t[(int64_t)n * RR + j] = v;
 }
 
 // The whole prologue of this path in one launch: blocks [0, nconv) build the H image, its
-// corrections and the zeroed counters; the next r_c + r_r blocks form t.
+// corrections and the zeroed counters; the next ceil((r_c + r_r) / 16) blocks form t.
 __global__ void __launch_bounds__(256) dec_prologue_kernel(
     const uint16_t* __restrict__ H, __half* __restrict__ img, int64_t N, int ntok, int64_t D,
     int scale_b, unsigned* __restrict__ counters, int64_t n_counters, int nconv,
@@ -895,13 +919,13 @@ cudaError_t launch_dec_prologue(const uint16_t* H, const archead_head* head, con
   const int64_t ntok = 8 * pl.nt8;
   const int64_t n_counters = (s.V + 127) / 128;
   // one warp per (token, 128-column block), the counters on the same blocks; then one
-  // block per factor index for t
+  // block per 16 factors for t
   int64_t blocks = (ntok * (s.D / 128) * 32 + 255) / 256;
   const int64_t cb = (n_counters + 255) / 256;
   if (cb > blocks) blocks = cb;
   if (blocks > 148 * 8) blocks = 148 * 8;
   const int RR = s.r_c + s.r_r;
-  dec_prologue_kernel<<<(unsigned)(blocks + RR), 256, 0, st>>>(
+  dec_prologue_kernel<<<(unsigned)(blocks + (RR + 15) / 16), 256, 0, st>>>(
       H, img, s.N, (int)ntok, s.D, s.g >= 128 ? 1 : 0, counters, n_counters, (int)blocks,
       head->Bc, head->sBc, head->Bw, head->sBw, s.r_c, s.r_r, s.g, t, err);
   ++*launches;

@@ -36,7 +36,8 @@ import numpy as np
 import torch
 
 __all__ = ["build_head", "q8_rowwise", "q8_groupwise", "sc4", "pack_nibbles",
-           "metric_transform", "randomized_svd", "dequant_head_torch", "storage_ratio"]
+           "metric_transform", "randomized_svd", "dequant_head_torch", "storage_ratio",
+           "save_head", "load_head", "serialized_nbytes", "shard_rows"]
 
 
 def _rne(x: torch.Tensor) -> torch.Tensor:
@@ -258,3 +259,76 @@ def shard_rows(head: dict, v0: int, v1: int) -> dict:
     for k in _ROW_KEYS:
         out[k] = np.ascontiguousarray(head[k][v0:v1])
     return out
+
+
+# ---------------------------------------------------------------------------------------
+# The serialised module (Sec. 3: storage is measured over every parameter and buffer the
+# serialised module holds).  File layout, little-endian:
+#   8 bytes   magic b"ARCHEAD1"
+#   8 bytes   uint64 length L of the JSON header
+#   L bytes   JSON: {"meta": {V, D, r_c, r_r, g}, "arrays": [[key, dtype, shape, offset,
+#             nbytes], ...]}, offsets counted from the start of the data section
+#   padding   to a multiple of 16 bytes, then the data section: every array's raw bytes
+#             (C order), each starting on a 16-byte boundary
+# Loading returns arrays whose bytes equal the saved ones.
+# ---------------------------------------------------------------------------------------
+_MAGIC = b"ARCHEAD1"
+_HEAD_KEYS = ("r_nib", "r_code", "r_super", "Ac", "sAc", "Bc", "sBc", "Aw", "sAw", "Bw", "sBw")
+_META_KEYS = ("V", "D", "r_c", "r_r", "g")
+
+
+def _layout(head: dict):
+    entries, off = [], 0
+    for k in _HEAD_KEYS:
+        a = np.ascontiguousarray(head[k])
+        entries.append([k, a.dtype.str, list(a.shape), off, int(a.nbytes)])
+        off += (a.nbytes + 15) // 16 * 16
+    return entries, off
+
+
+def save_head(head: dict, path: str) -> int:
+    """Write the canonical packed head to `path`; returns the file size in bytes."""
+    import json
+    entries, data_bytes = _layout(head)
+    hdr = json.dumps({"meta": {k: int(head[k]) for k in _META_KEYS}, "arrays": entries},
+                     separators=(",", ":")).encode()
+    pre = len(_MAGIC) + 8 + len(hdr)
+    pad = (-pre) % 16
+    with open(path, "wb") as f:
+        f.write(_MAGIC)
+        f.write(np.uint64(len(hdr)).tobytes())
+        f.write(hdr)
+        f.write(b"\0" * pad)
+        for k, _, _, off, nb in entries:
+            a = np.ascontiguousarray(head[k])
+            f.write(a.tobytes())
+            f.write(b"\0" * ((nb + 15) // 16 * 16 - nb))
+    return pre + pad + data_bytes
+
+
+def load_head(path: str) -> dict:
+    """Read a head written by save_head (the arrays are copies of the saved bytes)."""
+    import json
+    with open(path, "rb") as f:
+        if f.read(8) != _MAGIC:
+            raise ValueError(f"{path}: not a packed head file")
+        n = int(np.frombuffer(f.read(8), dtype=np.uint64)[0])
+        hdr = json.loads(f.read(n).decode())
+        f.read((-(16 + n)) % 16)
+        data = f.read()
+    head = {k: int(v) for k, v in hdr["meta"].items()}
+    for k, dt, shape, off, nb in hdr["arrays"]:
+        if off + nb > len(data):
+            raise ValueError(f"{path}: truncated at array {k}")
+        head[k] = np.frombuffer(data[off:off + nb], dtype=np.dtype(dt)).reshape(shape).copy()
+    return head
+
+
+def serialized_nbytes(head: dict) -> int:
+    """Size of the file save_head writes for this head (header and padding included)."""
+    import json
+    entries, data_bytes = _layout(head)
+    hdr = json.dumps({"meta": {k: int(head[k]) for k in _META_KEYS}, "arrays": entries},
+                     separators=(",", ":")).encode()
+    pre = len(_MAGIC) + 8 + len(hdr)
+    return pre + (-pre) % 16 + data_bytes

@@ -209,3 +209,31 @@ def test_agreement_with_the_dense_head_on_tiny_head():
     kl_c, t5_c = measures(pack.build_head(W, Hc, w.r_c, 0, w.g, w.p, w.lam, seed=w.seed_rsvd))
     assert kl_f < 0.5 * kl_n and kl_f < 0.5 * kl_c, (kl_f, kl_n, kl_c)
     assert t5_f > t5_n and t5_f > t5_c, (t5_f, t5_n, t5_c)
+
+
+def test_serialized_module_round_trip_is_bit_identical(tmp_path):
+    """Sec. 3 measures storage over the serialised module: the packed head written to a
+    file and read back has the same bytes in every array, the same shape metadata, and a
+    file size equal to the arrays' bytes plus a small header."""
+    from workloads import random_canonical_head
+    from packed_int4_lm_b200 import pack
+    for (V, D, r_c, r_r, g) in [(300, 512, 5, 3, 64), (129, 256, 0, 0, 128), (64, 128, 16, 0, 32)]:
+        head = random_canonical_head(V, D, r_c, r_r, g, seed=V + D, zero_rows=2)
+        path = tmp_path / f"h{V}.archead"
+        size = pack.save_head(head, str(path))
+        assert size == path.stat().st_size == pack.serialized_nbytes(head)
+        back = pack.load_head(str(path))
+        for k in ("V", "D", "r_c", "r_r", "g"):
+            assert back[k] == head[k]
+        for k in ("r_nib", "r_code", "r_super", "Ac", "sAc", "Bc", "sBc", "Aw", "sAw", "Bw", "sBw"):
+            a, b = np.ascontiguousarray(head[k]), back[k]
+            assert a.dtype == b.dtype and a.shape == b.shape, k
+            assert a.tobytes() == b.tobytes(), k
+        payload = sum(np.asarray(head[k]).nbytes for k in head if isinstance(head[k], np.ndarray))
+        assert payload <= size <= payload + 11 * 16 + 1024
+        Hb = bf16_bits(make_hidden(3, make_channel_scales(D, 0.5, 4, 20.0, 1), 2))
+        assert np.array_equal(oracle.logits(back, Hb), oracle.logits(head, Hb))
+    bad = tmp_path / "bad.archead"
+    bad.write_bytes(b"NOTAHEAD" + b"\0" * 32)
+    with pytest.raises(ValueError):
+        pack.load_head(str(bad))
