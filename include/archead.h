@@ -199,6 +199,19 @@ int archead_dequant(const archead_head* head, int64_t row0, int64_t nrows, float
  */
 int archead_check(void* stream);
 
+/*
+ * archead_test_hooks -- failure-detection hook of the test build (libarchead_testhooks.so,
+ *   compiled with ARCHEAD_TEST_HOOKS); the product library returns ARCHEAD_ERR_UNSUPPORTED
+ *   and changes nothing.  In the test build it sets, for later calls on this process, the
+ *   bound of the decode kernel's (N <= 16) bounded mbarrier waits in SM cycles (default
+ *   2^31) and the CTA index whose first consumer warp waits on a barrier that no thread
+ *   ever arrives on (-1: none).  That wait gives up after the bound, the kernel finishes
+ *   with ARCHEAD_ERR_TIMEOUT in the device error word (archead_check reports it) and the
+ *   logits of the call are undefined; the device stays usable.  wait_limit_cycles < 1
+ *   gives ARCHEAD_ERR_SHAPE.
+ */
+int archead_test_hooks(long long wait_limit_cycles, int stall_cta);
+
 /* Human-readable text of a status code (static string, never NULL). */
 const char* archead_strerror(int status);
 

@@ -163,7 +163,14 @@ def vocab_parallel_nll(H: torch.Tensor, dh: DeviceHead, targets: torch.Tensor, v
     and every rank merges them in rank order.  H and targets are the same on every rank."""
     import torch.distributed as dist
     part = nll_partials(H, dh, targets, v_begin, v_total)
+    if not (dist.is_available() and dist.is_initialized()):  # one process holds the head
+        return nll_merge(part[None])
     G = dist.get_world_size(group)
+    if dist.get_backend(group) == "gloo":  # host collectives (tests without NCCL)
+        host = part.cpu()
+        gathered = [torch.empty_like(host) for _ in range(G)]
+        dist.all_gather(gathered, host, group=group)
+        return nll_merge(torch.stack(gathered).to(part.device))
     gathered = [torch.empty_like(part) for _ in range(G)]
     dist.all_gather(gathered, part, group=group)
     return nll_merge(torch.stack(gathered))

@@ -55,10 +55,29 @@ _SIGS = {
                                      c_vp, c_i64, c_i64, c_i64, c_int, c_int, c_int, c_vp]),
     "archead_nll_merge": (c_int, [c_vp, c_int, c_i64, c_vp, c_vp]),
     "archead_profile": (c_int, [c_int]),
+    "archead_test_hooks": (c_int, [ctypes.c_longlong, c_int]),
     "archead_profile_read": (c_int, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(c_int)]),
 }
 
 _lib = None
+TESTHOOKS_PATH = os.path.join(HERE, "libarchead_testhooks.so")
+
+
+def _bind(L: ctypes.CDLL) -> ctypes.CDLL:
+    for name, (res, args) in _SIGS.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    return L
+
+
+def testhooks_lib() -> ctypes.CDLL:
+    """The failure-detection test build of the library (same entry points, plus working
+    archead_test_hooks).  Only tests load it."""
+    if not os.path.exists(TESTHOOKS_PATH):
+        raise ImportError(f"{TESTHOOKS_PATH} is missing: build it with "
+                          "`python -m packed_int4_lm_b200.build`.")
+    return _bind(ctypes.CDLL(TESTHOOKS_PATH))
 
 
 def lib() -> ctypes.CDLL:
@@ -69,12 +88,7 @@ def lib() -> ctypes.CDLL:
             raise ImportError(
                 f"{LIB_PATH} is missing: build it with `python -m packed_int4_lm_b200.build`. "
                 "The packed-head logit path has no CPU or Python fallback.")
-        L = ctypes.CDLL(LIB_PATH)
-        for name, (res, args) in _SIGS.items():
-            f = getattr(L, name)
-            f.restype = res
-            f.argtypes = args
-        _lib = L
+        _lib = _bind(ctypes.CDLL(LIB_PATH))
     return _lib
 
 

@@ -29,8 +29,11 @@ def _headers():
     return glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(ROOT, "include", "*.h"))
 
 
-def _compile(src: str, force: bool, extra) -> str:
-    obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+TESTHOOKS_LIB = os.path.join(HERE, "libarchead_testhooks.so")
+
+
+def _compile(src: str, force: bool, extra, outdir: str = BUILD) -> str:
+    obj = os.path.join(outdir, os.path.basename(src)[:-3] + ".o")
     newest = max([os.path.getmtime(src)] + [os.path.getmtime(h) for h in _headers()])
     if force or not os.path.exists(obj) or os.path.getmtime(obj) < newest:
         cmd = [NVCC, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
@@ -42,16 +45,27 @@ def _compile(src: str, force: bool, extra) -> str:
     return obj
 
 
-def build(force: bool = False, jobs: int = 8, extra=()) -> str:
+def _link(lib: str, objs, force: bool) -> None:
+    if force or not os.path.exists(lib) or os.path.getmtime(lib) < max(map(os.path.getmtime, objs)):
+        cmd = [NVCC, *ARCH, "-shared", "-cudart", "static", "-o", lib, *objs]
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        if r.returncode != 0:
+            raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
+
+
+def build(force: bool = False, jobs: int = 8, extra=(), testhooks: bool = True) -> str:
+    """Build libarchead.so and, unless testhooks is False, the failure-detection test build
+    libarchead_testhooks.so (the same sources with ARCHEAD_TEST_HOOKS defined)."""
     os.makedirs(BUILD, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     with cf.ThreadPoolExecutor(max_workers=jobs) as ex:
         objs = list(ex.map(lambda s: _compile(s, force, list(extra)), srcs))
-    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < max(map(os.path.getmtime, objs)):
-        cmd = [NVCC, *ARCH, "-shared", "-cudart", "static", "-o", LIB, *objs]
-        r = subprocess.run(cmd, capture_output=True, text=True)
-        if r.returncode != 0:
-            raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
+        _link(LIB, objs, force)
+        if testhooks:
+            tdir = os.path.join(BUILD, "testhooks")
+            os.makedirs(tdir, exist_ok=True)
+            tobjs = list(ex.map(lambda s: _compile(s, force, ["-DARCHEAD_TEST_HOOKS"], tdir), srcs))
+            _link(TESTHOOKS_LIB, tobjs, force)
     return LIB
 
 

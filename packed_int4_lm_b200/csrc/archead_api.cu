@@ -473,6 +473,18 @@ int archead_profile_read(double* total_ms, int* count) {
   return ARCHEAD_OK;
 }
 
+int archead_test_hooks(long long wait_limit_cycles, int stall_cta) {
+#ifdef ARCHEAD_TEST_HOOKS
+  if (wait_limit_cycles < 1) return ARCHEAD_ERR_SHAPE;
+  set_dec_test_hooks(wait_limit_cycles, stall_cta);
+  return ARCHEAD_OK;
+#else
+  (void)wait_limit_cycles;
+  (void)stall_cta;
+  return ARCHEAD_ERR_UNSUPPORTED;
+#endif
+}
+
 int archead_check(void* stream) {
   DeviceState* ds;
   int rc = current_state(&ds);

@@ -190,6 +190,13 @@ cudaError_t launch_residual_dec(const __half* img, const float* t, const archead
                                 float4* scratch, unsigned* counters, unsigned* err,
                                 cudaStream_t st, int* launches);
 
+#ifdef ARCHEAD_TEST_HOOKS
+// Failure-detection test builds: the bound of the decode kernel's mbarrier waits (SM
+// cycles) and the CTA whose consumer warp 0 waits on a barrier that never completes
+// (-1: none).
+void set_dec_test_hooks(long long wait_limit, int stall_cta);
+#endif
+
 // Residual dequant-contraction over token blocks of up to 64 (mma.sync path).
 // mode 0: write logits Y.  mode 1: write NLL partials (max, sum exp) per (token, vocabulary
 // block) into part[N x residual_gemm_vblocks] and the target logit into tlogit[N].

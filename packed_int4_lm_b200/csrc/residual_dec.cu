@@ -53,6 +53,8 @@ struct DecParams {
   int sp;  // packed ring stages
   int64_t n_vtiles;
   unsigned* err;
+  long long wait_limit;  // bound of every mbarrier wait, in SM cycles
+  int stall_cta;         // test builds: the CTA whose consumer warp 0 waits on a dead barrier
 };
 
 // FP16 element offset of (token n, column d) in the resident H image: rows of D
@@ -132,9 +134,9 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t saddr, uint32_t r[4]) {
 
 // Bounded wait that is skipped once this warp has already given up.
 __device__ __forceinline__ bool dec_wait(uint64_t* bar, uint32_t parity, unsigned* err,
-                                         bool ok) {
+                                         bool ok, long long limit) {
   if (!ok) return false;
-  return __all_sync(0xffffffffu, tc::mbar_wait(bar, parity, err));
+  return __all_sync(0xffffffffu, tc::mbar_wait(bar, parity, err, limit));
 }
 
 // Prologue of this path: the resident H image (zero rows up to NTOK), followed by the
@@ -196,87 +198,71 @@ __device__ __forceinline__ void dec_convert_h(const uint16_t* __restrict__ H,
 }
 
 // t[n, j] = sum_d h[n, d] fl32(B[j, d] s[j, d / g]) for the N <= 16 tokens of this path,
-// B = [Q8(B_c) | Q8(B_w)], on warp MMAs: block f computes the factors 16 f .. 16 f + 15 for
-// all tokens, warp w the K range [w D / 8, (w + 1) D / 8).  Per 16-column step the INT8
-// factor bytes (exact in FP16) meet the FP16 hidden states in one m16n8k16 MMA per token
-// block, and the step's FP32 result is scaled by the factor's group scale s[j, d / g]: t is
-// sum over groups of s_jk sum_{d in k} q_jd h_nd, the product fl32(q s) h of the dequantised
-// factor up to the rounding of that one product.  The warps' sums are added in a fixed order.
+// B = [Q8(B_c) | Q8(B_w)]: one block per factor index j, 256 threads striding over D, 8
+// columns each.  All of an iteration's loads (the 8 factor bytes, their scale and the 8
+// columns of every token) are issued before its FMAs, so an iteration costs one memory
+// latency whatever N is.
+constexpr int kDecPrologueThreads = 256;
+
 __device__ __forceinline__ void dec_lowrank_t(const uint16_t* __restrict__ H,
                                               const int8_t* __restrict__ Bc,
                                               const float* __restrict__ sBc,
                                               const int8_t* __restrict__ Bw,
                                               const float* __restrict__ sBw, int r_c, int r_r,
                                               int64_t N, int64_t D, int g, float* __restrict__ t,
-                                              int fb) {
+                                              int j) {
   const int RR = r_c + r_r;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gid = lane >> 2, tq = lane & 3;
-  const int64_t G = D / g;
-  const int8_t* qr[2];
-  const float* sr[2];
+  const int8_t* B = j < r_c ? Bc + (int64_t)j * D : Bw + (int64_t)(j - r_c) * D;
+  const float* sB = j < r_c ? sBc + (int64_t)j * (D / g) : sBw + (int64_t)(j - r_c) * (D / g);
+  float acc[16];
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int j = 16 * fb + gid + 8 * h;
-    qr[h] = j < r_c ? Bc + (int64_t)j * D : (j < RR ? Bw + (int64_t)(j - r_c) * D : nullptr);
-    sr[h] = j < r_c ? sBc + (int64_t)j * G : (j < RR ? sBw + (int64_t)(j - r_c) * G : nullptr);
-  }
-  const __half2 k1152 = __float2half2_rn(1152.f);
-  float acc[2][4];
+  for (int n = 0; n < 16; ++n) acc[n] = 0.f;
+  for (int64_t d0 = threadIdx.x * 8; d0 < D; d0 += kDecPrologueThreads * 8) {
+    const uint2 braw = *reinterpret_cast<const uint2*>(B + d0);
+    const float sc = sB[d0 / g];
+    // all 16 token rows are loaded (rows past N repeat the last one, and their sums are
+    // never stored), so the loads carry no predicate and issue together
+    uint4 hv[16];
 #pragma unroll
-  for (int b = 0; b < 2; ++b) acc[b][0] = acc[b][1] = acc[b][2] = acc[b][3] = 0.f;
-  const int64_t kw = D / 8;
-  for (int64_t k0 = warp * kw; k0 < (warp + 1) * kw; k0 += 16) {
-    // A: the factor rows gid (h = 0) and gid + 8 (h = 1), bytes k0 + 4 tq .. + 3 as the K
-    // slots 2 tq, 2 tq + 1 (bytes 0, 1) and 2 tq + 8, 2 tq + 9 (bytes 2, 3)
-    uint32_t a[4];
-    float sc[2];
+    for (int n = 0; n < 16; ++n)
+      hv[n] = __ldg(reinterpret_cast<const uint4*>(H + (n < N ? n : N - 1) * D + d0));
+    const int8_t* bq = reinterpret_cast<const int8_t*>(&braw);
+    float b[8];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint32_t w =
-          qr[h] ? __ldg(reinterpret_cast<const unsigned int*>(qr[h] + k0 + 4 * tq)) ^ 0x80808080u
-                : 0x80808080u;
-      // bytes b + 128 under the FP16 pattern 0x6400 read 1024 + b + 128: minus 1152
-      uint32_t q0 = __byte_perm(w, 0x64646464u, 0x5140), q1 = __byte_perm(w, 0x64646464u, 0x7352);
-      a[h] = h2_bits(__hsub2(*reinterpret_cast<__half2*>(&q0), k1152));
-      a[2 + h] = h2_bits(__hsub2(*reinterpret_cast<__half2*>(&q1), k1152));
-      sc[h] = sr[h] ? __ldg(sr[h] + k0 / g) : 0.f;
-    }
+    for (int k = 0; k < 8; ++k) b[k] = __fmul_rn((float)bq[k], sc);
 #pragma unroll
-    for (int b = 0; b < 2; ++b) {  // token blocks 0..7, 8..15
-      const int64_t n = 8 * b + gid;
-      uint2 hb = make_uint2(0u, 0u);
-      if (n < N) hb = __ldg(reinterpret_cast<const uint2*>(H + n * D + k0 + 4 * tq));
-      const __half2 b0 = __floats2half2_rn(__uint_as_float(hb.x << 16), __uint_as_float(hb.x & 0xFFFF0000u));
-      const __half2 b1 = __floats2half2_rn(__uint_as_float(hb.y << 16), __uint_as_float(hb.y & 0xFFFF0000u));
-      float d[4] = {0.f, 0.f, 0.f, 0.f};
-      mma_f16_16816(d, a, h2_bits(b0), h2_bits(b1));
-      acc[b][0] = fmaf(sc[0], d[0], acc[b][0]);
-      acc[b][1] = fmaf(sc[0], d[1], acc[b][1]);
-      acc[b][2] = fmaf(sc[1], d[2], acc[b][2]);
-      acc[b][3] = fmaf(sc[1], d[3], acc[b][3]);
+    for (int n = 0; n < 16; ++n) {
+      const uint32_t hw[4] = {hv[n].x, hv[n].y, hv[n].z, hv[n].w};
+      float a = acc[n];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        a = fmaf(__uint_as_float(hw[k] << 16), b[2 * k], a);
+        a = fmaf(__uint_as_float(hw[k] & 0xFFFF0000u), b[2 * k + 1], a);
+      }
+      acc[n] = a;
     }
   }
-  // accumulator: row gid (+ 8) = factor, column 2 tq (+ 1) = token of the block
-  __shared__ float red[8][16][17];
+  __shared__ float red[kDecPrologueThreads / 32][16];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
-  for (int b = 0; b < 2; ++b) {
-    red[warp][gid][8 * b + 2 * tq] = acc[b][0];
-    red[warp][gid][8 * b + 2 * tq + 1] = acc[b][1];
-    red[warp][gid + 8][8 * b + 2 * tq] = acc[b][2];
-    red[warp][gid + 8][8 * b + 2 * tq + 1] = acc[b][3];
+  for (int n = 0; n < 16; ++n) {
+    float v = acc[n];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) red[warp][n] = v;
   }
   __syncthreads();
-  const int row = threadIdx.x >> 4, n = threadIdx.x & 15;  // 256 = 16 factors x 16 tokens
-  float v = 0.f;
+  if ((int64_t)threadIdx.x < N) {
+    float v = 0.f;
 #pragma unroll
-  for (int w = 0; w < 8; ++w) v += red[w][row][n];
-  const int j = 16 * fb + row;
-  if (j < RR && n < N) t[(int64_t)n * RR + j] = v;
+    for (int w = 0; w < kDecPrologueThreads / 32; ++w) v += red[w][threadIdx.x];
+    t[(int64_t)threadIdx.x * RR + j] = v;
+  }
 }
 
 // The whole prologue of this path in one launch: blocks [0, nconv) build the H image, its
-// corrections and the zeroed counters; the next ceil((r_c + r_r) / 16) blocks form t.
-__global__ void __launch_bounds__(256) dec_prologue_kernel(
+// corrections and the zeroed counters; the next r_c + r_r blocks form t.
+__global__ void __launch_bounds__(kDecPrologueThreads) dec_prologue_kernel(
     const uint16_t* __restrict__ H, __half* __restrict__ img, int64_t N, int ntok, int64_t D,
     int scale_b, unsigned* __restrict__ counters, int64_t n_counters, int nconv,
     const int8_t* __restrict__ Bc, const float* __restrict__ sBc,
@@ -408,7 +394,8 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
   uint64_t* c_empty = bars + 3;  // [2]
   uint64_t* p_full = bars + 5;   // [SP]
   uint64_t* p_empty = p_full + SP;
-  int* flag = reinterpret_cast<int*>(p_empty + SP);
+  uint64_t* dead = p_empty + SP;  // test builds: a barrier nothing arrives on
+  int* flag = reinterpret_cast<int*>(dead + 1);
   const int code_bytes = 128 * G;
   const size_t code_slot = dec_round16((size_t)code_bytes);
   const size_t arc_slot = dec_round16((size_t)128 * p.r_c);
@@ -429,6 +416,7 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
       tc::mbar_init(&p_full[s], 1);
       tc::mbar_init(&p_empty[s], kDecRows);  // one warp per row group takes a stage
     }
+    tc::mbar_init(dead, 1);
     tc::mbar_fence_init();
   }
   __syncthreads();
@@ -459,7 +447,7 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
         const int kb1 = (int)((int64_t)nkb < kb0 + (u1 - u) ? (int64_t)nkb : kb0 + (u1 - u));
         const int cs = s & 1;
         if (s >= 2) issue_h();
-        if (s >= 2 && !tc::mbar_wait(&c_empty[cs], ((s >> 1) - 1) & 1, p.err)) {
+        if (s >= 2 && !tc::mbar_wait(&c_empty[cs], ((s >> 1) - 1) & 1, p.err, p.wait_limit)) {
           ok = false;
           break;
         }
@@ -478,7 +466,7 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
           const int st = k % SP;
           const uint32_t bytes = (uint32_t)(kb + 1 < kb1 ? 2 * kDecPk : kDecPk);
           if (k >= SP) issue_h();
-          if (k >= SP && !tc::mbar_wait(&p_empty[st], ((k / SP) - 1) & 1, p.err)) {
+          if (k >= SP && !tc::mbar_wait(&p_empty[st], ((k / SP) - 1) & 1, p.err, p.wait_limit)) {
             ok = false;
             break;
           }
@@ -491,13 +479,14 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
         u += kb1 - kb0;
       }
       issue_h();
-      tc::mbar_wait(h_full, 0, p.err);
-      if (!ok) {  // drain copies still in flight before the CTA exits
-        for (int q = np - SP < 0 ? 0 : np - SP; q < np; ++q)
-          tc::mbar_wait(&p_full[q % SP], (q / SP) & 1, p.err);
-        for (int q = nc - 2 < 0 ? 0 : nc - 2; q < nc; ++q)
-          tc::mbar_wait(&c_full[q & 1], (q >> 1) & 1, p.err);
-      }
+      tc::mbar_wait(h_full, 0, p.err, p.wait_limit);
+      // Every copy this thread issued has landed before the CTA exits, whether or not the
+      // consumers waited for it (after a timeout they stop waiting).  Each slot's last
+      // issued phase is the one waited for here; in a normal run it has completed already.
+      for (int q = np - SP < 0 ? 0 : np - SP; q < np; ++q)
+        tc::mbar_wait(&p_full[q % SP], (q / SP) & 1, p.err, p.wait_limit);
+      for (int q = nc - 2 < 0 ? 0 : nc - 2; q < nc; ++q)
+        tc::mbar_wait(&c_full[q & 1], (q >> 1) & 1, p.err, p.wait_limit);
     }
     return;
   }
@@ -508,7 +497,12 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
   const int par = warp / kDecRows;
   const int ctid = threadIdx.x;  // the first eight warps: 0 .. 255
   grid_dependency_wait();  // t and the tile counters come from the prologue kernel
-  bool ok = dec_wait(h_full, 0, p.err, true);
+  bool ok = dec_wait(h_full, 0, p.err, true, p.wait_limit);
+#ifdef ARCHEAD_TEST_HOOKS
+  // failure-detection test: one warp waits on a barrier that never completes; its bounded
+  // wait gives up, sets the device error word, and the warp skips its remaining waits
+  if ((int)blockIdx.x == p.stall_cta && warp == 0) ok = dec_wait(dead, 0, p.err, ok, p.wait_limit);
+#endif
   for (int i = ctid; i < NTOK * RR; i += CONSUMERS * 32) {  // ts[j * NTOK + n]
     const int j = i / NTOK, n = i - j * NTOK;
     const float tv = n < p.N ? __ldg(p.t + (int64_t)n * RR + j) : 0.f;
@@ -554,7 +548,7 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
     const float S_hi = bf16_bits_to_float(__ldg(p.sup + vc_hi));
     const float sac_lo = p.r_c ? __ldg(p.sAc + vc_lo) : 0.f, sac_hi = p.r_c ? __ldg(p.sAc + vc_hi) : 0.f;
     const float saw_lo = p.r_r ? __ldg(p.sAw + vc_lo) : 0.f, saw_hi = p.r_r ? __ldg(p.sAw + vc_hi) : 0.f;
-    ok = dec_wait(&c_full[cs], (s >> 1) & 1, p.err, ok);
+    ok = dec_wait(&c_full[cs], (s >> 1) & 1, p.err, ok, p.wait_limit);
     const unsigned char* crow_lo = cds + cs * code_slot + r_lo * G;
     const unsigned char* crow_hi = cds + cs * code_slot + r_hi * G;
 
@@ -574,7 +568,7 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
         }
         continue;
       }
-      ok = dec_wait(&p_full[st], ph, p.err, ok);
+      ok = dec_wait(&p_full[st], ph, p.err, ok, p.wait_limit);
       const int nb = kb2 + 1 < kb1 ? 2 : 1;
       uint32_t wlo[2][4], whi[2][4];  // [block][chunk]: word tq of rows r_lo, r_hi
       uint32_t clo[2], chi[2];
@@ -888,6 +882,17 @@ int fit_sp(const Shapes& s, size_t budget) {
 
 }  // namespace
 
+#ifdef ARCHEAD_TEST_HOOKS
+namespace {
+long long g_hook_wait_limit = 1ll << 31;
+int g_hook_stall_cta = -1;
+}  // namespace
+void set_dec_test_hooks(long long wait_limit, int stall_cta) {
+  g_hook_wait_limit = wait_limit;
+  g_hook_stall_cta = stall_cta;
+}
+#endif
+
 DecPlan dec_plan(const Shapes& s, bool nll) {
   DecPlan pl = {0, 0, 0};
   if (s.N < 1 || s.N > 16) return pl;
@@ -919,13 +924,13 @@ cudaError_t launch_dec_prologue(const uint16_t* H, const archead_head* head, con
   const int64_t ntok = 8 * pl.nt8;
   const int64_t n_counters = (s.V + 127) / 128;
   // one warp per (token, 128-column block), the counters on the same blocks; then one
-  // block per 16 factors for t
-  int64_t blocks = (ntok * (s.D / 128) * 32 + 255) / 256;
-  const int64_t cb = (n_counters + 255) / 256;
+  // block per factor index for t
+  int64_t blocks = (ntok * (s.D / 128) * 32 + kDecPrologueThreads - 1) / kDecPrologueThreads;
+  const int64_t cb = (n_counters + kDecPrologueThreads - 1) / kDecPrologueThreads;
   if (cb > blocks) blocks = cb;
   if (blocks > 148 * 8) blocks = 148 * 8;
   const int RR = s.r_c + s.r_r;
-  dec_prologue_kernel<<<(unsigned)(blocks + (RR + 15) / 16), 256, 0, st>>>(
+  dec_prologue_kernel<<<(unsigned)(blocks + RR), kDecPrologueThreads, 0, st>>>(
       H, img, s.N, (int)ntok, s.D, s.g >= 128 ? 1 : 0, counters, n_counters, (int)blocks,
       head->Bc, head->sBc, head->Bw, head->sBw, s.r_c, s.r_r, s.g, t, err);
   ++*launches;
@@ -964,6 +969,13 @@ cudaError_t launch_residual_dec(const __half* img, const float* t, const archead
   p.sp = pl.sp;
   p.n_vtiles = (s.V + 127) / 128;
   p.err = err;
+#ifdef ARCHEAD_TEST_HOOKS
+  p.wait_limit = g_hook_wait_limit;
+  p.stall_cta = g_hook_stall_cta;
+#else
+  p.wait_limit = 1ll << 31;
+  p.stall_cta = -1;
+#endif
   if (pl.nt8 < 1 || pl.nt8 > 2 || pl.sp < 3 || pl.sp > kDecMaxSP || pl.grid < 1)
     return cudaErrorInvalidValue;
   cudaError_t e;

@@ -51,13 +51,15 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the completion of the phase with the given parity, for at most ~2^31 SM cycles
-// (about a second).  On timeout the device error word gets kErrTimeout and false returns.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* err) {
+// Wait for the completion of the phase with the given parity, for at most `limit` SM
+// cycles (by default 2^31, about a second).  On timeout the device error word gets
+// kErrTimeout and false returns.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* err,
+                                          long long limit = 1ll << 31) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > (1ll << 31)) {
+    if (clock64() - t0 > limit) {
       atomicOr(err, kErrTimeout);
       return false;
     }

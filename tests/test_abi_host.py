@@ -126,3 +126,14 @@ def test_noalloc_rejects_sizes_beyond_its_scratch_before_any_product(L):
     assert na(_fake_head(D=4096), (1 << 31) - 1) == E["ARCHEAD_ERR_SHAPE"]
     assert na(_fake_head(D=4096, r_c=32, r_r=32), 256) == E["ARCHEAD_ERR_SHAPE"]
     assert na(_fake_head(), 0) == E["ARCHEAD_OK"]
+
+
+def test_product_library_refuses_the_test_hooks(L):
+    """archead_test_hooks works only in the failure-detection test build; the product
+    library reports ARCHEAD_ERR_UNSUPPORTED and changes nothing (no device is touched)."""
+    assert L.archead_test_hooks(1 << 20, 0) == E["ARCHEAD_ERR_UNSUPPORTED"]
+    if os.path.exists(_lib.TESTHOOKS_PATH):
+        T = _lib.testhooks_lib()
+        assert set(_lib.header_functions()) <= {n for n in _lib._SIGS}
+        for n in _lib.header_functions():
+            assert hasattr(T, n), n

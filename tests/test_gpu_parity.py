@@ -410,3 +410,48 @@ def test_workload_wide_nll(dev):
     got = out.cpu().double().numpy()[sample]
     assert np.max(np.abs(got - ref)) <= NLL_TOL, (got, ref)
     assert np.all(np.isfinite(out.cpu().numpy()))
+
+
+_GUARD = 4096          # floats before and after the output
+_CANARY = 0x7FC0DEAD   # a NaN bit pattern no kernel writes
+
+
+def _guarded(n, dev):
+    buf = torch.empty(2 * _GUARD + n, dtype=torch.float32, device=dev)
+    buf.view(torch.int32).fill_(_CANARY)
+    return buf, buf[_GUARD:_GUARD + n]
+
+
+def _guards_intact(buf):
+    iv = buf.view(torch.int32)
+    return bool((iv[:_GUARD] == _CANARY).all()) and bool((iv[-_GUARD:] == _CANARY).all())
+
+
+@pytest.mark.parametrize("V,D,N,g,path", [(1000, 512, 4, 128, "decode"),
+                                          (515, 1024, 12, 64, "decode, two token blocks"),
+                                          (1000, 512, 40, 64, "tcgen05"),
+                                          (40000, 256, 20, 64, "tcgen05, split tiles"),
+                                          (300, 16384, 8, 128, "warp-MMA fallback"),
+                                          (1000, 512, 300, 128, "tcgen05, several token tiles")])
+def test_outputs_stay_inside_their_rows(dev, V, D, N, g, path):
+    """Canary bands of a NaN pattern before and after Y (N x V, ragged V) and the NLL output
+    stay untouched on every kernel path, including the split tiles that go through scratch
+    and the ragged last vocabulary tile."""
+    head = random_canonical_head(V, D, 8, 8, g, seed=V + N, zero_rows=2,
+                                 super_exp_range=(-17, -13), factor_exp_range=(-13, -10))
+    dh = ah.DeviceHead.from_canonical(head, dev)
+    Hc = _rand_H(N, D, 1000 + N)
+    H = Hc.to(dev)
+    buf, flat = _guarded(N * V, dev)
+    Y = flat.view(N, V)
+    ah.logits(H, dh, out=Y)
+    ah.check()
+    assert _guards_intact(buf), path
+    rows = np.arange(0, V, max(1, V // 997))
+    _assert_logits(Y.cpu().numpy()[:, rows], oracle.logits(head, bf16_bits(Hc), rows=rows), path)
+    nbuf, nflat = _guarded(N, dev)
+    tg = make_targets(N, V, 2000 + N)
+    ah.nll(H, dh, tg.to(dev), out=nflat)
+    ah.check()
+    assert _guards_intact(nbuf), path
+    assert torch.isfinite(nflat).all()

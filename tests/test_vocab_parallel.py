@@ -4,7 +4,8 @@ merges them (ARCHead Sec. 5 cross-entropy, split over the vocabulary).
 
 CPU: the row-shard helper against the oracle, and the two-rank protocol on gloo with the
 two library calls replaced by fp64 test doubles.  GPU: the shard partials and the merge
-through the library against the oracle on the whole head."""
+through the library against the oracle on the whole head, and two gloo ranks (processes
+sharing the GPU, host all-gather) running the real library calls."""
 import os
 import socket
 
@@ -126,3 +127,35 @@ def test_shard_partials_and_merge_match_oracle(cuda_ok, N):
     # the target logit comes from exactly one shard
     owned = torch.stack(parts)[:, :, 2].ne(0).sum(dim=0)
     assert int(owned.max()) <= 1
+
+
+def _rank_lib(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        dev = torch.device("cuda:0")
+        head = _head()
+        v0, v1 = ((0, 450), (450, 1000))[rank]
+        dh = ah.DeviceHead.from_canonical(shard_rows(head, v0, v1), dev)
+        H = _H(9, 5).to(dev)
+        tg = make_targets(9, 1000, 6).to(dev)
+        nll = ah.vocab_parallel_nll(H, dh, tg, v0, 1000)
+        ah.check()
+        out[rank] = nll.cpu().double().numpy().tolist()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.gpu
+def test_two_gloo_ranks_with_library_partials(cuda_ok):
+    """The exchange of vocab_parallel_nll with the library's own partials and merge: two
+    ranks (processes on the same GPU, gloo all-gather through host memory) each hold half
+    of the rows; both must return the whole head's NLL, identical on the two ranks."""
+    world, port = 2, _free_port()
+    with mp.get_context("spawn").Manager() as m:
+        out = m.dict()
+        mp.spawn(_rank_lib, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    ref = oracle.nll(_head(), bf16_bits(_H(9, 5)), make_targets(9, 1000, 6).numpy())
+    assert res[0] == res[1]
+    assert np.max(np.abs(np.asarray(res[0]) - ref)) <= NLL_TOL
