@@ -163,7 +163,7 @@ class ClockSampler:
 def build_head(w, device, keep_dense=False):
     """The packed head of workload w, the channel scales of its activations, and the
     construction's wall seconds (Algorithm 1 on `device`, synchronised); with keep_dense
-    also the dense head as BF16 for the quality comparison of the fused-NLL workload."""
+    also the dense head W (FP32, on `device`) for the quality comparisons."""
     from packed_int4_lm_b200 import pack
     W = make_weight(w.V, w.D, w.rank, w.sigma0, w.noise, w.seed_w, device=device)
     s = make_channel_scales(w.D, w.sigma_s, w.n_outliers, w.outlier_mult, w.seed_scales)
@@ -173,10 +173,46 @@ def build_head(w, device, keep_dense=False):
     head = pack.build_head(W, Hc, w.r_c, w.r_r, w.g, w.p, w.lam, seed=w.seed_rsvd)
     torch.cuda.synchronize()
     cons_s = time.perf_counter() - t0
-    Wb = W.to(torch.bfloat16) if keep_dense else None
+    if keep_dense:
+        return head, s, cons_s, W, Hc
     del W, Hc
     torch.cuda.empty_cache()
-    return (head, s, cons_s, Wb) if keep_dense else (head, s, cons_s)
+    return head, s, cons_s
+
+
+def agreement_quality(ah, w, head, W, Hcal, Hq, dev):
+    """Quality context on the decode head, through the library's GPU path only: the packed
+    head and its storage-matched baselines (Sec. 5, Tables 3 and 8: plain group INT4 at a
+    matching storage, the quantized core without the correction, Row INT8 at about twice
+    the storage) against the dense head in BF16 on the same tokens.  Per head: storage over
+    BF16, relative logit error ||Y - Y_dense||_F / ||Y_dense||_F, mean KL(dense || head),
+    and the fraction of tokens whose dense top-1 id is among the head's top 1 / 5 / 10."""
+    from packed_int4_lm_b200 import pack
+    H = Hq.to(dev)
+    Yd = torch.matmul(H, W.to(torch.bfloat16).t()).float()  # the dense comparator (cuBLAS)
+    heads = {"archead": head}
+    heads["group_int4_g32"] = pack.build_head(W, Hcal, 0, 0, 32, w.p, w.lam, seed=w.seed_rsvd)
+    heads["core_only"] = pack.build_head(W, Hcal, w.r_c, 0, w.g, w.p, w.lam, seed=w.seed_rsvd)
+    heads["row_int8"] = pack.build_row8_head(W, g=w.g)
+    out = {"tokens": int(H.shape[0]), "dense": "H W^T with W in BF16 (torch.matmul, comparator)",
+           "synthetic_W": "rank-64 decaying spectrum plus N(0, 0.02^2) noise: the noise "
+                          "dominates, so these figures are not the paper's real-head ones"}
+    for name, hd in heads.items():
+        dh = ah.DeviceHead.from_canonical(hd, dev)
+        Y = ah.logits(H, dh)
+        a = ah.agreement(H, dh, Yd, 10)
+        ah.check()
+        top = a["topk"].long()
+        t1 = a["top1_dense"].long()[:, None]
+        out[name] = {"storage_vs_bf16": pack.storage_ratio(hd),
+                     "rel_logit_err": float((Y - Yd).norm() / Yd.norm()),
+                     "mean_kl": float(a["kl"].double().mean()),
+                     "top1_agree": float((top[:, :1] == t1).any(1).float().mean()),
+                     "top5_agree": float((top[:, :5] == t1).any(1).float().mean()),
+                     "top10_agree": float((top[:, :10] == t1).any(1).float().mean())}
+        del dh
+    torch.cuda.empty_cache()
+    return out
 
 
 def nll_quality(head, Wb, Hcpu, tg, ours, sample=16):
@@ -499,9 +535,14 @@ def main():
             device_id=torch.device("cuda", local))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    Wb = None
-    if nll_mode and rank == 0:
-        head, s, cons_s, Wb = build_head(w, dev, keep_dense=True)
+    Wb = Wf = Hcal = None
+    if rank == 0 and (nll_mode or w.name == "qwen_decode") and not a.ns:
+        head, s, cons_s, Wf, Hcal = build_head(w, dev, keep_dense=True)
+        if nll_mode:
+            Wb = Wf.to(torch.bfloat16)
+            del Wf, Hcal
+            Wf = Hcal = None
+            torch.cuda.empty_cache()
     else:
         head, s, cons_s = build_head(w, dev)
     dh = ah.DeviceHead.from_canonical(head, dev)
@@ -622,7 +663,11 @@ def main():
     d2h = sum(4 * N if nll_mode else 4 * N * w.V for N in Ns)
 
     quality = None
-    if nll_mode and rank == 0:
+    if Wf is not None:  # the decode head: agreement with the dense head, GPU path
+        quality = agreement_quality(ah, w, head, Wf, Hcal, Hcpu[max(Ns)], dev)
+        del Wf, Hcal
+        torch.cuda.empty_cache()
+    if nll_mode and rank == 0 and Wb is not None:
         Nq = Ns[0]
         ah.nll(H[Nq], dh, tgd[Nq], out=out[Nq])
         torch.cuda.synchronize()

@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define ARCHEAD_ABI_VERSION 1
+#define ARCHEAD_ABI_VERSION 2
 
 enum archead_status {
   ARCHEAD_OK = 0,
@@ -60,6 +60,13 @@ enum archead_status {
   ARCHEAD_ERR_CUDA = -7,        /* a CUDA runtime call or launch failed               */
   ARCHEAD_ERR_UNSUPPORTED = -8, /* no kernel for this device / configuration          */
   ARCHEAD_ERR_NOMEM = -9        /* stream-ordered allocation failed                   */
+};
+
+/* Storage formats of a head (archead_head.format). */
+enum archead_format {
+  ARCHEAD_FMT_SC4 = 0, /* the ARCHead packed head below (default)                        */
+  ARCHEAD_FMT_ROW8 = 1 /* Row INT8 baseline: W[v, d] = q8[v, d] * row_scale[v], no core,
+                          no correction (the storage-matched comparison of Sec. 5)        */
 };
 
 /*
@@ -78,11 +85,19 @@ enum archead_status {
  *   Bw int8 r_r x D, sBw f32 r_r x D/g correction right factor, group-wise
  * A factor entry's value is the IEEE-single product of the INT8 value and its scale.
  * Factor pointers may be NULL when their rank is 0.
+ *
+ * format ARCHEAD_FMT_ROW8 (the Row INT8 baseline the paper compares with, about twice the
+ * storage of the packed head):
+ *   r_nib     int8 V x D, row-major (no repack): q8[v, d] in [-127, 127]
+ *   row_scale float V: W[v, d] = q8[v, d] * row_scale[v] (the product taken exactly)
+ *   r_c = r_r = 0; r_code, r_super and the factor pointers are not read (may be NULL); g
+ *   must still be one of the supported values.  Such heads run on the token-block warp-MMA
+ *   kernel for every N.
  */
 typedef struct archead_head {
   int64_t V, D;
   int32_t r_c, r_r, g;
-  int32_t reserved;
+  int32_t format; /* archead_format */
   const uint8_t* r_nib;
   const uint8_t* r_code;
   const uint16_t* r_super;
@@ -94,6 +109,7 @@ typedef struct archead_head {
   const float* sAw;
   const int8_t* Bw;
   const float* sBw;
+  const float* row_scale; /* ARCHEAD_FMT_ROW8 only */
 } archead_head;
 
 /*
@@ -123,6 +139,32 @@ int archead_logits(const uint16_t* H, const archead_head* head, float* Y, int64_
 int archead_nll(const uint16_t* H, const archead_head* head, const int32_t* targets,
                 float* nll_out, int64_t N, int64_t V, int64_t D, int r_c, int r_r, int g,
                 void* stream);
+
+/*
+ * archead_agreement -- how closely the packed head's next-token distribution follows a
+ *   dense reference head on the same hidden states: the agreement measures of Sec. 5
+ *   (Table 8 and the paragraph on it: the dense top-1 token kept among the packed head's
+ *   top k, and the KL divergence), computed in the epilogue of the logit kernel without
+ *   writing the packed logits.
+ *   Y_dense        float N x V (device): the reference logits, e.g. H W^T with the dense
+ *                  BF16 head (the caller computes them).
+ *   k              1..16.
+ *   topk_out       int32 N x k (device): per token the ids of the k largest packed logits,
+ *                  in decreasing order; equal logits are ordered by the smaller id first;
+ *                  -1 where V < k.
+ *   top1_dense_out int32 N (device): argmax_v Y_dense[n, v] (equal values: smaller id).
+ *   kl_out         float N (device): KL(P_dense || P_packed) = sum_v p_d (log p_d - log p_p)
+ *                  in nats, with p = softmax over the V logits; NaN where Y_dense holds a
+ *                  non-finite value.
+ *   lse_out        float N (device, may be NULL): log sum_v exp(Y_packed[n, v]).
+ *   The top-k agreement of a token is top1_dense_out[n] in topk_out[n, :k'] for k' <= k.
+ *   Runs on the token-block warp-MMA kernel for every N.  Scratch: N x ceil(V/128) x
+ *   (6 + 2k) x 4 bytes from the library's pool.  Asynchronous on `stream`.
+ */
+int archead_agreement(const uint16_t* H, const archead_head* head, const float* Y_dense,
+                      int k, int32_t* topk_out, int32_t* top1_dense_out, float* kl_out,
+                      float* lse_out, int64_t N, int64_t V, int64_t D, int r_c, int r_r, int g,
+                      void* stream);
 
 /*
  * archead_nll_partials -- one vocabulary shard's share of archead_nll (cross-entropy of
@@ -186,7 +228,8 @@ int archead_repack_residual(const uint8_t* canon, uint8_t* dev, int64_t V, int64
  *   Ac_out float nrows x r_c, Aw_out float nrows x r_r : row-wise INT8 factors
  *   Bc_out float r_c x D, Bw_out float r_r x D : group-wise INT8 factors
  * Each INT8 entry is the single round-to-nearest-even product of value and scale.  Any
- * output may be NULL to skip it.  Reads the residual in the device layout.
+ * output may be NULL to skip it.  Reads the residual in the device layout.  A Row INT8
+ * head (ARCHEAD_FMT_ROW8) gives ARCHEAD_ERR_UNSUPPORTED.
  */
 int archead_dequant(const archead_head* head, int64_t row0, int64_t nrows, float* R_out,
                     float* Ac_out, float* Aw_out, float* Bc_out, float* Bw_out,

@@ -11,6 +11,8 @@ logits" and the inference statement closing Sec. 3 / Algorithm 1):
     W_hat = W_d + A_w B_w                             (final approximation)
     Y     = H W_hat^T  =  H W_d^T + (H B_w^T) A_w^T   (logits)
     nll_n = logsumexp_v Y[n, v] - Y[n, target_n]      (cross-entropy in nats, Sec. 5)
+    agreement with a dense head (Sec. 5, Table 8): the packed top-k ids, the dense top-1
+    id and KL(P_dense || P_packed), P = softmax of the logits
 
 Everything is evaluated in fp64 from the exact decoded values:
 
@@ -27,7 +29,8 @@ Parity pins (tests/test_oracle_pins.py): all-byte nibble decoding, single-entry 
 that fix every index and scale mapping, the r_c = r_r = 0 unit-scale case against an
 exact integer matmul, the BF16 decoding against torch over all 65536 patterns, the
 factored-vs-dense associativity identity, and the NLL special cases (constant logits,
-shift invariance, a library cross-entropy).
+shift invariance, a library cross-entropy), and for the agreement measures a library KL
+divergence, exact zeros, shift invariance and hand-checked orders of tied logits.
 """
 from __future__ import annotations
 
@@ -44,6 +47,9 @@ __all__ = [
     "logits_factored",
     "nll_from_logits",
     "nll",
+    "topk_ids",
+    "kl_dense_packed",
+    "agreement",
     "packed_nbytes",
 ]
 
@@ -107,9 +113,14 @@ def _factors(head: dict):
 
 
 def dense_head_rows(head: dict, rows=None) -> np.ndarray:
-    """W_hat = Q8(A_c) Q8(B_c) + SC4(R) + Q8(A_w) Q8(B_w) for the given vocab rows, fp64."""
+    """W_hat = Q8(A_c) Q8(B_c) + SC4(R) + Q8(A_w) Q8(B_w) for the given vocab rows, fp64.
+    A Row INT8 head (format "row8", the paper's storage-matched baseline) gives
+    W = q8 * row_scale, the product of the INT8 value and its row's FP32 scale, exact."""
     g = int(head["g"])
     sl = slice(None) if rows is None else rows
+    if head.get("format") == "row8":
+        q = np.asarray(head["q8"], dtype=np.int8)[sl].astype(np.float64)
+        return q * np.asarray(head["row_scale"], dtype=np.float32)[sl].astype(np.float64)[:, None]
     W = unpack_residual(head, rows)
     if int(head["r_c"]) > 0:
         Ac = dequant_int8_rowwise(head["Ac"][sl], head["sAc"][sl])
@@ -158,6 +169,44 @@ def nll_from_logits(Y: np.ndarray, targets: np.ndarray) -> np.ndarray:
 
 def nll(head: dict, H_bits: np.ndarray, targets: np.ndarray) -> np.ndarray:
     return nll_from_logits(logits(head, H_bits), targets)
+
+
+def topk_ids(y: np.ndarray, k: int) -> np.ndarray:
+    """Ids of the k largest entries of each row, largest first; equal values in increasing
+    id order; -1 past the row length."""
+    y = np.asarray(y, dtype=np.float64)
+    N, V = y.shape
+    out = -np.ones((N, k), dtype=np.int64)
+    for n in range(N):
+        # sort by (-value, id): a stable sort of -y keeps equal values in id order
+        order = np.argsort(-y[n], kind="stable")
+        m = min(k, V)
+        out[n, :m] = order[:m]
+    return out
+
+
+def kl_dense_packed(y_dense: np.ndarray, y_packed: np.ndarray) -> np.ndarray:
+    """KL(P_dense || P_packed) per row in nats, P = softmax of the row's logits:
+    sum_v p_d (log p_d - log p_p)."""
+    yd = np.asarray(y_dense, dtype=np.float64)
+    yp = np.asarray(y_packed, dtype=np.float64)
+    ld = yd - (yd.max(axis=1, keepdims=True)
+               + np.log(np.exp(yd - yd.max(axis=1, keepdims=True)).sum(axis=1, keepdims=True)))
+    lp = yp - (yp.max(axis=1, keepdims=True)
+               + np.log(np.exp(yp - yp.max(axis=1, keepdims=True)).sum(axis=1, keepdims=True)))
+    return (np.exp(ld) * (ld - lp)).sum(axis=1)
+
+
+def agreement(head: dict, H_bits: np.ndarray, y_dense: np.ndarray, k: int) -> dict:
+    """Agreement of the packed head with dense reference logits on the same tokens (Sec. 5,
+    Table 8): the packed head's top-k ids, the dense top-1 id (ties: smaller id), KL(dense
+    || packed) and the packed log-sum-exp, all from the fp64 packed logits."""
+    yp = logits(head, H_bits)
+    yd = np.asarray(y_dense, dtype=np.float64)
+    m = yp.max(axis=1)
+    return {"topk": topk_ids(yp, k), "top1_dense": np.argmax(yd, axis=1),
+            "kl": kl_dense_packed(yd, yp),
+            "lse": m + np.log(np.exp(yp - m[:, None]).sum(axis=1)), "y_packed": yp}
 
 
 def packed_nbytes(head: dict) -> int:

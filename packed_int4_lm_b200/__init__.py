@@ -21,7 +21,7 @@ import torch
 from . import _lib, pack
 from ._lib import ArcheadError, ArcheadHead
 
-__all__ = ["DeviceHead", "logits", "nll", "logits_host", "nll_host", "dequant", "check",
+__all__ = ["DeviceHead", "logits", "nll", "agreement", "logits_host", "nll_host", "dequant", "check",
            "last_launches", "profile", "profile_read", "ArcheadError", "pack"]
 
 _KEYS = ("r_nib", "r_code", "r_super", "Ac", "sAc", "Bc", "sBc", "Aw", "sAw", "Bw", "sBw")
@@ -38,17 +38,24 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
     return t.data_ptr()
 
 
+FMT_SC4, FMT_ROW8 = 0, 1  # archead_format
+
+
 class DeviceHead:
-    """A packed head resident in device memory, in the library's device layout."""
+    """A head resident in device memory: the packed ARCHead head in the library's device
+    layout, or (format "row8") the Row INT8 baseline head."""
 
     def __init__(self, meta: dict, tensors: dict):
         self.V, self.D = int(meta["V"]), int(meta["D"])
         self.r_c, self.r_r, self.g = int(meta["r_c"]), int(meta["r_r"]), int(meta["g"])
+        self.format = FMT_ROW8 if meta.get("format") == "row8" else FMT_SC4
         self.tensors = tensors  # keeps the device buffers alive
         s = ArcheadHead()
-        s.V, s.D, s.r_c, s.r_r, s.g, s.reserved = self.V, self.D, self.r_c, self.r_r, self.g, 0
+        s.V, s.D, s.r_c, s.r_r, s.g = self.V, self.D, self.r_c, self.r_r, self.g
+        s.format = self.format
         for k in _KEYS:
-            setattr(s, k, _ptr(tensors[k]))
+            setattr(s, k, _ptr(tensors.get(k)))
+        s.row_scale = _ptr(tensors.get("row_scale"))
         self.struct = s
 
     @property
@@ -61,6 +68,10 @@ class DeviceHead:
     @classmethod
     def from_canonical(cls, head: dict, device="cuda", stream=None) -> "DeviceHead":
         dev = torch.device(device)
+        if head.get("format") == "row8":  # INT8 V x D row-major and FP32 row scales
+            up = {"r_nib": torch.from_numpy(np.ascontiguousarray(head["q8"]).view(np.uint8)).to(dev),
+                  "row_scale": torch.from_numpy(np.ascontiguousarray(head["row_scale"])).to(dev)}
+            return cls(head, up)
         up = {}
         Vpad = (int(head["V"]) + 127) // 128 * 128
         for k in _KEYS:
@@ -176,6 +187,29 @@ def vocab_parallel_nll(H: torch.Tensor, dh: DeviceHead, targets: torch.Tensor, v
     return nll_merge(torch.stack(gathered))
 
 
+def agreement(H: torch.Tensor, dh: DeviceHead, Y_dense: torch.Tensor, k: int = 10,
+              stream=None) -> dict:
+    """archead_agreement: per token the ids of the k largest packed logits ("topk", N x k
+    int32, decreasing, equal logits by smaller id), the dense argmax ("top1_dense", N),
+    KL(P_dense || P_packed) in nats ("kl", N) and the packed log-sum-exp ("lse", N), all
+    on the device.  Y_dense: N x V float32 reference logits on the same device."""
+    _check_H(H, dh)
+    N = H.shape[0]
+    if (Y_dense.dtype != torch.float32 or tuple(Y_dense.shape) != (N, dh.V)
+            or not Y_dense.is_cuda or not Y_dense.is_contiguous()):
+        raise ValueError(f"Y_dense must be a contiguous float32 CUDA tensor of shape ({N}, {dh.V})")
+    dev = H.device
+    out = {"topk": torch.empty(N, k, dtype=torch.int32, device=dev),
+           "top1_dense": torch.empty(N, dtype=torch.int32, device=dev),
+           "kl": torch.empty(N, dtype=torch.float32, device=dev),
+           "lse": torch.empty(N, dtype=torch.float32, device=dev)}
+    _lib.check(_lib.lib().archead_agreement(
+        H.data_ptr(), ctypes.byref(dh.struct), Y_dense.data_ptr(), int(k),
+        *[out[x].data_ptr() if N else None for x in ("topk", "top1_dense", "kl", "lse")],
+        N, *dh.shape_args, _stream_handle(stream)), "archead_agreement")
+    return out
+
+
 def logits_host(H: torch.Tensor, dh: DeviceHead, out: Optional[torch.Tensor] = None,
                 stream=None) -> torch.Tensor:
     """archead_logits_host: host H in, host Y out (copies inside the call, synchronous)."""
@@ -207,7 +241,7 @@ def nll_host(H: torch.Tensor, dh: DeviceHead, targets: torch.Tensor,
 def dequant(dh: DeviceHead, row0: int = 0, nrows: Optional[int] = None, stream=None) -> dict:
     """FP32 dequantised components via the archead_dequant hook (for bit-exact checks)."""
     nrows = dh.V - row0 if nrows is None else nrows
-    dev = dh.tensors["r_code"].device
+    dev = dh.tensors["r_nib"].device
     out = {
         "R": torch.empty(nrows, dh.D, device=dev),
         "Ac": torch.empty(nrows, dh.r_c, device=dev),

@@ -26,10 +26,11 @@ class ArcheadHead(ctypes.Structure):
     _fields_ = [
         ("V", c_i64), ("D", c_i64),
         ("r_c", ctypes.c_int32), ("r_r", ctypes.c_int32), ("g", ctypes.c_int32),
-        ("reserved", ctypes.c_int32),
+        ("format", ctypes.c_int32),
         ("r_nib", c_vp), ("r_code", c_vp), ("r_super", c_vp),
         ("Ac", c_vp), ("sAc", c_vp), ("Bc", c_vp), ("sBc", c_vp),
         ("Aw", c_vp), ("sAw", c_vp), ("Bw", c_vp), ("sBw", c_vp),
+        ("row_scale", c_vp),
     ]
 
 
@@ -54,6 +55,8 @@ _SIGS = {
     "archead_nll_partials": (c_int, [c_vp, ctypes.POINTER(ArcheadHead), c_vp, c_i64, c_i64,
                                      c_vp, c_i64, c_i64, c_i64, c_int, c_int, c_int, c_vp]),
     "archead_nll_merge": (c_int, [c_vp, c_int, c_i64, c_vp, c_vp]),
+    "archead_agreement": (c_int, [c_vp, ctypes.POINTER(ArcheadHead), c_vp, c_int, c_vp, c_vp,
+                                  c_vp, c_vp, c_i64, c_i64, c_i64, c_int, c_int, c_int, c_vp]),
     "archead_profile": (c_int, [c_int]),
     "archead_test_hooks": (c_int, [ctypes.c_longlong, c_int]),
     "archead_profile_read": (c_int, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(c_int)]),

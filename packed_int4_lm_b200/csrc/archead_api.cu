@@ -80,6 +80,13 @@ int check_head(const archead_head* h, int64_t N, int64_t V, int64_t D, int r_c, 
     return ARCHEAD_ERR_SHAPE;
   if (!(g == 32 || g == 64 || g == 128 || g == 256) || D % g != 0) return ARCHEAD_ERR_SHAPE;
   if (r_c < 0 || r_c > 128 || r_r < 0 || r_r > 128) return ARCHEAD_ERR_SHAPE;
+  if (h->format == ARCHEAD_FMT_ROW8) {  // Row INT8: weights and row scales only
+    if (r_c != 0 || r_r != 0) return ARCHEAD_ERR_SHAPE;
+    if (!h->r_nib || !h->row_scale) return ARCHEAD_ERR_NULLPTR;
+    if (!aligned(h->r_nib, 16) || !aligned(h->row_scale, 16)) return ARCHEAD_ERR_ALIGN;
+    return ARCHEAD_OK;
+  }
+  if (h->format != ARCHEAD_FMT_SC4) return ARCHEAD_ERR_SHAPE;
   if (!h->r_nib || !h->r_code || !h->r_super) return ARCHEAD_ERR_NULLPTR;
   if (r_c > 0 && (!h->Ac || !h->sAc || !h->Bc || !h->sBc)) return ARCHEAD_ERR_NULLPTR;
   if (r_r > 0 && (!h->Aw || !h->sAw || !h->Bw || !h->sBw)) return ARCHEAD_ERR_NULLPTR;
@@ -182,9 +189,11 @@ int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* ta
   // fits; larger N: the tensor-memory (tcgen05) kernel when its shared-memory rings fit;
   // other shapes: the token-block warp-MMA kernel.  All three have a fused
   // split-vocabulary NLL epilogue.
-  const DecPlan dplan = dec_plan(s, nll_mode);
+  // Row INT8 heads run on the token-block warp-MMA kernel only
+  const bool row8 = head->format == ARCHEAD_FMT_ROW8;
+  const DecPlan dplan = row8 ? DecPlan{0, 0, 0} : dec_plan(s, nll_mode);
   if (dplan.nt8 > 0) return run_dec(H, head, Y, targets, nll, s, dplan, ds, st, shard);
-  const TcPlan plan = s.N > 8 ? tc_plan(s, nll_mode) : TcPlan{0, 0, 0, 0};
+  const TcPlan plan = s.N > 8 && !row8 ? tc_plan(s, nll_mode) : TcPlan{0, 0, 0, 0};
   const bool use_tc = plan.nt > 0;
   const int64_t tb = use_tc ? plan.nt : residual_token_block(s.N);
   const int64_t Npad = (s.N + tb - 1) / tb * tb;
@@ -354,6 +363,55 @@ int archead_nll_merge(const float* partials, int G, int64_t N, float* nll_out, v
   return ARCHEAD_OK;
 }
 
+int archead_agreement(const uint16_t* H, const archead_head* head, const float* Y_dense,
+                      int k, int32_t* topk_out, int32_t* top1_dense_out, float* kl_out,
+                      float* lse_out, int64_t N, int64_t V, int64_t D, int r_c, int r_r, int g,
+                      void* stream) {
+  int rc = check_head(head, N, V, D, r_c, r_r, g);
+  if (rc) return rc;
+  if (k < 1 || k > 16) return ARCHEAD_ERR_SHAPE;
+  if (N == 0) {
+    t_last_launches = 0;
+    return ARCHEAD_OK;
+  }
+  if (!H || !Y_dense || !topk_out || !top1_dense_out || !kl_out) return ARCHEAD_ERR_NULLPTR;
+  if (!aligned(H, 16) || !aligned(Y_dense, 4) || !aligned(topk_out, 4) ||
+      !aligned(top1_dense_out, 4) || !aligned(kl_out, 4) || (lse_out && !aligned(lse_out, 4)))
+    return ARCHEAD_ERR_ALIGN;
+  DeviceState* ds;
+  rc = current_state(&ds);
+  if (rc) return rc;
+  const Shapes s = make_shapes(N, V, D, r_c, r_r, g);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t tb = residual_token_block(N);
+  const int64_t Npad = (N + tb - 1) / tb * tb;
+  const int64_t nvblk = residual_gemm_vblocks(s);
+  Carve cv;
+  const size_t o_hh = cv.take((size_t)Npad * D * 2);
+  const size_t o_t = cv.take((size_t)N * (r_c + r_r) * 4);
+  const size_t o_st = cv.take((size_t)N * nvblk * 6 * 4);
+  const size_t o_kv = cv.take((size_t)N * nvblk * k * 4);
+  const size_t o_ki = cv.take((size_t)N * nvblk * k * 4);
+  void* base = nullptr;
+  if (cudaMallocFromPoolAsync(&base, cv.off, ds->pool, st) != cudaSuccess) {
+    cudaGetLastError();
+    return ARCHEAD_ERR_NOMEM;
+  }
+  char* b = static_cast<char*>(base);
+  int launches = 0;
+  __half* Hh = reinterpret_cast<__half*>(b + o_hh);
+  float* t = reinterpret_cast<float*>(b + o_t);
+  cudaError_t e = launch_prologue(H, head, s, Npad, Hh, t, ds->err, st, &launches);
+  if (e == cudaSuccess)
+    e = launch_agreement(Hh, t, head, s, Y_dense, k, reinterpret_cast<float*>(b + o_st),
+                         reinterpret_cast<float*>(b + o_kv), reinterpret_cast<int*>(b + o_ki),
+                         topk_out, top1_dense_out, kl_out, lse_out, st, &launches);
+  cudaFreeAsync(base, st);
+  if (e != cudaSuccess) return ARCHEAD_ERR_CUDA;
+  t_last_launches = launches;
+  return ARCHEAD_OK;
+}
+
 int archead_logits_host(const uint16_t* H_host, const archead_head* head, float* Y_host,
                         int64_t N, int64_t V, int64_t D, int r_c, int r_r, int g,
                         void* stream) {
@@ -439,6 +497,7 @@ int archead_dequant(const archead_head* head, int64_t row0, int64_t nrows, float
   if (!head) return ARCHEAD_ERR_NULLPTR;
   int rc = check_head(head, 0, head->V, head->D, head->r_c, head->r_r, head->g);
   if (rc) return rc;
+  if (head->format != ARCHEAD_FMT_SC4) return ARCHEAD_ERR_UNSUPPORTED;
   if (row0 < 0 || nrows < 0 || row0 + nrows > head->V) return ARCHEAD_ERR_SHAPE;
   return launch_dequant(head, row0, nrows, R_out, Ac_out, Aw_out, Bc_out, Bw_out,
                         static_cast<cudaStream_t>(stream)) == cudaSuccess

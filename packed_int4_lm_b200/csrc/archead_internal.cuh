@@ -99,6 +99,14 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
 }
 
+__device__ __forceinline__ uint2 ldg_stream8(const void* p) {
+  uint2 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];\n"
+               : "=r"(r.x), "=r"(r.y)
+               : "l"(p));
+  return r;
+}
+
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   uint4 r;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];\n"
@@ -205,6 +213,14 @@ cudaError_t launch_residual_gemm(const __half* Hh, const float* t, const archead
                                  float2* part, float* tlogit, cudaStream_t st, int* launches,
                                  int mode);
 int residual_gemm_vblocks(const Shapes& s);
+// Agreement with a dense reference head (mode 2 of the warp-MMA kernel, then a merge):
+// per token the ids of the topk largest packed logits, the dense argmax, KL(dense ||
+// packed) and the packed log-sum-exp.  Scratch: astat N x nvblk x 6 floats, akval and akid
+// N x nvblk x topk each (nvblk = residual_gemm_vblocks).
+cudaError_t launch_agreement(const __half* Hh, const float* t, const archead_head* head,
+                             const Shapes& s, const float* Yd, int topk, float* astat,
+                             float* akval, int* akid, int32_t* topk_out, int32_t* top1_dense,
+                             float* kl_out, float* lse_out, cudaStream_t st, int* launches);
 int64_t residual_token_block(int64_t N);  // rows of the zero-padded FP16 copy of H
 
 // nll[n] from the partials; a target outside [0, V) gives NaN and sets kErrTarget.

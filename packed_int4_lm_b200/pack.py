@@ -37,7 +37,7 @@ import torch
 
 __all__ = ["build_head", "q8_rowwise", "q8_groupwise", "sc4", "pack_nibbles",
            "metric_transform", "randomized_svd", "dequant_head_torch", "storage_ratio",
-           "save_head", "load_head", "serialized_nbytes", "shard_rows"]
+           "save_head", "load_head", "serialized_nbytes", "shard_rows", "build_row8_head"]
 
 
 def _rne(x: torch.Tensor) -> torch.Tensor:
@@ -207,6 +207,18 @@ def build_head(W: torch.Tensor, H_cal: torch.Tensor, r_c: int, r_r: int, g: int,
     return head
 
 
+def build_row8_head(W: torch.Tensor, g: int = 128) -> dict:
+    """The Row INT8 baseline head the paper compares with (Sec. 5, Tables 3 and 8): every
+    row of W quantized to INT8 with its own FP32 scale (the row-wise Q8 above: absmax / 127,
+    round to nearest even, clamp to +-127), no core and no correction.  `g` is recorded only
+    as the nominal group size the library's argument checks expect."""
+    V, D = W.shape
+    q, s, _ = q8_rowwise(W.to(torch.float64))
+    return {"format": "row8", "V": int(V), "D": int(D), "r_c": 0, "r_r": 0, "g": int(g),
+            "q8": q.detach().cpu().contiguous().numpy(),
+            "row_scale": s.detach().cpu().contiguous().numpy()}
+
+
 def dequant_head_torch(head: dict, device="cpu", dtype=torch.float64) -> torch.Tensor:
     """Dense W_hat from a canonical head with torch ops (construction-side diagnostics)."""
     g = head["g"]
@@ -236,9 +248,10 @@ def dequant_head_torch(head: dict, device="cpu", dtype=torch.float64) -> torch.T
 
 
 def storage_ratio(head: dict) -> float:
-    """Packed persistent bytes over the BF16 dense head's bytes."""
-    nb = sum(np.asarray(head[k]).nbytes for k in
-             ("r_nib", "r_code", "r_super", "Ac", "sAc", "Bc", "sBc", "Aw", "sAw", "Bw", "sBw"))
+    """Persistent bytes over the BF16 dense head's bytes."""
+    keys = (("q8", "row_scale") if head.get("format") == "row8" else
+            ("r_nib", "r_code", "r_super", "Ac", "sAc", "Bc", "sBc", "Aw", "sAw", "Bw", "sBw"))
+    nb = sum(np.asarray(head[k]).nbytes for k in keys)
     return nb / (2.0 * head["V"] * head["D"])
 
 

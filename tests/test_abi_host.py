@@ -27,7 +27,7 @@ def test_exports_every_declared_function(L):
 
 
 def test_abi_version_and_strerror(L):
-    assert L.archead_abi_version() == 1
+    assert L.archead_abi_version() == 2
     for code in STATUS_CODE.values():
         s = L.archead_strerror(code)
         assert s and s != b"unknown status"

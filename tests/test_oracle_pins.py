@@ -264,3 +264,68 @@ def test_packed_nbytes_closed_form(V, D, r_c, r_r, g):
     assert oracle.packed_nbytes(head) == closed
     # against the dense BF16 head: INT4 plus its code and super-scale overheads
     assert oracle.packed_nbytes(head) < 2 * V * D
+
+
+# ---------------------------------------------------------------------------------------
+# agreement with a dense head (Sec. 5, Table 8: top-1 / top-k agreement and KL)
+# ---------------------------------------------------------------------------------------
+def test_topk_ids_order_and_ties():
+    y = np.array([[1.0, 3.0, 3.0, -2.0, 3.0, 0.5],
+                  [0.0, 0.0, 0.0, 0.0, 0.0, 0.0]])
+    assert oracle.topk_ids(y, 4).tolist() == [[1, 2, 4, 0], [0, 1, 2, 3]]
+    assert oracle.topk_ids(y[:, :2], 4).tolist() == [[1, 0, -1, -1], [0, 1, -1, -1]]
+
+
+def test_kl_matches_torch_and_its_special_cases():
+    rng = np.random.default_rng(3)
+    yd = rng.normal(size=(5, 50)) * 3
+    yp = yd + rng.normal(size=(5, 50)) * 0.3
+    ours = oracle.kl_dense_packed(yd, yp)
+    ref = torch.nn.functional.kl_div(torch.log_softmax(torch.tensor(yp), 1),
+                                     torch.log_softmax(torch.tensor(yd), 1), log_target=True,
+                                     reduction="none").sum(1).numpy()
+    assert np.allclose(ours, ref, rtol=1e-10, atol=1e-12)
+    assert np.all(ours > 0)
+    assert np.allclose(oracle.kl_dense_packed(yd, yd), 0.0, atol=1e-12)
+    # a constant added to either row changes neither distribution
+    assert np.allclose(oracle.kl_dense_packed(yd + 7.0, yp - 3.0), ours, atol=1e-12)
+    # two logits: closed form p log(p / q) + (1 - p) log((1 - p) / (1 - q))
+    d = np.array([[0.0, math.log(3.0)]])  # p = (1/4, 3/4)
+    q = np.array([[0.0, 0.0]])            # q = (1/2, 1/2)
+    closed = 0.25 * math.log(0.5) + 0.75 * math.log(1.5)
+    assert abs(oracle.kl_dense_packed(d, q)[0] - closed) < 1e-14
+
+
+def test_agreement_of_a_head_with_its_own_logits():
+    head = random_canonical_head(70, 128, 2, 2, 64, seed=4)
+    Hb = np.asarray(torch.randn(3, 128).to(torch.bfloat16).view(torch.int16).numpy()).view(np.uint16)
+    yp = oracle.logits(head, Hb)
+    a = oracle.agreement(head, Hb, yp, 5)
+    assert np.array_equal(a["top1_dense"], a["topk"][:, 0])
+    assert np.allclose(a["kl"], 0.0, atol=1e-12)
+    from scipy.special import logsumexp
+    assert np.allclose(a["lse"], logsumexp(yp, axis=1), rtol=1e-12)
+
+
+def test_row8_head_single_entries_and_integer_matmul():
+    """The Row INT8 baseline (Sec. 5): W[v, d] = q8[v, d] * s[v].  A single nonzero entry
+    lands at its row and column with its row's scale; unit scales reduce the logits to an
+    exact integer matmul."""
+    V, D = 5, 128
+    q8 = np.zeros((V, D), np.int8)
+    q8[3, 77] = -100
+    s = np.array([1.0, 2.0, 0.5, 0.25, 4.0], np.float32)
+    head = {"format": "row8", "V": V, "D": D, "r_c": 0, "r_r": 0, "g": 128, "q8": q8, "row_scale": s}
+    W = oracle.dense_head_rows(head)
+    expect = np.zeros((V, D))
+    expect[3, 77] = -25.0
+    assert np.array_equal(W, expect)
+    Hb = _identity_H(D)
+    assert np.array_equal(oracle.logits(head, Hb), expect.T)
+    rng = np.random.default_rng(0)
+    q8 = rng.integers(-127, 128, size=(40, 256)).astype(np.int8)
+    head = {"format": "row8", "V": 40, "D": 256, "r_c": 0, "r_r": 0, "g": 128, "q8": q8,
+            "row_scale": np.ones(40, np.float32)}
+    hi = rng.integers(-20, 21, size=(3, 256))
+    Hb = _bf16_bits_of(hi.astype(np.float32))
+    assert np.array_equal(oracle.logits(head, Hb), (hi @ q8.astype(np.int64).T).astype(np.float64))
