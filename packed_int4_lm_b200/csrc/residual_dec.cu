@@ -427,6 +427,7 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
     // layout, so one bulk copy).
     if (lane == 0) {
       bool ok = true;
+      const uint64_t pol_first = tc::l2_policy_evict_first();  // the head streams once
       const uint32_t hbytes = (uint32_t)(NTOK * D * 2 + (int64_t)nkb * NTOK * 4);
       // The H image comes from the prologue kernel, which may still be running (this
       // kernel is a programmatic dependent launch): the packed stream starts at once, and
@@ -472,8 +473,8 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
           }
           tc::fence_proxy_async_smem();
           tc::mbar_arrive_expect_tx(&p_full[st], bytes);
-          tc::bulk_g2s(pk + (size_t)st * 2 * kDecPk, p.nib + ((T * nkb + kb) << 13), bytes,
-                       &p_full[st]);
+          tc::bulk_g2s_hint(pk + (size_t)st * 2 * kDecPk, p.nib + ((T * nkb + kb) << 13), bytes,
+                            &p_full[st], pol_first);
           ++np;
         }
         u += kb1 - kb0;
@@ -793,7 +794,7 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
               const int64_t tok = 8 * j + 2 * tq + e;
-              if (tok < p.N) p.Y[tok * p.V + v] = y[j][2 * h + e];
+              if (tok < p.N) __stcs(p.Y + tok * p.V + v, y[j][2 * h + e]);
             }
         }
       } else {

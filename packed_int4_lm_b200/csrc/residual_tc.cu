@@ -714,7 +714,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
               float* yp = p.Y + t16 * p.V + v;
 #pragma unroll
               for (int q = 0; q < 16; ++q) {
-                if (q < nq) *yp = y[q];
+                if (q < nq) __stcs(yp, y[q]);  // streaming: Y does not displace the B image
                 yp += p.V;
               }
             }
