@@ -74,19 +74,22 @@ __global__ void __launch_bounds__(256) lowrank_t_kernel(
     const int8_t* bq = reinterpret_cast<const int8_t*>(&braw);
 #pragma unroll
     for (int k = 0; k < 8; ++k) b[k] = __fmul_rn((float)bq[k], s);
+    // all kTN token rows are loaded (rows past N repeat the last one, and their sums are
+    // never stored), so the loads carry no predicate and are in flight together
+    uint4 hv[kTN];
+#pragma unroll
+    for (int n = 0; n < kTN; ++n)
+      hv[n] = __ldg(reinterpret_cast<const uint4*>(H + (n0 + (n < nv ? n : nv - 1)) * D + d0));
 #pragma unroll
     for (int n = 0; n < kTN; ++n) {
-      if (n < nv) {
-        uint4 hv = *reinterpret_cast<const uint4*>(H + (n0 + n) * D + d0);
-        uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
-        float a = acc[n];
+      const uint32_t hw[4] = {hv[n].x, hv[n].y, hv[n].z, hv[n].w};
+      float a = acc[n];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          a = fmaf(__uint_as_float(hw[k] << 16), b[2 * k], a);
-          a = fmaf(__uint_as_float(hw[k] & 0xFFFF0000u), b[2 * k + 1], a);
-        }
-        acc[n] = a;
+      for (int k = 0; k < 4; ++k) {
+        a = fmaf(__uint_as_float(hw[k] << 16), b[2 * k], a);
+        a = fmaf(__uint_as_float(hw[k] & 0xFFFF0000u), b[2 * k + 1], a);
       }
+      acc[n] = a;
     }
   }
   // block reduction of the kTN sums
