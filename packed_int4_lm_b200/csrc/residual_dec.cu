@@ -5,23 +5,26 @@
 //
 // for N <= 16 tokens, where every packed byte is used by at most 16 tokens and the kernel
 // has to stream the head at HBM speed.  Design:
-//  * persistent grid, one CTA per SM: warp 8 is a producer that bulk-copies (TMA engine,
-//    no tensor map, no multicast) the 8 KB packed blocks of 128-row tiles into a deep
-//    shared-memory ring, plus each tile's group codes and INT8 factor rows; warps 0-7
-//    each own 16 rows of the tile;
+//  * persistent grid, one CTA per SM: the last warp is a producer that bulk-copies (TMA
+//    engine, no tensor map, no multicast) two-block stages of the 8 KB packed blocks of
+//    128-row tiles into a shared-memory ring, plus each tile's group codes and INT8 factor
+//    rows; each consumer warp owns 16 rows of the tile (for N <= 8 two warps per 16 rows,
+//    taking the even and the odd stages, iterating over their own stages only);
 //  * the FP16 hidden states of all (<= 16) tokens stay resident in shared memory for the
 //    whole launch, stored with a chunk swizzle that makes the B-fragment reads
 //    conflict-free;
 //  * A fragments come from the ring with ldmatrix: in the tiled device layout the 16-byte
 //    chunk i of 8 consecutive rows is 128 contiguous bytes, so each 8x8 matrix load is
 //    conflict-free, and thread (g, q) receives word q of chunk i of row g -- exactly the
-//    eight columns it dequantises (exact FP16 q*c) into an m16n8k16 fragment;
+//    eight columns it feeds into an m16n8k16 fragment (raw magic-number nibble reads with
+//    one group code per 128-column block, exact FP16 q*c otherwise);
 //  * the work is split evenly over CTAs in units of (tile, 128-column block), so all CTAs
 //    finish together.  A tile split between CTAs is finished by the CTA that arrives
 //    last (an atomic counter per tile, no waiting): it sums the partial accumulators of
 //    all contributors in CTA order, so the result does not depend on arrival order;
-//  * epilogue: S_v times the accumulator plus the rank terms in FP32 from t; MODE 1
-//    writes split-vocabulary (max, sum exp) partials and target logits instead of Y.
+//  * epilogue: S_v times the accumulator plus the rank terms (mma.sync on the INT8 factor
+//    rows and FP16 hi / lo pieces of t, or FP32 from t); MODE 1 writes split-vocabulary
+//    (max, sum exp) partials and target logits instead of Y.
 // Every mbarrier wait is bounded; a wait that gives up sets the device error word and the
 // warp skips its remaining waits, so the launch always ends.
 #include "tc_common.cuh"
@@ -95,8 +98,8 @@ __host__ __device__ inline DecSmem dec_smem(int64_t D, int G, int r_c, int r_r, 
   constexpr int NTOK = DecCfg<NT8>::NTOK;
   DecSmem m;
   size_t o = 0;
-  m.h = o;  // H image [NTOK x D] FP16, then corr [D / 128][NTOK] FP32
-  o += dec_round16((size_t)NTOK * D * 2 + (size_t)(D / 128) * NTOK * 4);
+  m.h = o;  // H image [NTOK x D] FP16, then corr quads [D / 128][NTOK / 2] float4
+  o += dec_round16((size_t)NTOK * D * 2 + (size_t)(D / 128) * NTOK * 8);
   m.pk = o;  // ring of sp stages of two packed blocks
   o += (size_t)sp * 2 * kDecPk;
   m.codes = o;  // [2][128 x G]
@@ -140,7 +143,9 @@ __device__ __forceinline__ bool dec_wait(uint64_t* bar, uint32_t parity, unsigne
 }
 
 // Prologue of this path: the resident H image (zero rows up to NTOK), followed by the
-// offset corrections corr[kb][n], and zeroed tile counters.  One warp per (token, block);
+// offset corrections, and zeroed tile counters.  The corrections of block kb are stored as
+// quads (corr[kb][2i], corr[kb][2i + 1], corr[kb][2i], corr[kb][2i + 1]) for token pairs
+// i: a quad is the C operand that starts an m16n8k16 chain of the decode kernel.  One warp per (token, block);
 // lane l converts columns 4l .. 4l + 3 of the block.
 //
 // With scale_b (one group code per 128-column block), the kernel feeds the MMA the raw
@@ -161,7 +166,7 @@ __device__ __forceinline__ void dec_convert_h(const uint16_t* __restrict__ H,
   const int lane = threadIdx.x & 31;
   const int64_t gw = (blk * (int64_t)blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = (nblk * (int64_t)blockDim.x) >> 5;
-  float* corr = reinterpret_cast<float*>(img + (int64_t)ntok * D);  // [nkb][ntok]
+  float* corr = reinterpret_cast<float*>(img + (int64_t)ntok * D);  // [nkb][ntok / 2] quads
   bool bad = false;
   for (int64_t wi = gw; wi < (int64_t)ntok * nkb; wi += nw) {
     const int64_t n = wi / nkb, kb = wi - n * nkb;
@@ -189,7 +194,10 @@ __device__ __forceinline__ void dec_convert_h(const uint16_t* __restrict__ H,
     *reinterpret_cast<uint2*>(img + dec_h_offset(n, d, D)) = make_uint2(lo, hi);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    if (lane == 0) corr[kb * ntok + n] = scale_b ? -sum : 0.f;
+    if (lane == 0) {
+      const int64_t q = (kb * (ntok / 2) + (n >> 1)) * 4 + (n & 1);
+      corr[q] = corr[q + 2] = scale_b ? -sum : 0.f;
+    }
   }
   for (int64_t i = blk * (int64_t)blockDim.x + threadIdx.x; i < n_counters;
        i += nblk * (int64_t)blockDim.x)
@@ -283,16 +291,6 @@ __host__ __device__ __forceinline__ bool dec_arow_copy(int64_t rows, int r_c, in
   return ((rows * r_c) % 16) == 0 && ((rows * r_r) % 16) == 0;
 }
 
-// m16n8k16 FP16 MMA, D = A * B + (c0, c1, c0, c1): the chain's start value per accumulator column pair.
-__device__ __forceinline__ void mma_f16_16816_c(float d[4], const uint32_t a[4], uint32_t b0,
-                                                uint32_t b1, float c0, float c1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-      "{%8, %9}, {%10, %11, %10, %11};\n"
-      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(c0), "f"(c1));
-}
-
 // Raw magic-number reads of the eight nibbles of a device-layout word (no FP16 math):
 // pairs 0 and 2 read 1032 + q, pairs 1 and 3 read 1152 + 16 q (see dec_convert_h).
 __device__ __forceinline__ void nibble_reads(uint32_t w, uint32_t x[4]) {
@@ -303,28 +301,38 @@ __device__ __forceinline__ void nibble_reads(uint32_t w, uint32_t x[4]) {
   x[3] = and_xor(w2, 0x00F000F0u, 0x64806480u);
 }
 
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];\n"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a));
+  return v;
+}
+
+// m16n8k16 FP16 MMA whose chain starts from the quad c (C operand).
+__device__ __forceinline__ void mma_f16_16816_q(float d[4], const uint32_t a[4], uint32_t b0,
+                                                uint32_t b1, uint4 c) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%10, %11, %12, %13};\n"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(c.x), "r"(c.y),
+        "r"(c.z), "r"(c.w));
+}
+
 // NB (1 or 2) consecutive blocks with one group code each (g >= 128): raw nibble reads
-// (nibble_reads) times the resident B image, one chain of eight MMAs per block, plus the
-// block's negated offset constant (corr: the chain's start value for one token block,
-// added after the chain for two), then acc += code * (chain + offset).  The blocks'
-// chains are independent; one chain per block needs no adds to combine partial chains,
-// which costs less than the longer MMA dependency.
+// (nibble_reads) times the resident B image, one chain of eight MMAs per block starting
+// from the block's negated offset constant (a quad of corr), then acc += code * chain.
+// hs: shared address of this thread's H row (token gid) at block kb2, chunk 0; cq: shared
+// address of its corr quad at block kb2.
 template <int NT8, int NB>
 __device__ __forceinline__ void dec_blocks_q(const uint32_t (&wlo)[2][4],
                                              const uint32_t (&whi)[2][4],
                                              const uint32_t (&clo)[2], const uint32_t (&chi)[2],
-                                             const unsigned char* Hb, const int (&hrow)[NT8],
-                                             const int (&hoff)[4], const float* corr, int kb2,
-                                             int tq, float (&acc)[NT8][4]) {
+                                             uint32_t hs, uint32_t hj, const uint32_t (&hoff)[4],
+                                             uint32_t cq, float (&acc)[NT8][4]) {
   constexpr int NTOK = 8 * NT8;
   float t[NB][NT8][4];
-  float2 ncr[NB][NT8];
-#pragma unroll
-  for (int b = 0; b < NB; ++b)
-#pragma unroll
-    for (int j = 0; j < NT8; ++j)
-      if (NT8 == 1)
-        ncr[b][j] = *reinterpret_cast<const float2*>(corr + (kb2 + b) * NTOK + 8 * j + 2 * tq);
 #pragma unroll
   for (int c = 0; c < 4; ++c)
 #pragma unroll
@@ -336,12 +344,11 @@ __device__ __forceinline__ void dec_blocks_q(const uint32_t (&wlo)[2][4],
       const uint32_t a1[4] = {xa[2], xb[2], xa[3], xb[3]};
 #pragma unroll
       for (int j = 0; j < NT8; ++j) {
-        const uint4 hv =
-            *reinterpret_cast<const uint4*>(Hb + hrow[j] + (kb2 + b) * 256 + hoff[c]);
-        if (c == 0)  // chain start: the negated offset (one token block), or zero
-          mma_f16_16816_c(t[b][j], a0, hv.x, hv.y, NT8 == 1 ? ncr[b][j].x : 0.f,
-                          NT8 == 1 ? ncr[b][j].y : 0.f);
-        else mma_f16_16816(t[b][j], a0, hv.x, hv.y);
+        const uint4 hv = lds128(hs + j * hj + b * 256 + hoff[c]);
+        if (c == 0)
+          mma_f16_16816_q(t[b][j], a0, hv.x, hv.y, lds128(cq + (b * (NTOK / 2) + 4 * j) * 16));
+        else
+          mma_f16_16816(t[b][j], a0, hv.x, hv.y);
         mma_f16_16816(t[b][j], a1, hv.z, hv.w);
       }
     }
@@ -350,14 +357,10 @@ __device__ __forceinline__ void dec_blocks_q(const uint32_t (&wlo)[2][4],
     const float fl = (float)clo[b], fh = (float)chi[b];
 #pragma unroll
     for (int j = 0; j < NT8; ++j) {
-      if (NT8 != 1)
-        ncr[b][j] = *reinterpret_cast<const float2*>(corr + (kb2 + b) * NTOK + 8 * j + 2 * tq);
-      // two token blocks: the offset is added here (fewer registers live across the chain)
-      const float ox = NT8 == 1 ? 0.f : ncr[b][j].x, oy = NT8 == 1 ? 0.f : ncr[b][j].y;
-      acc[j][0] = fmaf(fl, t[b][j][0] + ox, acc[j][0]);
-      acc[j][1] = fmaf(fl, t[b][j][1] + oy, acc[j][1]);
-      acc[j][2] = fmaf(fh, t[b][j][2] + ox, acc[j][2]);
-      acc[j][3] = fmaf(fh, t[b][j][3] + oy, acc[j][3]);
+      acc[j][0] = fmaf(fl, t[b][j][0], acc[j][0]);
+      acc[j][1] = fmaf(fl, t[b][j][1], acc[j][1]);
+      acc[j][2] = fmaf(fh, t[b][j][2], acc[j][2]);
+      acc[j][3] = fmaf(fh, t[b][j][3], acc[j][3]);
     }
   }
 }
@@ -376,7 +379,7 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
   const int SP = p.sp;
   const DecSmem m = dec_smem<NT8, MODE>(D, G, p.r_c, p.r_r, SP);
   const unsigned char* Hb = smem + m.h;
-  const float* corr = reinterpret_cast<const float*>(smem + m.h + (size_t)NTOK * D * 2);
+  const uint32_t corr_s = tc::smem_u32(smem + m.h + (size_t)NTOK * D * 2);
   unsigned char* pk = smem + m.pk;
   unsigned char* cds = smem + m.codes;
   int8_t* arc = reinterpret_cast<int8_t*>(smem + m.arow_c);
@@ -428,7 +431,7 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
     if (lane == 0) {
       bool ok = true;
       const uint64_t pol_first = tc::l2_policy_evict_first();  // the head streams once
-      const uint32_t hbytes = (uint32_t)(NTOK * D * 2 + (int64_t)nkb * NTOK * 4);
+      const uint32_t hbytes = (uint32_t)(NTOK * D * 2 + (int64_t)nkb * NTOK * 8);
       // The H image comes from the prologue kernel, which may still be running (this
       // kernel is a programmatic dependent launch): the packed stream starts at once, and
       // the image is fetched after the prologue grid completes, before the first wait that
@@ -534,6 +537,12 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
   int hoff[4];
 #pragma unroll
   for (int c = 0; c < 4; ++c) hoff[c] = 16 * (c ^ hx);
+  uint32_t hoffu[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) hoffu[c] = (uint32_t)hoff[c];
+  const uint32_t hs0 = tc::smem_u32(Hb) + (uint32_t)hrow[0];
+  const uint32_t hj = (uint32_t)(8 * D * 2);
+  const uint32_t cq0 = corr_s + (uint32_t)tq * 16;
 
   int k = 0, s = 0;
   for (int64_t u = u0; u < u1; ++s) {
@@ -559,17 +568,14 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
 
-    int st = k % SP;
-    uint32_t ph = (uint32_t)(k / SP) & 1u;
-    for (int kb2 = kb0; kb2 < kb1; kb2 += 2, ++k) {
-      if (PAR == 2 && (k & 1) != par) {  // the other warp of the pair takes this stage
-        if (++st == SP) {
-          st = 0;
-          ph ^= 1u;
-        }
-        continue;
-      }
-      ok = dec_wait(&p_full[st], ph, p.err, ok, p.wait_limit);
+    const int nst = (kb1 - kb0 + 1) >> 1;  // stages of this tile segment
+    int i0 = (PAR == 2 && (k & 1) != par) ? 1 : 0;  // this warp's first stage of them
+    int st = (k + i0) % SP;
+    uint32_t ph = (uint32_t)((k + i0) / SP) & 1u;
+    k += nst;
+    for (int i = i0; i < nst; i += PAR) {
+      const int kb2 = kb0 + 2 * i;
+      ok = ok && tc::mbar_wait(&p_full[st], ph, p.err, p.wait_limit);
       const int nb = kb2 + 1 < kb1 ? 2 : 1;
       uint32_t wlo[2][4], whi[2][4];  // [block][chunk]: word tq of rows r_lo, r_hi
       uint32_t clo[2], chi[2];
@@ -592,15 +598,18 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
       }
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&p_empty[st]);
-      if (++st == SP) {
-        st = 0;
+      st += PAR;
+      if (st >= SP) {
+        st -= SP;
         ph ^= 1u;
       }
       if (CPC == 1) {
+        const uint32_t hs = hs0 + (uint32_t)kb2 * 256u;
+        const uint32_t cq = cq0 + (uint32_t)kb2 * (NTOK * 8);
         if (nb == 2)
-          dec_blocks_q<NT8, 2>(wlo, whi, clo, chi, Hb, hrow, hoff, corr, kb2, tq, acc);
+          dec_blocks_q<NT8, 2>(wlo, whi, clo, chi, hs, hj, hoffu, cq, acc);
         else
-          dec_blocks_q<NT8, 1>(wlo, whi, clo, chi, Hb, hrow, hoff, corr, kb2, tq, acc);
+          dec_blocks_q<NT8, 1>(wlo, whi, clo, chi, hs, hj, hoffu, cq, acc);
       } else {
 #pragma unroll
         for (int b = 0; b < 2; ++b) {
@@ -915,7 +924,7 @@ DecPlan dec_plan(const Shapes& s, bool nll) {
 }
 
 size_t dec_image_bytes(const Shapes& s, const DecPlan& pl) {
-  return (size_t)8 * pl.nt8 * s.D * 2 + (size_t)(s.D / 128) * 8 * pl.nt8 * 4;
+  return (size_t)8 * pl.nt8 * s.D * 2 + (size_t)(s.D / 128) * 8 * pl.nt8 * 8;
 }
 size_t dec_partial_bytes(const DecPlan& pl) { return (size_t)pl.grid * 2 * 256 * pl.nt8 * 16; }
 
