@@ -545,6 +545,7 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
   const uint32_t cq0 = corr_s + (uint32_t)tq * 16;
 
   int k = 0, s = 0;
+  bool nready = false;  // this warp's next stage, probed one stage ahead
   for (int64_t u = u0; u < u1; ++s) {
     const int64_t T = u / nkb;
     const int kb0 = (int)(u - T * nkb);
@@ -575,7 +576,7 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
     k += nst;
     for (int i = i0; i < nst; i += PAR) {
       const int kb2 = kb0 + 2 * i;
-      ok = ok && tc::mbar_wait(&p_full[st], ph, p.err, p.wait_limit);
+      if (!nready) ok = ok && tc::mbar_wait(&p_full[st], ph, p.err, p.wait_limit);
       const int nb = kb2 + 1 < kb1 ? 2 : 1;
       uint32_t wlo[2][4], whi[2][4];  // [block][chunk]: word tq of rows r_lo, r_hi
       uint32_t clo[2], chi[2];
@@ -603,6 +604,10 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
         st -= SP;
         ph ^= 1u;
       }
+      // The next stage's barrier is probed now (non-blocking) and its answer used at the
+      // next stage, so the round trip overlaps this stage's arithmetic; a phase seen
+      // complete stays complete until this warp releases the slot.
+      nready = tc::mbar_test(&p_full[st], ph);
       if (CPC == 1) {
         const uint32_t hs = hs0 + (uint32_t)kb2 * 256u;
         const uint32_t cq = cq0 + (uint32_t)kb2 * (NTOK * 8);
