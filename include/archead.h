@@ -30,13 +30,16 @@
  *    0 <= r_c, r_r <= 128; 1 <= V <= 8388480 (65535 blocks of 128 rows); 0 <= N < 2^31;
  *    N == 0 is a successful no-op.  V needs no multiple of any tile: the vocabulary tail
  *    is predicated.
- *  - |H| must stay within the FP16 range (|h| <= 65504); larger or non-finite entries
- *    raise ARCHEAD_ERR_RANGE_H (see archead_logits).  Where the rank terms run on the
- *    tensor cores (r_c and r_r multiples of 16 for N <= 16; every shape for N > 16) the
- *    same holds for the prologue products t = H [Q8(B_c) | Q8(B_w)]^T.  With one group code
- *    per 128 columns (g >= 128, N <= 16) half of the columns of H are stored as H / 16;
- *    such values that fall below the FP16 normal range keep fewer bits, as H's own
- *    rounding to FP16 does.
+ *  - Any finite BF16 H is accepted.  The kernels take FP16 operands, so each token row n
+ *    is scaled by the power of two 2^-e_n, e_n = max(0, ilogb(max_d |h[n, d]|) - 14),
+ *    which brings it below 2^15 exactly, and its logits are multiplied back by 2^e_n (a
+ *    row with max |h| < 2^15 is not scaled).  Non-finite entries of H raise
+ *    ARCHEAD_ERR_RANGE_H.  Where the rank terms run on the tensor cores (r_c and r_r
+ *    multiples of 16 for N <= 16; every shape for N > 16) the scaled prologue products
+ *    t 2^-e_n, t = H [Q8(B_c) | Q8(B_w)]^T, must stay below 65504 in magnitude, or the call
+ *    raises ARCHEAD_ERR_RANGE_H.  Entries of the scaled rows below the FP16 normal range
+ *    (2^-14; with one group code per 128 columns, g >= 128 and N <= 16, half of the
+ *    columns are stored divided by 16) keep fewer bits, as rounding to FP16 does.
  */
 #ifndef ARCHEAD_H_
 #define ARCHEAD_H_
@@ -54,7 +57,7 @@ enum archead_status {
   ARCHEAD_ERR_NULLPTR = -1,     /* a required pointer is NULL                         */
   ARCHEAD_ERR_ALIGN = -2,       /* a pointer is not 16-byte aligned                   */
   ARCHEAD_ERR_SHAPE = -3,       /* sizes disagree with the head or break a limit      */
-  ARCHEAD_ERR_RANGE_H = -4,     /* an entry of H is outside the FP16 range / not finite */
+  ARCHEAD_ERR_RANGE_H = -4,     /* H not finite, or a scaled rank product beyond FP16  */
   ARCHEAD_ERR_TARGET = -5,      /* a target id is outside [0, V)                      */
   ARCHEAD_ERR_TIMEOUT = -6,     /* a bounded device wait gave up                      */
   ARCHEAD_ERR_CUDA = -7,        /* a CUDA runtime call or launch failed               */

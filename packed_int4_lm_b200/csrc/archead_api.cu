@@ -202,6 +202,7 @@ int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* ta
   // tcgen05: the B image holds H and the rank blocks; warp MMAs: FP16 H plus FP32 t
   const size_t o_hh = cv.take((size_t)Npad * (s.D + (use_tc ? 128 * plan.nrb : 0)) * 2);
   const size_t o_t = cv.take(use_tc ? 0 : (size_t)s.N * RR * 4);
+  const size_t o_tsc = cv.take((size_t)s.N * 4);  // token scales 2^e_n
   const size_t o_part = nll_mode ? cv.take((size_t)s.N * nvblk * 8) : 0;
   const size_t o_tl = nll_mode ? cv.take((size_t)s.N * 4) : 0;
   // a single token tile is split evenly over the CTAs (partials + per-tile counters)
@@ -219,6 +220,7 @@ int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* ta
   float* scr = split_bytes ? reinterpret_cast<float*>(b + o_scr) : nullptr;
   unsigned* cnt = split_bytes ? reinterpret_cast<unsigned*>(b + o_cnt) : nullptr;
   float* t = reinterpret_cast<float*>(b + o_t);
+  float* tsc = reinterpret_cast<float*>(b + o_tsc);
   int32_t* tloc = shard ? reinterpret_cast<int32_t*>(b + o_tloc) : nullptr;
   cudaError_t e = cudaSuccess;
   if (shard)  // shard-local targets and zeroed target logits, before the prologue
@@ -226,14 +228,14 @@ int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* ta
                               reinterpret_cast<float*>(b + o_tl), ds->err, st, &launches);
   const int32_t* tg = shard ? tloc : targets;
   if (e == cudaSuccess)
-    e = use_tc ? launch_prologue_blocked(H, head, s, plan, Hh, cnt, ds->err, st, &launches)
-               : launch_prologue(H, head, s, Npad, Hh, t, ds->err, st, &launches);
+    e = use_tc ? launch_prologue_blocked(H, head, s, plan, Hh, tsc, cnt, ds->err, st, &launches)
+               : launch_prologue(H, head, s, Npad, Hh, t, tsc, ds->err, st, &launches);
   if (e == cudaSuccess) {
     if (use_tc) {
       float2* part = nll_mode ? reinterpret_cast<float2*>(b + o_part) : nullptr;
       float* tl = nll_mode ? reinterpret_cast<float*>(b + o_tl) : nullptr;
       prof_mark(0, st);
-      e = launch_residual_tc(Hh, head, s, plan, nll_mode ? nullptr : Y, tg, part, tl, scr, cnt,
+      e = launch_residual_tc(Hh, tsc, head, s, plan, nll_mode ? nullptr : Y, tg, part, tl, scr, cnt,
                              ds->err, st, &launches);
       prof_mark(1, st);
       if (e == cudaSuccess && nll_mode)
@@ -241,13 +243,13 @@ int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* ta
                   : launch_nll_combine(part, tl, targets, s, nll, ds->err, st, &launches);
     } else if (!nll_mode) {
       prof_mark(0, st);
-      e = launch_residual_gemm(Hh, t, head, s, Y, nullptr, nullptr, nullptr, st, &launches, 0);
+      e = launch_residual_gemm(Hh, t, tsc, head, s, Y, nullptr, nullptr, nullptr, st, &launches, 0);
       prof_mark(1, st);
     } else {
       float2* part = reinterpret_cast<float2*>(b + o_part);
       float* tl = reinterpret_cast<float*>(b + o_tl);
       prof_mark(0, st);
-      e = launch_residual_gemm(Hh, t, head, s, nullptr, tg, part, tl, st, &launches, 1);
+      e = launch_residual_gemm(Hh, t, tsc, head, s, nullptr, tg, part, tl, st, &launches, 1);
       prof_mark(1, st);
       if (e == cudaSuccess)
         e = shard ? launch_nll_partials(part, tl, s, shard->partials, st, &launches)
@@ -291,7 +293,7 @@ const char* archead_strerror(int status) {
     case ARCHEAD_ERR_NULLPTR: return "a required pointer is NULL";
     case ARCHEAD_ERR_ALIGN: return "a pointer is not suitably aligned (16 bytes)";
     case ARCHEAD_ERR_SHAPE: return "sizes disagree with the head or break a limit";
-    case ARCHEAD_ERR_RANGE_H: return "an entry of H is outside the FP16 range or not finite";
+    case ARCHEAD_ERR_RANGE_H: return "an entry of H is not finite, or a scaled rank product exceeds the FP16 range";
     case ARCHEAD_ERR_TARGET: return "a target id is outside [0, V)";
     case ARCHEAD_ERR_TIMEOUT: return "a bounded device wait gave up";
     case ARCHEAD_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
@@ -389,6 +391,7 @@ int archead_agreement(const uint16_t* H, const archead_head* head, const float* 
   Carve cv;
   const size_t o_hh = cv.take((size_t)Npad * D * 2);
   const size_t o_t = cv.take((size_t)N * (r_c + r_r) * 4);
+  const size_t o_tsc = cv.take((size_t)N * 4);
   const size_t o_st = cv.take((size_t)N * nvblk * 6 * 4);
   const size_t o_kv = cv.take((size_t)N * nvblk * k * 4);
   const size_t o_ki = cv.take((size_t)N * nvblk * k * 4);
@@ -401,9 +404,10 @@ int archead_agreement(const uint16_t* H, const archead_head* head, const float* 
   int launches = 0;
   __half* Hh = reinterpret_cast<__half*>(b + o_hh);
   float* t = reinterpret_cast<float*>(b + o_t);
-  cudaError_t e = launch_prologue(H, head, s, Npad, Hh, t, ds->err, st, &launches);
+  float* tsc = reinterpret_cast<float*>(b + o_tsc);
+  cudaError_t e = launch_prologue(H, head, s, Npad, Hh, t, tsc, ds->err, st, &launches);
   if (e == cudaSuccess)
-    e = launch_agreement(Hh, t, head, s, Y_dense, k, reinterpret_cast<float*>(b + o_st),
+    e = launch_agreement(Hh, t, tsc, head, s, Y_dense, k, reinterpret_cast<float*>(b + o_st),
                          reinterpret_cast<float*>(b + o_kv), reinterpret_cast<int*>(b + o_ki),
                          topk_out, top1_dense_out, kl_out, lse_out, st, &launches);
   cudaFreeAsync(base, st);

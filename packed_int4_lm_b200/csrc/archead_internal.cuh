@@ -99,6 +99,31 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
 }
 
+// Token scaling.  H enters as BF16, whose range far exceeds FP16's; the kernels take FP16
+// operands.  Token n is therefore scaled by 2^-e_n with e_n = max(0, ilogb(m_n) - 14),
+// m_n = max_d |h[n, d]| (0 for a zero or non-finite m_n), so every entry of the scaled row
+// is below 2^15 in magnitude; scaling by a power of two is exact.  The rank products t of
+// the token are scaled the same way, the logits come out scaled by 2^-e_n, and each
+// epilogue multiplies them by 2^e_n (tsc[n]).  Every kernel that needs e_n computes it from
+// the same row maximum, so they agree bit for bit.
+__device__ __forceinline__ int token_shift(float m) {
+  if (!(m <= 3.402823466e38f) || m == 0.f) return 0;  // zero, infinite or NaN
+  const int e = ilogbf(m) - 14;
+  return e > 0 ? e : 0;
+}
+
+// The largest |h| of eight BF16 values (a 16-byte chunk of a row).
+__device__ __forceinline__ float bf16x8_absmax(uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  float m = 0.f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    m = fmaxf(m, fabsf(__uint_as_float(w[k] << 16)));
+    m = fmaxf(m, fabsf(__uint_as_float(w[k] & 0xFFFF0000u)));
+  }
+  return m;
+}
+
 __device__ __forceinline__ uint2 ldg_stream8(const void* p) {
   uint2 r;
   asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];\n"
@@ -124,12 +149,13 @@ struct Shapes {
   int r_c, r_r, g;
 };
 
-// Prologue: Hh = fp16(H) padded with zero rows to Npad, t = H [Q8(B_c) | Q8(B_w)]^T.
+// Prologue: Hh = fp16(H 2^-e_n) padded with zero rows to Npad, t = (H [Q8(B_c) |
+// Q8(B_w)]^T) 2^-e_n, tsc[n] = 2^e_n (token scaling, see token_shift).
 cudaError_t launch_prologue(const uint16_t* H, const archead_head* head, const Shapes& s,
-                            int64_t Npad, __half* Hh, float* t, unsigned* err,
+                            int64_t Npad, __half* Hh, float* t, float* tsc, unsigned* err,
                             cudaStream_t st, int* launches);
 
-// t = H [Q8(B_c) | Q8(B_w)]^T (N x (r_c + r_r) FP32).  With img != nullptr the products
+// t = (H [Q8(B_c) | Q8(B_w)]^T) 2^-e_n (N x (r_c + r_r) FP32).  With img != nullptr the products
 // go instead, split into FP16 pieces, into the rank blocks of the tcgen05 B image (token
 // tile nt, nkbt blocks per tile); a piece outside the FP16 range sets kErrRangeH.
 cudaError_t launch_lowrank_t(const uint16_t* H, const archead_head* head, const Shapes& s,
@@ -162,7 +188,7 @@ __host__ __device__ __forceinline__ int64_t tc_image_offset(int64_t tt, int64_t 
 // counters: the per-tile counters of a split launch (ceil(V/128) words, zeroed here), or
 // nullptr.
 cudaError_t launch_prologue_blocked(const uint16_t* H, const archead_head* head,
-                                    const Shapes& s, const TcPlan& plan, __half* Hb,
+                                    const Shapes& s, const TcPlan& plan, __half* Hb, float* tsc,
                                     unsigned* counters, unsigned* err, cudaStream_t st,
                                     int* launches);
 // Bytes of scratch for a launch whose single token tile is split evenly over the CTAs
@@ -172,8 +198,9 @@ size_t tc_split_scratch_bytes(const Shapes& s, const TcPlan& plan);
 // into part[N x ceil(V/128)] and target logits into tlogit[N] (see launch_nll_combine).
 // scratch / counters (tc_split_scratch_bytes, launch_prologue_blocked): the split of a
 // single token tile over the CTAs, or nullptr for whole tiles per CTA.
-cudaError_t launch_residual_tc(const __half* Hb, const archead_head* head, const Shapes& s,
-                               const TcPlan& plan, float* Y, const int32_t* targets,
+cudaError_t launch_residual_tc(const __half* Hb, const float* tsc, const archead_head* head,
+                               const Shapes& s, const TcPlan& plan, float* Y,
+                               const int32_t* targets,
                                float2* part, float* tlogit, float* scratch, unsigned* counters,
                                unsigned* err, cudaStream_t st, int* launches);
 
@@ -187,7 +214,9 @@ struct DecPlan {
 DecPlan dec_plan(const Shapes& s, bool nll);
 size_t dec_image_bytes(const Shapes& s, const DecPlan& pl);  // resident H image
 size_t dec_partial_bytes(const DecPlan& pl);                 // split-tile partials
-// H image + zeroed per-tile counters (ceil(V/128) words), then t (N x RR FP32).
+// H image (tokens scaled by 2^-e_n, with the offset corrections and the token scales 2^e_n
+// after it) + zeroed per-tile counters (ceil(V/128) words), then t (N x RR FP32, unscaled:
+// the decode kernel divides by 2^e_n when it stages t).
 cudaError_t launch_dec_prologue(const uint16_t* H, const archead_head* head, const Shapes& s,
                                 const DecPlan& pl, __half* img, float* t, unsigned* counters,
                                 unsigned* err, cudaStream_t st, int* launches);
@@ -208,7 +237,8 @@ void set_dec_test_hooks(long long wait_limit, int stall_cta);
 // Residual dequant-contraction over token blocks of up to 64 (mma.sync path).
 // mode 0: write logits Y.  mode 1: write NLL partials (max, sum exp) per (token, vocabulary
 // block) into part[N x residual_gemm_vblocks] and the target logit into tlogit[N].
-cudaError_t launch_residual_gemm(const __half* Hh, const float* t, const archead_head* head,
+cudaError_t launch_residual_gemm(const __half* Hh, const float* t, const float* tsc,
+                                 const archead_head* head,
                                  const Shapes& s, float* Y, const int32_t* targets,
                                  float2* part, float* tlogit, cudaStream_t st, int* launches,
                                  int mode);
@@ -217,7 +247,8 @@ int residual_gemm_vblocks(const Shapes& s);
 // per token the ids of the topk largest packed logits, the dense argmax, KL(dense ||
 // packed) and the packed log-sum-exp.  Scratch: astat N x nvblk x 6 floats, akval and akid
 // N x nvblk x topk each (nvblk = residual_gemm_vblocks).
-cudaError_t launch_agreement(const __half* Hh, const float* t, const archead_head* head,
+cudaError_t launch_agreement(const __half* Hh, const float* t, const float* tsc,
+                             const archead_head* head,
                              const Shapes& s, const float* Yd, int topk, float* astat,
                              float* akval, int* akid, int32_t* topk_out, int32_t* top1_dense,
                              float* kl_out, float* lse_out, cudaStream_t st, int* launches);

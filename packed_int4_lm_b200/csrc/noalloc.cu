@@ -78,15 +78,17 @@ extern "C" int archead_logits_noalloc(const uint16_t* H, const archead_head* hea
   if (D > cap / 2 || Npad > cap / 2 / D || N > cap / 4 / (r_c + r_r + 1))
     return ARCHEAD_ERR_SHAPE;
   const size_t hh_bytes = round256((size_t)Npad * D * 2);
-  const size_t t_bytes = round256((size_t)N * (r_c + r_r) * 4 + 16);
+  const size_t t_bytes = round256((size_t)N * (r_c + r_r + 1) * 4 + 16);  // t, token scales
   if (hh_bytes + t_bytes > kScratchBytes) return ARCHEAD_ERR_SHAPE;
   NoAllocDevice* d = nullptr;
   rc = device_setup(&d);
   if (rc) return rc;
   // Every scratch byte a kernel reads is written earlier in the same call (the FP16 copy
-  // of H including its zero padding rows, then t), so nothing needs clearing between calls.
+  // of H including its zero padding rows, then t and the token scales), so nothing needs
+  // clearing between calls.
   __half* Hh = reinterpret_cast<__half*>(d->scratch);
   float* t = reinterpret_cast<float*>(d->scratch + hh_bytes);
+  float* tsc = t + N * (r_c + r_r);
   Shapes s;
   s.N = N;
   s.V = V;
@@ -96,8 +98,8 @@ extern "C" int archead_logits_noalloc(const uint16_t* H, const archead_head* hea
   s.g = g;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int launches = 0;
-  cudaError_t e = launch_prologue(H, head, s, Npad, Hh, t, d->err, st, &launches);
+  cudaError_t e = launch_prologue(H, head, s, Npad, Hh, t, tsc, d->err, st, &launches);
   if (e == cudaSuccess)
-    e = launch_residual_gemm(Hh, t, head, s, Y, nullptr, nullptr, nullptr, st, &launches, 0);
+    e = launch_residual_gemm(Hh, t, tsc, head, s, Y, nullptr, nullptr, nullptr, st, &launches, 0);
   return e == cudaSuccess ? ARCHEAD_OK : ARCHEAD_ERR_CUDA;
 }

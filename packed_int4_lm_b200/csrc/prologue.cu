@@ -1,46 +1,73 @@
 // Prologue of the ARCHead logit path (ARCHead Sec. 3, the bracket (H B_w^T) of the logit
 // formula, and its core analogue H B_c^T):
-//   * Hh = fp16(H), zero-padded to Npad rows -- the B operand of the residual contraction;
-//   * t  = H [Q8(B_c) | Q8(B_w)]^T, N x (r_c + r_r) FP32 -- the rank terms' left products
-//     (for the tcgen05 path, split into FP16 pieces inside the MMA's B image instead).
+//   * Hh = fp16(H 2^-e_n), zero-padded to Npad rows -- the B operand of the residual
+//     contraction, each token scaled by its power of two (token_shift);
+//   * t  = (H [Q8(B_c) | Q8(B_w)]^T) 2^-e_n, N x (r_c + r_r) FP32 -- the rank terms' left
+//     products (for the tcgen05 path, split into FP16 pieces inside the MMA's B image);
+//   * tsc[n] = 2^e_n, by which the epilogues multiply token n's logits.
 #include "tc_common.cuh"
 
 namespace archead {
 namespace {
 
-// One thread converts 8 consecutive BF16 values.  Rows n >= N are written as zeros.
+// Block-wide maximum of v (blockDim.x a multiple of 32, at most 1024); every thread gets it.
+__device__ __forceinline__ float block_max(float v, float* red32) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __syncthreads();  // red32 may still be read from the previous use
+  if (lane == 0) red32[warp] = v;
+  __syncthreads();
+  v = 0.f;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) v = fmaxf(v, red32[w]);
+  return v;
+}
+
+// One block per token row (grid-stride over rows): the row's largest |h| gives its scale
+// 2^-e_n, then each thread converts 8 consecutive BF16 values at a time.  Rows n >= N are
+// written as zeros.  Non-finite entries set kErrRangeH.
 __global__ void __launch_bounds__(256) convert_h_kernel(const uint16_t* __restrict__ H,
-                                                        __half* __restrict__ Hh, int64_t N,
+                                                        __half* __restrict__ Hh,
+                                                        float* __restrict__ tsc, int64_t N,
                                                         int64_t Npad, int64_t D,
                                                         unsigned* err) {
-  const int64_t total = Npad * D / 8;
-  const int64_t valid = N * D / 8;
+  __shared__ float red32[8];
+  const int64_t chunks = D / 8;
   bool bad = false;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    uint4 out = make_uint4(0, 0, 0, 0);
-    if (i < valid) {
-      uint4 in = *reinterpret_cast<const uint4*>(H + i * 8);
-      uint32_t w[4] = {in.x, in.y, in.z, in.w};
-      uint32_t o[4];
+  for (int64_t n = blockIdx.x; n < Npad; n += gridDim.x) {
+    float m = 0.f;
+    if (n < N)
+      for (int64_t c = threadIdx.x; c < chunks; c += blockDim.x)
+        m = fmaxf(m, bf16x8_absmax(__ldg(reinterpret_cast<const uint4*>(H + n * D + c * 8))));
+    const int e = token_shift(block_max(m, red32));
+    const float sc = ldexpf(1.f, -e);
+    if (n < N && threadIdx.x == 0) tsc[n] = ldexpf(1.f, e);
+    for (int64_t c = threadIdx.x; c < chunks; c += blockDim.x) {
+      uint4 out = make_uint4(0, 0, 0, 0);
+      if (n < N) {
+        const uint4 in = __ldg(reinterpret_cast<const uint4*>(H + n * D + c * 8));
+        const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+        uint32_t o[4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        float lo = __uint_as_float(w[k] << 16);
-        float hi = __uint_as_float(w[k] & 0xFFFF0000u);
-        __half2 h = __floats2half2_rn(lo, hi);
-        o[k] = h2_bits(h);
-        // exponent field all ones: infinite or NaN after rounding to FP16
-        bad |= ((o[k] & 0x7C00u) == 0x7C00u) | ((o[k] & 0x7C000000u) == 0x7C000000u);
+        for (int k = 0; k < 4; ++k) {
+          const float lo = __uint_as_float(w[k] << 16) * sc;
+          const float hi = __uint_as_float(w[k] & 0xFFFF0000u) * sc;
+          o[k] = h2_bits(__floats2half2_rn(lo, hi));
+          // exponent field all ones: infinite or NaN
+          bad |= ((o[k] & 0x7C00u) == 0x7C00u) | ((o[k] & 0x7C000000u) == 0x7C000000u);
+        }
+        out = make_uint4(o[0], o[1], o[2], o[3]);
       }
-      out = make_uint4(o[0], o[1], o[2], o[3]);
+      *reinterpret_cast<uint4*>(Hh + n * D + c * 8) = out;
     }
-    *reinterpret_cast<uint4*>(Hh + i * 8) = out;
   }
   if (bad) atomicOr(err, kErrRangeH);
 }
 
-// t[n, j] = sum_d h[n, d] * fl32(B[j, d] * sB[j, d / g]) with j < r_c from B_c and the
-// rest from B_w.  Block (token group of kTN, j); 256 threads stride over D, 8 columns each.
+// t[n, j] = 2^-e_n sum_d h[n, d] * fl32(B[j, d] * sB[j, d / g]) with j < r_c from B_c and
+// the rest from B_w.  Block (token group of kTN, j); 256 threads stride over D, 8 columns
+// each.  The block sees the whole rows of its tokens, so it finds each token's e_n itself
+// (token_shift of the same row maximum as the conversion kernels).
 constexpr int kTN = 8;
 
 __global__ void __launch_bounds__(256) lowrank_t_kernel(
@@ -63,9 +90,9 @@ __global__ void __launch_bounds__(256) lowrank_t_kernel(
   const int64_t G = D / g;
   const int64_t n0 = (int64_t)blockIdx.x * kTN;
   const int nv = (N - n0) < kTN ? (int)(N - n0) : kTN;
-  float acc[kTN];
+  float acc[kTN], mx[kTN];
 #pragma unroll
-  for (int n = 0; n < kTN; ++n) acc[n] = 0.f;
+  for (int n = 0; n < kTN; ++n) acc[n] = mx[n] = 0.f;
 
   for (int64_t d0 = threadIdx.x * 8; d0 < D; d0 += 256 * 8) {
     uint2 braw = *reinterpret_cast<const uint2*>(B + jj * D + d0);
@@ -82,6 +109,7 @@ __global__ void __launch_bounds__(256) lowrank_t_kernel(
       hv[n] = __ldg(reinterpret_cast<const uint4*>(H + (n0 + (n < nv ? n : nv - 1)) * D + d0));
 #pragma unroll
     for (int n = 0; n < kTN; ++n) {
+      mx[n] = fmaxf(mx[n], bf16x8_absmax(hv[n]));
       const uint32_t hw[4] = {hv[n].x, hv[n].y, hv[n].z, hv[n].w};
       float a = acc[n];
 #pragma unroll
@@ -92,21 +120,31 @@ __global__ void __launch_bounds__(256) lowrank_t_kernel(
       acc[n] = a;
     }
   }
-  // block reduction of the kTN sums
-  __shared__ float red[8][kTN];
+  // block reduction of the kTN sums and row maxima
+  __shared__ float red[8][kTN], redm[8][kTN];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
   for (int n = 0; n < kTN; ++n) {
-    float v = acc[n];
+    float v = acc[n], m = mx[n];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0) red[warp][n] = v;
+    for (int o = 16; o > 0; o >>= 1) {
+      v += __shfl_xor_sync(0xffffffffu, v, o);
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    }
+    if (lane == 0) {
+      red[warp][n] = v;
+      redm[warp][n] = m;
+    }
   }
   __syncthreads();
   if (threadIdx.x < kTN && (int)threadIdx.x < nv) {
-    float v = 0.f;
+    float v = 0.f, m = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) v += red[w][threadIdx.x];
+    for (int w = 0; w < 8; ++w) {
+      v += red[w][threadIdx.x];
+      m = fmaxf(m, redm[w][threadIdx.x]);
+    }
+    v *= ldexpf(1.f, -token_shift(m));  // exact: a power of two
     const int64_t n = n0 + threadIdx.x;
     // the image's rank blocks were zero-filled by the previous kernel (this one may be a
     // programmatic dependent launch of it)
@@ -130,14 +168,12 @@ __global__ void __launch_bounds__(256) lowrank_t_kernel(
 }  // namespace
 
 cudaError_t launch_prologue(const uint16_t* H, const archead_head* head, const Shapes& s,
-                            int64_t Npad, __half* Hh, float* t, unsigned* err,
+                            int64_t Npad, __half* Hh, float* t, float* tsc, unsigned* err,
                             cudaStream_t st, int* launches) {
   {
-    const int64_t chunks = Npad * s.D / 8;
-    int64_t blocks = (chunks + 255) / 256;
-    if (blocks > 148 * 16) blocks = 148 * 16;
+    int64_t blocks = Npad < 148 * 16 ? Npad : 148 * 16;  // one block per row (grid-stride)
     if (blocks < 1) blocks = 1;
-    convert_h_kernel<<<(unsigned)blocks, 256, 0, st>>>(H, Hh, s.N, Npad, s.D, err);
+    convert_h_kernel<<<(unsigned)blocks, 256, 0, st>>>(H, Hh, tsc, s.N, Npad, s.D, err);
     ++*launches;
   }
   cudaError_t e = cudaGetLastError();

@@ -98,8 +98,8 @@ __host__ __device__ inline DecSmem dec_smem(int64_t D, int G, int r_c, int r_r, 
   constexpr int NTOK = DecCfg<NT8>::NTOK;
   DecSmem m;
   size_t o = 0;
-  m.h = o;  // H image [NTOK x D] FP16, then corr quads [D / 128][NTOK / 2] float4
-  o += dec_round16((size_t)NTOK * D * 2 + (size_t)(D / 128) * NTOK * 8);
+  m.h = o;  // H image [NTOK x D] FP16, corr quads [D / 128][NTOK / 2] float4, scales [NTOK]
+  o += dec_round16((size_t)NTOK * D * 2 + (size_t)(D / 128) * NTOK * 8 + (size_t)NTOK * 4);
   m.pk = o;  // ring of sp stages of two packed blocks
   o += (size_t)sp * 2 * kDecPk;
   m.codes = o;  // [2][128 x G]
@@ -154,7 +154,9 @@ __device__ __forceinline__ bool dec_wait(uint64_t* bar, uint32_t parity, unsigne
 // two).  Each k-block sum then carries the constant 1032 sum_A b + 1152 sum_B b over the
 // stored values b; corr holds its negation, from which the kernel's MMA chain of the block
 // starts, so the chain ends at the block's dot product.
-// Non-finite or out-of-range FP16 values set kErrRangeH.
+// Each token is scaled by 2^-e_n (token_shift of its row maximum, which every warp of the
+// token finds from the whole row: 16 KB per warp at most, from L2), and tsc[n] = 2^e_n
+// follows the corrections (1 for the zero rows).  Non-finite entries set kErrRangeH.
 // Runs on blocks blk of nblk.
 __device__ __forceinline__ void dec_convert_h(const uint16_t* __restrict__ H,
                                               __half* __restrict__ img, int64_t N, int ntok,
@@ -167,17 +169,38 @@ __device__ __forceinline__ void dec_convert_h(const uint16_t* __restrict__ H,
   const int64_t gw = (blk * (int64_t)blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = (nblk * (int64_t)blockDim.x) >> 5;
   float* corr = reinterpret_cast<float*>(img + (int64_t)ntok * D);  // [nkb][ntok / 2] quads
+  float* tsc = corr + nkb * ntok * 2;                                 // [ntok]
   bool bad = false;
   for (int64_t wi = gw; wi < (int64_t)ntok * nkb; wi += nw) {
     const int64_t n = wi / nkb, kb = wi - n * nkb;
     const int64_t d = kb * 128 + 4 * lane;
     float f[4] = {0.f, 0.f, 0.f, 0.f};
+    float sc = 1.f;
     if (n < N) {
       const uint2 in = *reinterpret_cast<const uint2*>(H + n * D + d);
       f[0] = __uint_as_float(in.x << 16);
       f[1] = __uint_as_float(in.x & 0xFFFF0000u);
       f[2] = __uint_as_float(in.y << 16);
       f[3] = __uint_as_float(in.y & 0xFFFF0000u);
+      float m = 0.f;  // the row maximum, sixteen 16-byte loads in flight per lane at a time
+      for (int64_t c0 = lane; c0 < D / 8; c0 += 16 * 32) {
+        uint4 v[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+          v[q] = c0 + 32 * q < D / 8 ? __ldg(reinterpret_cast<const uint4*>(H + n * D + (c0 + 32 * q) * 8))
+                                     : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) m = fmaxf(m, bf16x8_absmax(v[q]));
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      const int e = token_shift(m);
+      sc = ldexpf(1.f, -e);
+      if (kb == 0 && lane == 0) tsc[n] = ldexpf(1.f, e);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) f[k] *= sc;  // exact: a power of two
+    } else if (kb == 0 && lane == 0) {
+      tsc[n] = 1.f;
     }
     float sum = 0.f;
     __half hv[4];
@@ -186,7 +209,7 @@ __device__ __forceinline__ void dec_convert_h(const uint16_t* __restrict__ H,
       const bool typeb = ((d + e) & 2) != 0;
       hv[e] = __float2half_rn(scale_b && typeb ? f[e] * 0.0625f : f[e]);
       const float b = __half2float(hv[e]);
-      bad |= !(fabsf(b) <= 65504.f);
+      bad |= !(fabsf(b) <= 65504.f);  // only a non-finite h after the scaling
       sum += (typeb ? 1152.f : 1032.f) * b;
     }
     const uint32_t lo = (uint32_t)__half_as_ushort(hv[0]) | ((uint32_t)__half_as_ushort(hv[1]) << 16);
@@ -264,7 +287,7 @@ __device__ __forceinline__ void dec_lowrank_t(const uint16_t* __restrict__ H,
     float v = 0.f;
 #pragma unroll
     for (int w = 0; w < kDecPrologueThreads / 32; ++w) v += red[w][threadIdx.x];
-    t[(int64_t)threadIdx.x * RR + j] = v;
+    t[(int64_t)threadIdx.x * RR + j] = v;  // unscaled: the decode kernel applies 2^-e_n
   }
 }
 
@@ -431,7 +454,7 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
     if (lane == 0) {
       bool ok = true;
       const uint64_t pol_first = tc::l2_policy_evict_first();  // the head streams once
-      const uint32_t hbytes = (uint32_t)(NTOK * D * 2 + (int64_t)nkb * NTOK * 8);
+      const uint32_t hbytes = (uint32_t)(NTOK * D * 2 + (int64_t)nkb * NTOK * 8 + NTOK * 4);
       // The H image comes from the prologue kernel, which may still be running (this
       // kernel is a programmatic dependent launch): the packed stream starts at once, and
       // the image is fetched after the prologue grid completes, before the first wait that
@@ -507,9 +530,12 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
   // wait gives up, sets the device error word, and the warp skips its remaining waits
   if ((int)blockIdx.x == p.stall_cta && warp == 0) ok = dec_wait(dead, 0, p.err, ok, p.wait_limit);
 #endif
+  const float* tsc_s =
+      reinterpret_cast<const float*>(smem + m.h + (size_t)NTOK * D * 2 + (size_t)nkb * NTOK * 8);
   for (int i = ctid; i < NTOK * RR; i += CONSUMERS * 32) {  // ts[j * NTOK + n]
     const int j = i / NTOK, n = i - j * NTOK;
-    const float tv = n < p.N ? __ldg(p.t + (int64_t)n * RR + j) : 0.f;
+    // t of the scaled token: t 2^-e_n (the token scales follow the image's corrections)
+    const float tv = n < p.N ? __ldg(p.t + (int64_t)n * RR + j) / tsc_s[n] : 0.f;
     ts[i] = tv;
     // FP16 pieces: t1 + t2 carries 22 significant bits of t
     const __half t1 = __float2half_rn(tv);
@@ -798,6 +824,16 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
           }
         }
       }
+      // the logits of the scaled tokens (8 j + 2 tq + e): times 2^e_n
+#pragma unroll
+      for (int j = 0; j < NT8; ++j) {
+        const float2 tk = *reinterpret_cast<const float2*>(
+            smem + m.h + (size_t)NTOK * D * 2 + (size_t)nkb * NTOK * 8 + (8 * j + 2 * tq) * 4);
+        y[j][0] *= tk.x;
+        y[j][1] *= tk.y;
+        y[j][2] *= tk.x;
+        y[j][3] *= tk.y;
+      }
       if (MODE == 0) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -929,7 +965,7 @@ DecPlan dec_plan(const Shapes& s, bool nll) {
 }
 
 size_t dec_image_bytes(const Shapes& s, const DecPlan& pl) {
-  return (size_t)8 * pl.nt8 * s.D * 2 + (size_t)(s.D / 128) * 8 * pl.nt8 * 8;
+  return (size_t)8 * pl.nt8 * s.D * 2 + (size_t)(s.D / 128) * 8 * pl.nt8 * 8 + (size_t)8 * pl.nt8 * 4;
 }
 size_t dec_partial_bytes(const DecPlan& pl) { return (size_t)pl.grid * 2 * 256 * pl.nt8 * 16; }
 

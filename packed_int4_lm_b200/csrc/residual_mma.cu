@@ -32,8 +32,9 @@ constexpr int kKC = 128;     // columns per pipeline chunk (one 64-byte block of
 constexpr int kStages = 3;   // cp.async ring depth for the hidden-state chunks
 
 struct GemmParams {
-  const __half* Hh;  // Npad x D
-  const float* t;    // N x RR
+  const __half* Hh;  // Npad x D (token n scaled by 2^-e_n)
+  const float* t;    // N x RR (scaled the same way)
+  const float* tsc;  // N token scales 2^e_n
   const uint8_t* nib;        // SC4: tiled nibbles; Row INT8 (CPC = 0): V x D int8 row-major
   const float* row_scale;    // Row INT8: W[v, d] = q8[v, d] * row_scale[v]
   const uint8_t* code;
@@ -281,6 +282,8 @@ __global__ void __launch_bounds__(WARPS * 32)
     int64_t tok = tok0 + n;
     ts[n * TS + j] = tok < p.N ? p.t[tok * RR + j] : 0.f;
   }
+  for (int n = threadIdx.x; n < C::NTOK; n += C::THREADS)  // column RR: the token scale
+    ts[n * TS + RR] = tok0 + n < p.N ? p.tsc[tok0 + n] : 1.f;
   __syncthreads();
 
   float y[R][NT][4];
@@ -319,6 +322,11 @@ __global__ void __launch_bounds__(WARPS * 32)
 #pragma unroll
           for (int e = 0; e < 2; ++e) y[r][j][2 * h + e] = fmaf(sa, lr[j][e], y[r][j][2 * h + e]);
       }
+      // the logits of the scaled tokens: times 2^e_n
+#pragma unroll
+      for (int j = 0; j < NT; ++j)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) y[r][j][2 * h + e] *= ts[(8 * j + 2 * tq + e) * TS + RR];
     }
   }
 
@@ -597,13 +605,15 @@ int64_t residual_token_block(int64_t N) {
 
 int residual_gemm_vblocks(const Shapes& s) { return (int)((s.V + kRows - 1) / kRows); }
 
-cudaError_t launch_residual_gemm(const __half* Hh, const float* t, const archead_head* head,
+cudaError_t launch_residual_gemm(const __half* Hh, const float* t, const float* tsc,
+                                 const archead_head* head,
                                  const Shapes& s, float* Y, const int32_t* targets,
                                  float2* part, float* tlogit, cudaStream_t st, int* launches,
                                  int mode) {
   GemmParams p;
   p.Hh = Hh;
   p.t = t;
+  p.tsc = tsc;
   p.nib = head->r_nib;
   p.row_scale = head->format == ARCHEAD_FMT_ROW8 ? head->row_scale : nullptr;
   p.code = head->r_code;
@@ -731,13 +741,15 @@ __global__ void __launch_bounds__(256) agreement_merge_kernel(
   }
 }
 
-cudaError_t launch_agreement(const __half* Hh, const float* t, const archead_head* head,
+cudaError_t launch_agreement(const __half* Hh, const float* t, const float* tsc,
+                             const archead_head* head,
                              const Shapes& s, const float* Yd, int topk, float* astat,
                              float* akval, int* akid, int32_t* topk_out, int32_t* top1_dense,
                              float* kl_out, float* lse_out, cudaStream_t st, int* launches) {
   GemmParams p;
   p.Hh = Hh;
   p.t = t;
+  p.tsc = tsc;
   p.nib = head->r_nib;
   p.row_scale = head->format == ARCHEAD_FMT_ROW8 ? head->row_scale : nullptr;
   p.code = head->r_code;

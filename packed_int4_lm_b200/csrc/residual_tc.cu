@@ -52,6 +52,7 @@ constexpr int kMaxSP = 8;        // deepest packed ring
 
 struct TcParams {
   const __half* Hb;  // B image: [token tile][nkb + nrb blocks][NT x 128]
+  const float* tsc;  // N token scales 2^e_n (the image holds H 2^-e_n)
   const uint8_t* nib;
   const uint8_t* code;  // Vpad x G
   const uint16_t* sup;
@@ -117,7 +118,7 @@ template <int NT>
 size_t tc_smem_bytes(int sb, int sp, int G, bool nll) {
   using C = TcCfg<NT>;
   return (size_t)sb * C::HSTAGE + (size_t)sp * kPkBytes + 2 * round16((size_t)128 * G) +
-         (nll ? nll_scratch_bytes<NT>() : 0) + 512;
+         (nll ? nll_scratch_bytes<NT>() : 0) + (size_t)NT * 4 + 512;
 }
 
 // The k-th work item of this CTA: its tile's first row, its row limit, its token tile.
@@ -254,8 +255,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
   unsigned char* after_codes = cds + 2 * round16(code_bytes);
   float* nll_y = reinterpret_cast<float*>(after_codes);  // [16][128]
   int32_t* tgt_s = reinterpret_cast<int32_t*>(nll_y + 16 * 128);  // [NT]
-  uint64_t* bars =
-      reinterpret_cast<uint64_t*>(after_codes + (MODE ? nll_scratch_bytes<NT>() : 0));
+  float* tsc_s = reinterpret_cast<float*>(after_codes + (MODE ? nll_scratch_bytes<NT>() : 0));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(tsc_s + NT);  // tsc_s: [NT] token scales
   uint64_t* b_full = bars;
   uint64_t* b_empty = b_full + kMaxSB;
   uint64_t* p_full = b_empty + kMaxSB;
@@ -622,10 +623,12 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
     for (int i = 0; get_item(p, i, it); ++i) {
       const int ab = i % C::NACC, use = i / C::NACC;
       const int64_t tok0 = (int64_t)it.tt * NT;
-      if (MODE == 1 && it.tt != cur_tt) {  // the token tile's targets
+      if (it.tt != cur_tt) {  // the token tile's scales (and targets)
         asm volatile("bar.sync 1, 128;\n" ::: "memory");
-        for (int q = e; q < NT; q += 128)
-          tgt_s[q] = tok0 + q < p.N ? __ldg(p.targets + tok0 + q) : -1;
+        if (e < NT) {
+          if (MODE == 1) tgt_s[e] = tok0 + e < p.N ? __ldg(p.targets + tok0 + e) : -1;
+          tsc_s[e] = tok0 + e < p.N ? __ldg(p.tsc + tok0 + e) : 1.f;
+        }
         asm volatile("bar.sync 1, 128;\n" ::: "memory");
         cur_tt = it.tt;
       }
@@ -704,8 +707,15 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
         for (int c = 0; c < HC / 16; ++c) {
           const int c16 = h * (HC / 16) + c;  // 16-token chunk of the tile
           float y[16];
+          const float4* ts4 = reinterpret_cast<const float4*>(tsc_s + 16 * c16);
 #pragma unroll
-          for (int q = 0; q < 16; ++q) y[q] = __uint_as_float(r[c][q]) * sp;
+          for (int q4 = 0; q4 < 4; ++q4) {  // the logit of token q: accumulator x S'_v x 2^e_q
+            const float4 f = ts4[q4];
+            y[4 * q4 + 0] = __uint_as_float(r[c][4 * q4 + 0]) * sp * f.x;
+            y[4 * q4 + 1] = __uint_as_float(r[c][4 * q4 + 1]) * sp * f.y;
+            y[4 * q4 + 2] = __uint_as_float(r[c][4 * q4 + 2]) * sp * f.z;
+            y[4 * q4 + 3] = __uint_as_float(r[c][4 * q4 + 3]) * sp * f.w;
+          }
           if (MODE == 0) {
             if (live) {
               // token rows of the chunk below N, one pointer stepped by a row of Y
@@ -764,13 +774,15 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
   }
 }
 
-// The B image of the residual blocks: FP16 copy of H, for token tile tt of nt rows and
-// 128-column block kb a contiguous nt x 128 block at tc_image_offset (K-major, 128-byte
-// swizzle).  Rows >= N are zero, and so are the nrb rank blocks after the nkb blocks of H,
-// which the low-rank prologue then fills.  Non-finite or out-of-range FP16 values set
-// kErrRangeH.
+// The B image of the residual blocks: FP16 copy of H 2^-e_n (token scaling, see
+// token_shift), for token tile tt of nt rows and 128-column block kb a contiguous nt x 128
+// block at tc_image_offset (K-major, 128-byte swizzle).  Rows >= N are zero, and so are
+// the nrb rank blocks after the nkb blocks of H, which the low-rank prologue then fills.
+// One block per token row (grid-stride over rows): the row maximum first, then the
+// conversion; tsc[n] = 2^e_n.  Non-finite entries set kErrRangeH.
 __global__ void __launch_bounds__(256) convert_h_blocked_kernel(const uint16_t* __restrict__ H,
                                                                 __half* __restrict__ Hb,
+                                                                float* __restrict__ tsc,
                                                                 int64_t N, int64_t Npad,
                                                                 int64_t D, int64_t nkbt, int nt,
                                                                 unsigned* counters, int64_t ncnt,
@@ -779,31 +791,45 @@ __global__ void __launch_bounds__(256) convert_h_blocked_kernel(const uint16_t* 
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < ncnt;
        i += (int64_t)gridDim.x * blockDim.x)
     counters[i] = 0u;
+  __shared__ float red32[8];
   const int64_t chunks_per_row = nkbt * 16;  // 8 FP16 per chunk
-  const int64_t total = Npad * chunks_per_row;
   const int64_t hchunks = D / 8;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   bool bad = false;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t n = i / chunks_per_row;
-    const int64_t kc = i - n * chunks_per_row;
-    uint4 out = make_uint4(0, 0, 0, 0);
-    if (n < N && kc < hchunks) {
-      const uint4 in = *reinterpret_cast<const uint4*>(H + n * D + kc * 8);
-      const uint32_t w[4] = {in.x, in.y, in.z, in.w};
-      uint32_t o[4];
+  for (int64_t n = blockIdx.x; n < Npad; n += gridDim.x) {
+    float m = 0.f;
+    if (n < N)
+      for (int64_t kc = threadIdx.x; kc < hchunks; kc += blockDim.x)
+        m = fmaxf(m, bf16x8_absmax(__ldg(reinterpret_cast<const uint4*>(H + n * D + kc * 8))));
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const __half2 h = __floats2half2_rn(__uint_as_float(w[k] << 16),
-                                            __uint_as_float(w[k] & 0xFFFF0000u));
-        o[k] = h2_bits(h);
-        bad |= ((o[k] & 0x7C00u) == 0x7C00u) | ((o[k] & 0x7C000000u) == 0x7C000000u);
-      }
-      out = make_uint4(o[0], o[1], o[2], o[3]);
-    }
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    __syncthreads();  // red32 of the previous row has been read
+    if (lane == 0) red32[warp] = m;
+    __syncthreads();
+    m = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, red32[w]);
+    const int e = token_shift(m);
+    const float sc = ldexpf(1.f, -e);
+    if (n < N && threadIdx.x == 0) tsc[n] = ldexpf(1.f, e);
     const int64_t tt = n / nt, nn = n - tt * nt;
-    *reinterpret_cast<uint4*>(Hb + tc_image_offset(tt, kc >> 4, nkbt, nt, nn,
-                                                   (int)(kc & 15) * 8)) = out;
+    for (int64_t kc = threadIdx.x; kc < chunks_per_row; kc += blockDim.x) {
+      uint4 out = make_uint4(0, 0, 0, 0);
+      if (n < N && kc < hchunks) {
+        const uint4 in = __ldg(reinterpret_cast<const uint4*>(H + n * D + kc * 8));
+        const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const __half2 h = __floats2half2_rn(__uint_as_float(w[k] << 16) * sc,
+                                              __uint_as_float(w[k] & 0xFFFF0000u) * sc);
+          o[k] = h2_bits(h);
+          bad |= ((o[k] & 0x7C00u) == 0x7C00u) | ((o[k] & 0x7C000000u) == 0x7C000000u);
+        }
+        out = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+      *reinterpret_cast<uint4*>(Hb + tc_image_offset(tt, kc >> 4, nkbt, nt, nn,
+                                                     (int)(kc & 15) * 8)) = out;
+    }
   }
   if (bad) atomicOr(err, kErrRangeH);
 }
@@ -908,28 +934,29 @@ size_t tc_split_scratch_bytes(const Shapes& s, const TcPlan& plan) {
 }
 
 cudaError_t launch_prologue_blocked(const uint16_t* H, const archead_head* head,
-                                    const Shapes& s, const TcPlan& plan, __half* Hb,
+                                    const Shapes& s, const TcPlan& plan, __half* Hb, float* tsc,
                                     unsigned* counters, unsigned* err, cudaStream_t st,
                                     int* launches) {
   const int nt = plan.nt;
   const int64_t Npad = (s.N + nt - 1) / nt * nt;
   const int64_t nkbt = s.D / 128 + plan.nrb;
-  int64_t blocks = (Npad * nkbt * 16 + 255) / 256;
-  if (blocks > 148 * 16) blocks = 148 * 16;
+  int64_t blocks = Npad < 148 * 16 ? Npad : 148 * 16;  // one block per row (grid-stride)
   convert_h_blocked_kernel<<<(unsigned)(blocks < 1 ? 1 : blocks), 256, 0, st>>>(
-      H, Hb, s.N, Npad, s.D, nkbt, nt, counters, counters ? (s.V + 127) / 128 : 0, err);
+      H, Hb, tsc, s.N, Npad, s.D, nkbt, nt, counters, counters ? (s.V + 127) / 128 : 0, err);
   ++*launches;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_lowrank_t(H, head, s, nullptr, Hb, nt, nkbt, err, st, launches);
 }
 
-cudaError_t launch_residual_tc(const __half* Hb, const archead_head* head, const Shapes& s,
-                               const TcPlan& plan, float* Y, const int32_t* targets,
+cudaError_t launch_residual_tc(const __half* Hb, const float* tsc, const archead_head* head,
+                               const Shapes& s, const TcPlan& plan, float* Y,
+                               const int32_t* targets,
                                float2* part, float* tlogit, float* scratch, unsigned* counters,
                                unsigned* err, cudaStream_t st, int* launches) {
   TcParams p;
   p.Hb = Hb;
+  p.tsc = tsc;
   p.nib = head->r_nib;
   p.code = head->r_code;
   p.sup = head->r_super;

@@ -286,10 +286,16 @@ def test_empty_batch_is_noop(dev, rhead):
     ah.check()
 
 
-def test_fp16_overflow_in_H_is_reported(dev, rhead):
-    _, dh = rhead
+def test_h_beyond_fp16_is_scaled_and_non_finite_h_is_reported(dev, rhead):
+    """An entry beyond the FP16 range is taken (its token is scaled by a power of two,
+    see test_token_scaling.py); a NaN entry is reported and its token's logits are NaN."""
+    head, dh = rhead
     H = _rand_H(3, 512, 9)
     H[1, 17] = 1.0e5
+    Y = ah.logits(H.to(dev), dh)
+    ah.check()
+    _assert_logits(Y.cpu().numpy()[1], oracle.logits(head, bf16_bits(H))[1], "token scaled")
+    H[1, 17] = float("nan")
     Y = ah.logits(H.to(dev), dh)
     with pytest.raises(ah.ArcheadError) as ei:
         ah.check()
