@@ -8,8 +8,10 @@
 //  * persistent grid, one CTA per SM: the last warp is a producer that bulk-copies (TMA
 //    engine, no tensor map, no multicast) two-block stages of the 8 KB packed blocks of
 //    128-row tiles into a shared-memory ring, plus each tile's group codes and INT8 factor
-//    rows; each consumer warp owns 16 rows of the tile (for N <= 8 two warps per 16 rows,
-//    taking the even and the odd stages, iterating over their own stages only);
+//    rows; for N <= 8 each consumer warp owns two 16-row groups of the tile (their H
+//    fragments are loaded once for both) and three warps take the stages of the same rows
+//    in turn, for N <= 16 each warp owns 16 rows and takes every stage; a warp iterates over
+//    its own stages only and probes the next one's barrier one stage ahead;
 //  * the FP16 hidden states of all (<= 16) tokens stay resident in shared memory for the
 //    whole launch, stored with a chunk swizzle that makes the B-fragment reads
 //    conflict-free;
@@ -72,10 +74,14 @@ __host__ __device__ __forceinline__ int64_t dec_h_offset(int64_t n, int64_t d, i
 template <int NT8>
 struct DecCfg {
   static constexpr int NTOK = 8 * NT8;
-  // consumer warps per row group, taking alternate ring stages (latency hiding where the
-  // registers allow two)
-  static constexpr int PAR = NT8 == 1 ? 2 : 1;
-  static constexpr int CONSUMERS = kDecRows * PAR;
+  // consumer warps per set of rows, taking the ring stages in turn (latency hiding where
+  // the registers allow it)
+  static constexpr int PAR = NT8 == 1 ? 3 : 1;
+  // 16-row groups per consumer warp: two for one token block (the H fragments are loaded
+  // once for both, and a stage's handshake serves twice the work)
+  static constexpr int RG = NT8 == 1 ? 2 : 1;
+  static constexpr int WPP = kDecRows / RG;  // consumer warps per stage
+  static constexpr int CONSUMERS = WPP * PAR;
   static constexpr int THREADS = (CONSUMERS + 1) * 32;  // + producer warp
 };
 
@@ -115,7 +121,7 @@ __host__ __device__ inline DecSmem dec_smem(int64_t D, int G, int r_c, int r_r, 
   m.red = o;  // MODE 1: [8 warps][NTOK] float2
   o += MODE ? dec_round16((size_t)kDecRows * NTOK * 8) : 0;
   m.xch = o;  // paired warps: [2][256][NT8] float4 partial sums handed over per tile
-  o += DecCfg<NT8>::PAR == 2 ? (size_t)2 * 256 * NT8 * 16 : 0;
+  o += (size_t)2 * (DecCfg<NT8>::PAR - 1) * 256 * NT8 * 16;
   m.bars = o;
   o += 256;
   m.total = o;
@@ -343,49 +349,62 @@ __device__ __forceinline__ void mma_f16_16816_q(float d[4], const uint32_t a[4],
         "r"(c.z), "r"(c.w));
 }
 
-// NB (1 or 2) consecutive blocks with one group code each (g >= 128): raw nibble reads
-// (nibble_reads) times the resident B image, one chain of eight MMAs per block starting
-// from the block's negated offset constant (a quad of corr), then acc += code * chain.
-// hs: shared address of this thread's H row (token gid) at block kb2, chunk 0; cq: shared
-// address of its corr quad at block kb2.
-template <int NT8, int NB>
-__device__ __forceinline__ void dec_blocks_q(const uint32_t (&wlo)[2][4],
-                                             const uint32_t (&whi)[2][4],
-                                             const uint32_t (&clo)[2], const uint32_t (&chi)[2],
-                                             uint32_t hs, uint32_t hj, const uint32_t (&hoff)[4],
-                                             uint32_t cq, float (&acc)[NT8][4]) {
+// NB (1 or 2) consecutive blocks with one group code each (g >= 128) for RG 16-row groups:
+// raw nibble reads (nibble_reads) times the resident B image (each B fragment loaded once
+// for all row groups), one chain of eight MMAs per (row group, block) starting from the
+// block's negated offset constant (a quad of corr), then acc += code * chain.  hs: shared
+// address of this thread's H row (token gid) at block kb2, chunk 0; cq: shared address of
+// its corr quad at block kb2.
+template <int NT8, int NB, int RG>
+__device__ __forceinline__ void dec_blocks_q(const uint32_t (&wlo)[RG][2][4],
+                                             const uint32_t (&whi)[RG][2][4],
+                                             const uint32_t (&clo)[RG][2],
+                                             const uint32_t (&chi)[RG][2], uint32_t hs,
+                                             uint32_t hj, const uint32_t (&hoff)[4],
+                                             uint32_t cq, float (&acc)[RG][NT8][4]) {
   constexpr int NTOK = 8 * NT8;
-  float t[NB][NT8][4];
+  float t[RG][NB][NT8][4];
 #pragma unroll
   for (int c = 0; c < 4; ++c)
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
-      uint32_t xa[4], xb[4];
-      nibble_reads(wlo[b][c], xa);
-      nibble_reads(whi[b][c], xb);
-      const uint32_t a0[4] = {xa[0], xb[0], xa[1], xb[1]};
-      const uint32_t a1[4] = {xa[2], xb[2], xa[3], xb[3]};
+      uint32_t a0[RG][4], a1[RG][4];
+#pragma unroll
+      for (int r = 0; r < RG; ++r) {
+        uint32_t xa[4], xb[4];
+        nibble_reads(wlo[r][b][c], xa);
+        nibble_reads(whi[r][b][c], xb);
+        a0[r][0] = xa[0]; a0[r][1] = xb[0]; a0[r][2] = xa[1]; a0[r][3] = xb[1];
+        a1[r][0] = xa[2]; a1[r][1] = xb[2]; a1[r][2] = xa[3]; a1[r][3] = xb[3];
+      }
 #pragma unroll
       for (int j = 0; j < NT8; ++j) {
         const uint4 hv = lds128(hs + j * hj + b * 256 + hoff[c]);
-        if (c == 0)
-          mma_f16_16816_q(t[b][j], a0, hv.x, hv.y, lds128(cq + (b * (NTOK / 2) + 4 * j) * 16));
-        else
-          mma_f16_16816(t[b][j], a0, hv.x, hv.y);
-        mma_f16_16816(t[b][j], a1, hv.z, hv.w);
+        uint4 cqv = make_uint4(0, 0, 0, 0);
+        if (c == 0) cqv = lds128(cq + (b * (NTOK / 2) + 4 * j) * 16);
+#pragma unroll
+        for (int r = 0; r < RG; ++r) {
+          if (c == 0)
+            mma_f16_16816_q(t[r][b][j], a0[r], hv.x, hv.y, cqv);
+          else
+            mma_f16_16816(t[r][b][j], a0[r], hv.x, hv.y);
+          mma_f16_16816(t[r][b][j], a1[r], hv.z, hv.w);
+        }
       }
     }
 #pragma unroll
-  for (int b = 0; b < NB; ++b) {
-    const float fl = (float)clo[b], fh = (float)chi[b];
+  for (int r = 0; r < RG; ++r)
 #pragma unroll
-    for (int j = 0; j < NT8; ++j) {
-      acc[j][0] = fmaf(fl, t[b][j][0], acc[j][0]);
-      acc[j][1] = fmaf(fl, t[b][j][1], acc[j][1]);
-      acc[j][2] = fmaf(fh, t[b][j][2], acc[j][2]);
-      acc[j][3] = fmaf(fh, t[b][j][3], acc[j][3]);
+    for (int b = 0; b < NB; ++b) {
+      const float fl = (float)clo[r][b], fh = (float)chi[r][b];
+#pragma unroll
+      for (int j = 0; j < NT8; ++j) {
+        acc[r][j][0] = fmaf(fl, t[r][b][j][0], acc[r][j][0]);
+        acc[r][j][1] = fmaf(fl, t[r][b][j][1], acc[r][j][1]);
+        acc[r][j][2] = fmaf(fh, t[r][b][j][2], acc[r][j][2]);
+        acc[r][j][3] = fmaf(fh, t[r][b][j][3], acc[r][j][3]);
+      }
     }
-  }
 }
 
 template <int NT8, int CPC, int MODE>
@@ -440,7 +459,7 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
     }
     for (int s = 0; s < SP; ++s) {
       tc::mbar_init(&p_full[s], 1);
-      tc::mbar_init(&p_empty[s], kDecRows);  // one warp per row group takes a stage
+      tc::mbar_init(&p_empty[s], DecCfg<NT8>::WPP);  // the warps that take a stage
     }
     tc::mbar_init(dead, 1);
     tc::mbar_fence_init();
@@ -518,11 +537,15 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
     return;
   }
 
-  // ---- consumers: warps w and w + 8 own tile rows 16w .. 16w + 15, taking the even and
-  // the odd ring stages (PAR = 2) ----
+  // ---- consumers: warp w takes the stages k with k % PAR == w / WPP and owns the RG
+  // 16-row groups RG (w % WPP) .. + RG - 1 of the tile ----
+  constexpr int RG = DecCfg<NT8>::RG;
+  constexpr int WPP = DecCfg<NT8>::WPP;
   const int gid = lane >> 2, tq = lane & 3;
-  const int par = warp / kDecRows;
-  const int ctid = threadIdx.x;  // the first eight warps: 0 .. 255
+  const int par = warp / WPP;
+  const int wg = warp % WPP;
+  const int ctid = threadIdx.x;  // 0 .. CONSUMERS * 32 - 1
+  const int etid = wg * 32 + lane;  // the warps of parity 0 (which finish the tiles)
   grid_dependency_wait();  // t and the tile counters come from the prologue kernel
   bool ok = dec_wait(h_full, 0, p.err, true, p.wait_limit);
 #ifdef ARCHEAD_TEST_HOOKS
@@ -547,12 +570,16 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
   asm volatile("bar.sync 10, %0;\n" ::"r"(CONSUMERS * 32) : "memory");
 
   const uint32_t pk_base = tc::smem_u32(pk);
-  // ldmatrix row address of this lane: matrix lane / 8 = (chunk lane / 16, row half
-  // (lane / 8) % 2), row lane % 8; the second load takes chunks 2 and 3
+  // ldmatrix row address of this lane for row group x: matrix lane / 8 = (chunk lane / 16,
+  // row half (lane / 8) % 2), row lane % 8, plus 256 x; the second load takes chunks 2 and 3
   const uint32_t lm_off =
-      (uint32_t)(((lane >> 4) * 128 + 16 * (warp % kDecRows) + 8 * ((lane >> 3) & 1) +
-                  (lane & 7)) * 16);
-  const int r_lo = 16 * (warp % kDecRows) + gid, r_hi = r_lo + 8;
+      (uint32_t)(((lane >> 4) * 128 + 16 * (RG * wg) + 8 * ((lane >> 3) & 1) + (lane & 7)) * 16);
+  int r_lo[RG], r_hi[RG];
+#pragma unroll
+  for (int r = 0; r < RG; ++r) {
+    r_lo[r] = 16 * (RG * wg + r) + gid;
+    r_hi[r] = r_lo[r] + 8;
+  }
   const float NEG_INF = __int_as_float(0xff800000);
   // B reads: byte offset of token 8j + gid's columns 32 tq + 8c of block kb in the
   // resident image is hrow[j] + 256 kb + hoff[c] (dec_h_offset unrolled)
@@ -561,11 +588,12 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
   for (int j = 0; j < NT8; ++j) hrow[j] = (8 * j + gid) * (int)D * 2 + 64 * tq;
   const int hx = (((tq >> 1) & 1) << 1) ^ (gid & 1);
   int hoff[4];
-#pragma unroll
-  for (int c = 0; c < 4; ++c) hoff[c] = 16 * (c ^ hx);
   uint32_t hoffu[4];
 #pragma unroll
-  for (int c = 0; c < 4; ++c) hoffu[c] = (uint32_t)hoff[c];
+  for (int c = 0; c < 4; ++c) {
+    hoff[c] = 16 * (c ^ hx);
+    hoffu[c] = (uint32_t)hoff[c];
+  }
   const uint32_t hs0 = tc::smem_u32(Hb) + (uint32_t)hrow[0];
   const uint32_t hj = (uint32_t)(8 * D * 2);
   const uint32_t cq0 = corr_s + (uint32_t)tq * 16;
@@ -578,25 +606,25 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
     const int kb1 = (int)((int64_t)nkb < kb0 + (u1 - u) ? (int64_t)nkb : kb0 + (u1 - u));
     const int cs = s & 1;
     const int64_t row0 = T * 128;
-    const int64_t v_lo = row0 + r_lo, v_hi = row0 + r_hi;
-    const int64_t vc_lo = v_lo < p.V ? v_lo : p.V - 1, vc_hi = v_hi < p.V ? v_hi : p.V - 1;
-    // row scales for the epilogue: the loads overlap the block loop
-    const float S_lo = bf16_bits_to_float(__ldg(p.sup + vc_lo));
-    const float S_hi = bf16_bits_to_float(__ldg(p.sup + vc_hi));
-    const float sac_lo = p.r_c ? __ldg(p.sAc + vc_lo) : 0.f, sac_hi = p.r_c ? __ldg(p.sAc + vc_hi) : 0.f;
-    const float saw_lo = p.r_r ? __ldg(p.sAw + vc_lo) : 0.f, saw_hi = p.r_r ? __ldg(p.sAw + vc_hi) : 0.f;
     ok = dec_wait(&c_full[cs], (s >> 1) & 1, p.err, ok, p.wait_limit);
-    const unsigned char* crow_lo = cds + cs * code_slot + r_lo * G;
-    const unsigned char* crow_hi = cds + cs * code_slot + r_hi * G;
+    const unsigned char* crow_lo[RG];
+    const unsigned char* crow_hi[RG];
+#pragma unroll
+    for (int r = 0; r < RG; ++r) {
+      crow_lo[r] = cds + cs * code_slot + r_lo[r] * G;
+      crow_hi[r] = cds + cs * code_slot + r_hi[r] * G;
+    }
 
-    float acc[NT8][4];
+    float acc[RG][NT8][4];
 #pragma unroll
-    for (int j = 0; j < NT8; ++j)
+    for (int r = 0; r < RG; ++r)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
+      for (int j = 0; j < NT8; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[r][j][e] = 0.f;
 
     const int nst = (kb1 - kb0 + 1) >> 1;  // stages of this tile segment
-    int i0 = (PAR == 2 && (k & 1) != par) ? 1 : 0;  // this warp's first stage of them
+    int i0 = (par - k % PAR + PAR) % PAR;  // this warp's first stage of them
     int st = (k + i0) % SP;
     uint32_t ph = (uint32_t)((k + i0) / SP) & 1u;
     k += nst;
@@ -604,23 +632,26 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
       const int kb2 = kb0 + 2 * i;
       if (!nready) ok = ok && tc::mbar_wait(&p_full[st], ph, p.err, p.wait_limit);
       const int nb = kb2 + 1 < kb1 ? 2 : 1;
-      uint32_t wlo[2][4], whi[2][4];  // [block][chunk]: word tq of rows r_lo, r_hi
-      uint32_t clo[2], chi[2];
+      uint32_t wlo[RG][2][4], whi[RG][2][4];  // [group][block][chunk]: word tq of rows r_lo, r_hi
+      uint32_t clo[RG][2], chi[RG][2];
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
         if (b < nb) {
-          const uint32_t sa = pk_base + (uint32_t)(st * 2 + b) * kDecPk + lm_off;
-          uint32_t r[4];
-          ldmatrix_x4(sa, r);
-          wlo[b][0] = r[0]; whi[b][0] = r[1]; wlo[b][1] = r[2]; whi[b][1] = r[3];
-          ldmatrix_x4(sa + 2 * 128 * 16, r);
-          wlo[b][2] = r[0]; whi[b][2] = r[1]; wlo[b][3] = r[2]; whi[b][3] = r[3];
           // group code of this thread's 32-column window (columns 32 tq .. 32 tq + 31)
           const int kb = kb2 + b;
           const int ci = CPC == 1 ? ((kb * 128) >> p.g_shift)
                                   : (CPC == 2 ? kb * 2 + (tq >> 1) : kb * 4 + tq);
-          clo[b] = crow_lo[ci];
-          chi[b] = crow_hi[ci];
+#pragma unroll
+          for (int r = 0; r < RG; ++r) {
+            const uint32_t sa = pk_base + (uint32_t)(st * 2 + b) * kDecPk + lm_off + 256 * r;
+            uint32_t q[4];
+            ldmatrix_x4(sa, q);
+            wlo[r][b][0] = q[0]; whi[r][b][0] = q[1]; wlo[r][b][1] = q[2]; whi[r][b][1] = q[3];
+            ldmatrix_x4(sa + 2 * 128 * 16, q);
+            wlo[r][b][2] = q[0]; whi[r][b][2] = q[1]; wlo[r][b][3] = q[2]; whi[r][b][3] = q[3];
+            clo[r][b] = crow_lo[r][ci];
+            chi[r][b] = crow_hi[r][ci];
+          }
         }
       }
       __syncwarp();
@@ -630,52 +661,58 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
         st -= SP;
         ph ^= 1u;
       }
-      // The next stage's barrier is probed now (non-blocking) and its answer used at the
-      // next stage, so the round trip overlaps this stage's arithmetic; a phase seen
-      // complete stays complete until this warp releases the slot.
       nready = tc::mbar_test(&p_full[st], ph);
       if (CPC == 1) {
         const uint32_t hs = hs0 + (uint32_t)kb2 * 256u;
         const uint32_t cq = cq0 + (uint32_t)kb2 * (NTOK * 8);
         if (nb == 2)
-          dec_blocks_q<NT8, 2>(wlo, whi, clo, chi, hs, hj, hoffu, cq, acc);
+          dec_blocks_q<NT8, 2, RG>(wlo, whi, clo, chi, hs, hj, hoffu, cq, acc);
         else
-          dec_blocks_q<NT8, 1>(wlo, whi, clo, chi, hs, hj, hoffu, cq, acc);
+          dec_blocks_q<NT8, 1, RG>(wlo, whi, clo, chi, hs, hj, hoffu, cq, acc);
       } else {
 #pragma unroll
         for (int b = 0; b < 2; ++b) {
           if (b >= nb) break;
           const int hb = (kb2 + b) * 256;
-          const __half2 c2lo = __half2half2(__ushort2half_rn((unsigned short)clo[b]));
-          const __half2 c2hi = __half2half2(__ushort2half_rn((unsigned short)chi[b]));
-          const __half2 m24 = __float2half2_rn(-24.f);
-          const __half2 n2lo = __hmul2(c2lo, m24), n2hi = __hmul2(c2hi, m24);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            __half2 pa[4], pb[4];
-            dequant_word(wlo[b][c], c2lo, n2lo, pa);
-            dequant_word(whi[b][c], c2hi, n2hi, pb);
-            const uint32_t a0[4] = {h2_bits(pa[0]), h2_bits(pb[0]), h2_bits(pa[1]), h2_bits(pb[1])};
-            const uint32_t a1[4] = {h2_bits(pa[2]), h2_bits(pb[2]), h2_bits(pa[3]), h2_bits(pb[3])};
+          for (int r = 0; r < RG; ++r) {
+            const __half2 c2lo = __half2half2(__ushort2half_rn((unsigned short)clo[r][b]));
+            const __half2 c2hi = __half2half2(__ushort2half_rn((unsigned short)chi[r][b]));
+            const __half2 m24 = __float2half2_rn(-24.f);
+            const __half2 n2lo = __hmul2(c2lo, m24), n2hi = __hmul2(c2hi, m24);
 #pragma unroll
-            for (int j = 0; j < NT8; ++j) {
-              const uint4 hv = *reinterpret_cast<const uint4*>(Hb + hrow[j] + hb + hoff[c]);
-              mma_f16_16816(acc[j], a0, hv.x, hv.y);
-              mma_f16_16816(acc[j], a1, hv.z, hv.w);
+            for (int c = 0; c < 4; ++c) {
+              __half2 pa[4], pb[4];
+              dequant_word(wlo[r][b][c], c2lo, n2lo, pa);
+              dequant_word(whi[r][b][c], c2hi, n2hi, pb);
+              const uint32_t a0[4] = {h2_bits(pa[0]), h2_bits(pb[0]), h2_bits(pa[1]), h2_bits(pb[1])};
+              const uint32_t a1[4] = {h2_bits(pa[2]), h2_bits(pb[2]), h2_bits(pa[3]), h2_bits(pb[3])};
+#pragma unroll
+              for (int j = 0; j < NT8; ++j) {
+                const uint4 hv = *reinterpret_cast<const uint4*>(Hb + hrow[j] + hb + hoff[c]);
+                mma_f16_16816(acc[r][j], a0, hv.x, hv.y);
+                mma_f16_16816(acc[r][j], a1, hv.z, hv.w);
+              }
             }
           }
         }
       }
     }
 
-    // ---- paired warps: the odd-stage warp hands its sums to the even-stage warp ----
-    if (PAR == 2) {
-      float4* xs = xch + ((size_t)(s & 1) * 256 + (warp % kDecRows) * 32 + lane) * NT8;
+    // ---- warps of one row-group set: the warps of parity > 0 hand their sums to parity 0
+    // (double-buffered by segment parity: parity 0 has read the buffers of segment s - 2
+    // before it met the others at the barrier of segment s - 1) ----
+    if (PAR > 1) {
       if (par) {
 #pragma unroll
-        for (int j = 0; j < NT8; ++j) xs[j] = make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
+        for (int r = 0; r < RG; ++r) {
+          float4* xs = xch + ((((size_t)(s & 1) * (PAR - 1) + par - 1) * 256) + (RG * wg + r) * 32 + lane) * NT8;
+#pragma unroll
+          for (int j = 0; j < NT8; ++j)
+            xs[j] = make_float4(acc[r][j][0], acc[r][j][1], acc[r][j][2], acc[r][j][3]);
+        }
       }
-      asm volatile("bar.sync %0, 64;\n" ::"r"(2 + warp % kDecRows) : "memory");
+      asm volatile("bar.sync %0, %1;\n" ::"r"(2 + wg), "r"(32 * PAR) : "memory");
       if (par) {
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&c_empty[cs]);
@@ -683,201 +720,230 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
         continue;
       }
 #pragma unroll
-      for (int j = 0; j < NT8; ++j) {
-        const float4 q = xs[j];
-        acc[j][0] += q.x; acc[j][1] += q.y; acc[j][2] += q.z; acc[j][3] += q.w;
-      }
+      for (int q2 = 1; q2 < PAR; ++q2)
+#pragma unroll
+        for (int r = 0; r < RG; ++r) {
+          const float4* xs = xch + ((((size_t)(s & 1) * (PAR - 1) + q2 - 1) * 256) + (RG * wg + r) * 32 + lane) * NT8;
+#pragma unroll
+          for (int j = 0; j < NT8; ++j) {
+            const float4 q = xs[j];
+            acc[r][j][0] += q.x; acc[r][j][1] += q.y; acc[r][j][2] += q.z; acc[r][j][3] += q.w;
+          }
+        }
     }
 
     // ---- a tile split between CTAs: the last contributor to arrive finishes it ----
     bool finish = kb0 == 0 && kb1 == nkb;
     if (!finish) {
       const int slot = u == u0 ? 0 : 1;
-      float4* dst = p.scratch + (((int64_t)blockIdx.x * 2 + slot) * 256 + ctid) * NT8;
 #pragma unroll
-      for (int j = 0; j < NT8; ++j) dst[j] = make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
+      for (int r = 0; r < RG; ++r) {
+        float4* dst = p.scratch + (((int64_t)blockIdx.x * 2 + slot) * 256 + (RG * wg + r) * 32 + lane) * NT8;
+#pragma unroll
+        for (int j = 0; j < NT8; ++j)
+          dst[j] = make_float4(acc[r][j][0], acc[r][j][1], acc[r][j][2], acc[r][j][3]);
+      }
       __threadfence();
-      asm volatile("bar.sync 1, 256;\n" ::: "memory");
+      asm volatile("bar.sync 1, %0;\n" ::"r"(WPP * 32) : "memory");
       const int64_t cf = dec_cta_of(T * nkb, U, C), cl = dec_cta_of(T * nkb + nkb - 1, U, C);
-      if (ctid == 0) {
+      if (etid == 0) {
         const unsigned old = atomicAdd(p.counters + T, 1u);
         *flag = (int64_t)old + 1 == cl - cf + 1;
       }
-      asm volatile("bar.sync 1, 256;\n" ::: "memory");
+      asm volatile("bar.sync 1, %0;\n" ::"r"(WPP * 32) : "memory");
       finish = *flag != 0;
       if (finish) {
         __threadfence();
 #pragma unroll
-        for (int j = 0; j < NT8; ++j)
+        for (int r = 0; r < RG; ++r)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
+          for (int j = 0; j < NT8; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[r][j][e] = 0.f;
         for (int64_t c = cf; c <= cl; ++c) {  // fixed order: the sum is deterministic
           const int64_t first_tile = (U * c / C) / nkb;
           const int sl = T == first_tile ? 0 : 1;
-          const float4* src = p.scratch + ((c * 2 + sl) * 256 + ctid) * NT8;
 #pragma unroll
-          for (int j = 0; j < NT8; ++j) {
-            const float4 q = __ldcg(src + j);
-            acc[j][0] += q.x; acc[j][1] += q.y; acc[j][2] += q.z; acc[j][3] += q.w;
+          for (int r = 0; r < RG; ++r) {
+            const float4* src = p.scratch + ((c * 2 + sl) * 256 + (RG * wg + r) * 32 + lane) * NT8;
+#pragma unroll
+            for (int j = 0; j < NT8; ++j) {
+              const float4 q = __ldcg(src + j);
+              acc[r][j][0] += q.x; acc[r][j][1] += q.y; acc[r][j][2] += q.z; acc[r][j][3] += q.w;
+            }
           }
         }
       }
     }
 
     if (finish) {
-      // ---- epilogue: S_v acc + sAc Ac . t_c + sAw Aw . t_w ----
+      // ---- epilogue: S_v acc + sAc Ac . t_c + sAw Aw . t_w, per row group ----
       const int64_t rows = p.V - row0 < 128 ? p.V - row0 : 128;
       const bool acopy = dec_arow_copy(rows, p.r_c, p.r_r);
-      float y[NT8][4];
 #pragma unroll
-      for (int j = 0; j < NT8; ++j) {
-        y[j][0] = S_lo * acc[j][0];
-        y[j][1] = S_lo * acc[j][1];
-        y[j][2] = S_hi * acc[j][2];
-        y[j][3] = S_hi * acc[j][3];
-      }
-      if (rank_mma) {
-        // [A_c | A_w] rows (INT8, exact in FP16) x FP16 hi / lo pieces of t, one FP32
-        // accumulator per factor; thread q's K slots hold factor entries 16 s + 4 q + 0..3
+      for (int r = 0; r < RG; ++r) {
+        const int64_t v_lo = row0 + r_lo[r], v_hi = row0 + r_hi[r];
+        const int64_t vc_lo = v_lo < p.V ? v_lo : p.V - 1, vc_hi = v_hi < p.V ? v_hi : p.V - 1;
+        // row scales of the epilogue: the warps of parity 0 load them here while the others
+        // already stream the next segment
+        const float S_lo = bf16_bits_to_float(__ldg(p.sup + vc_lo));
+        const float S_hi = bf16_bits_to_float(__ldg(p.sup + vc_hi));
+        const float sac_lo = p.r_c ? __ldg(p.sAc + vc_lo) : 0.f, sac_hi = p.r_c ? __ldg(p.sAc + vc_hi) : 0.f;
+        const float saw_lo = p.r_r ? __ldg(p.sAw + vc_lo) : 0.f, saw_hi = p.r_r ? __ldg(p.sAw + vc_hi) : 0.f;
+        float y[NT8][4];
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          const int rank = part == 0 ? p.r_c : p.r_r;
-          if (rank == 0) continue;
-          const int8_t* abase = acopy ? (part == 0 ? arc + cs * arc_slot : arw + cs * arw_slot)
-                                      : (part == 0 ? p.Ac : p.Aw);
-          const int8_t* alo = abase + (acopy ? (int64_t)r_lo : vc_lo) * rank;
-          const int8_t* ahi = abase + (acopy ? (int64_t)r_hi : vc_hi) * rank;
-          const int off = part == 0 ? 0 : p.r_c;
-          float L[NT8][4];
+        for (int j = 0; j < NT8; ++j) {
+          y[j][0] = S_lo * acc[r][j][0];
+          y[j][1] = S_lo * acc[r][j][1];
+          y[j][2] = S_hi * acc[r][j][2];
+          y[j][3] = S_hi * acc[r][j][3];
+        }
+        if (rank_mma) {
+          // [A_c | A_w] rows (INT8, exact in FP16) x FP16 hi / lo pieces of t, one FP32
+          // accumulator per factor; thread q's K slots hold factor entries 16 s + 4 q + 0..3
 #pragma unroll
-          for (int j = 0; j < NT8; ++j) L[j][0] = L[j][1] = L[j][2] = L[j][3] = 0.f;
-          const __half2 k1152 = __float2half2_rn(1152.f);
-          for (int st16 = 0; st16 < rank; st16 += 16) {
-            const uint32_t wl = *reinterpret_cast<const uint32_t*>(alo + st16 + 4 * tq) ^ 0x80808080u;
-            const uint32_t wh = *reinterpret_cast<const uint32_t*>(ahi + st16 + 4 * tq) ^ 0x80808080u;
-            // bytes b + 128 under the FP16 pattern 0x6400 read 1024 + b + 128: minus 1152
-            uint32_t q0 = __byte_perm(wl, 0x64646464u, 0x5140), q1 = __byte_perm(wl, 0x64646464u, 0x7352);
-            uint32_t q2 = __byte_perm(wh, 0x64646464u, 0x5140), q3 = __byte_perm(wh, 0x64646464u, 0x7352);
-            const uint32_t a[4] = {h2_bits(__hsub2(*reinterpret_cast<__half2*>(&q0), k1152)),
-                                   h2_bits(__hsub2(*reinterpret_cast<__half2*>(&q2), k1152)),
-                                   h2_bits(__hsub2(*reinterpret_cast<__half2*>(&q1), k1152)),
-                                   h2_bits(__hsub2(*reinterpret_cast<__half2*>(&q3), k1152))};
+          for (int part = 0; part < 2; ++part) {
+            const int rank = part == 0 ? p.r_c : p.r_r;
+            if (rank == 0) continue;
+            const int8_t* abase = acopy ? (part == 0 ? arc + cs * arc_slot : arw + cs * arw_slot)
+                                        : (part == 0 ? p.Ac : p.Aw);
+            const int8_t* alo = abase + (acopy ? (int64_t)r_lo[r] : vc_lo) * rank;
+            const int8_t* ahi = abase + (acopy ? (int64_t)r_hi[r] : vc_hi) * rank;
+            const int off = part == 0 ? 0 : p.r_c;
+            float L[NT8][4];
 #pragma unroll
-            for (int pc = 0; pc < 2; ++pc)
+            for (int j = 0; j < NT8; ++j) L[j][0] = L[j][1] = L[j][2] = L[j][3] = 0.f;
+            const __half2 k1152 = __float2half2_rn(1152.f);
+            for (int st16 = 0; st16 < rank; st16 += 16) {
+              const uint32_t wl = *reinterpret_cast<const uint32_t*>(alo + st16 + 4 * tq) ^ 0x80808080u;
+              const uint32_t wh = *reinterpret_cast<const uint32_t*>(ahi + st16 + 4 * tq) ^ 0x80808080u;
+              // bytes b + 128 under the FP16 pattern 0x6400 read 1024 + b + 128: minus 1152
+              uint32_t q0 = __byte_perm(wl, 0x64646464u, 0x5140), q1 = __byte_perm(wl, 0x64646464u, 0x7352);
+              uint32_t q2 = __byte_perm(wh, 0x64646464u, 0x5140), q3 = __byte_perm(wh, 0x64646464u, 0x7352);
+              const uint32_t a[4] = {h2_bits(__hsub2(*reinterpret_cast<__half2*>(&q0), k1152)),
+                                     h2_bits(__hsub2(*reinterpret_cast<__half2*>(&q2), k1152)),
+                                     h2_bits(__hsub2(*reinterpret_cast<__half2*>(&q1), k1152)),
+                                     h2_bits(__hsub2(*reinterpret_cast<__half2*>(&q3), k1152))};
+#pragma unroll
+              for (int pc = 0; pc < 2; ++pc)
+#pragma unroll
+                for (int j = 0; j < NT8; ++j) {
+                  const uint2 bv = *reinterpret_cast<const uint2*>(
+                      ts16 + (pc * NTOK + 8 * j + gid) * tsb + (off + st16 + 4 * tq) * 2);
+                  mma_f16_16816(L[j], a, bv.x, bv.y);
+                }
+            }
+            const float sl = part == 0 ? sac_lo : saw_lo, sh = part == 0 ? sac_hi : saw_hi;
+#pragma unroll
+            for (int j = 0; j < NT8; ++j) {
+              y[j][0] = fmaf(sl, L[j][0], y[j][0]);
+              y[j][1] = fmaf(sl, L[j][1], y[j][1]);
+              y[j][2] = fmaf(sh, L[j][2], y[j][2]);
+              y[j][3] = fmaf(sh, L[j][3], y[j][3]);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int part = 0; part < 2; ++part) {
+            const int rank = part == 0 ? p.r_c : p.r_r;
+            if (rank == 0) continue;
+            const int8_t* abase = acopy ? (part == 0 ? arc + cs * arc_slot : arw + cs * arw_slot)
+                                        : (part == 0 ? p.Ac : p.Aw);
+            const int8_t* alo = abase + (acopy ? (int64_t)r_lo[r] : vc_lo) * rank;
+            const int8_t* ahi = abase + (acopy ? (int64_t)r_hi[r] : vc_hi) * rank;
+            const float* tcol = ts + (part == 0 ? 0 : p.r_c) * NTOK + 2 * tq;
+            float llo[NT8][2], lhi[NT8][2];
+#pragma unroll
+            for (int j = 0; j < NT8; ++j) llo[j][0] = llo[j][1] = lhi[j][0] = lhi[j][1] = 0.f;
+            auto step = [&](float al, float ah, int i) {
 #pragma unroll
               for (int j = 0; j < NT8; ++j) {
-                const uint2 bv = *reinterpret_cast<const uint2*>(
-                    ts16 + (pc * NTOK + 8 * j + gid) * tsb + (off + st16 + 4 * tq) * 2);
-                mma_f16_16816(L[j], a, bv.x, bv.y);
+                const float2 tv = *reinterpret_cast<const float2*>(tcol + i * NTOK + 8 * j);
+                llo[j][0] = fmaf(al, tv.x, llo[j][0]);
+                llo[j][1] = fmaf(al, tv.y, llo[j][1]);
+                lhi[j][0] = fmaf(ah, tv.x, lhi[j][0]);
+                lhi[j][1] = fmaf(ah, tv.y, lhi[j][1]);
+              }
+            };
+            int i = 0;
+            if ((rank & 3) == 0) {  // four INT8 entries per 32-bit load (rows 4-byte aligned)
+              for (; i < rank; i += 4) {
+                const uint32_t wl = *reinterpret_cast<const uint32_t*>(alo + i);
+                const uint32_t wh = *reinterpret_cast<const uint32_t*>(ahi + i);
+#pragma unroll
+                for (int b = 0; b < 4; ++b)
+                  step((float)(int8_t)(wl >> (8 * b)), (float)(int8_t)(wh >> (8 * b)), i + b);
+              }
+            }
+            for (; i < rank; ++i) step((float)alo[i], (float)ahi[i], i);
+            const float sl = part == 0 ? sac_lo : saw_lo, sh = part == 0 ? sac_hi : saw_hi;
+#pragma unroll
+            for (int j = 0; j < NT8; ++j) {
+              y[j][0] = fmaf(sl, llo[j][0], y[j][0]);
+              y[j][1] = fmaf(sl, llo[j][1], y[j][1]);
+              y[j][2] = fmaf(sh, lhi[j][0], y[j][2]);
+              y[j][3] = fmaf(sh, lhi[j][1], y[j][3]);
+            }
+          }
+        }
+        // the logits of the scaled tokens (8 j + 2 tq + e): times 2^e_n
+#pragma unroll
+        for (int j = 0; j < NT8; ++j) {
+          const float2 tk = *reinterpret_cast<const float2*>(
+              smem + m.h + (size_t)NTOK * D * 2 + (size_t)nkb * NTOK * 8 + (8 * j + 2 * tq) * 4);
+          y[j][0] *= tk.x;
+          y[j][1] *= tk.y;
+          y[j][2] *= tk.x;
+          y[j][3] *= tk.y;
+        }
+        if (MODE == 0) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int64_t v = h ? v_hi : v_lo;
+            if (v >= p.V) continue;
+#pragma unroll
+            for (int j = 0; j < NT8; ++j)
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int64_t tok = 8 * j + 2 * tq + e;
+                if (tok < p.N) __stcs(p.Y + tok * p.V + v, y[j][2 * h + e]);
               }
           }
-          const float sl = part == 0 ? sac_lo : saw_lo, sh = part == 0 ? sac_hi : saw_hi;
-#pragma unroll
-          for (int j = 0; j < NT8; ++j) {
-            y[j][0] = fmaf(sl, L[j][0], y[j][0]);
-            y[j][1] = fmaf(sl, L[j][1], y[j][1]);
-            y[j][2] = fmaf(sh, L[j][2], y[j][2]);
-            y[j][3] = fmaf(sh, L[j][3], y[j][3]);
-          }
-        }
-      } else {
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          const int rank = part == 0 ? p.r_c : p.r_r;
-          if (rank == 0) continue;
-          const int8_t* abase = acopy ? (part == 0 ? arc + cs * arc_slot : arw + cs * arw_slot)
-                                      : (part == 0 ? p.Ac : p.Aw);
-          const int8_t* alo = abase + (acopy ? (int64_t)r_lo : vc_lo) * rank;
-          const int8_t* ahi = abase + (acopy ? (int64_t)r_hi : vc_hi) * rank;
-          const float* tcol = ts + (part == 0 ? 0 : p.r_c) * NTOK + 2 * tq;
-          float llo[NT8][2], lhi[NT8][2];
-  #pragma unroll
-          for (int j = 0; j < NT8; ++j) llo[j][0] = llo[j][1] = lhi[j][0] = lhi[j][1] = 0.f;
-          auto step = [&](float al, float ah, int i) {
-  #pragma unroll
-            for (int j = 0; j < NT8; ++j) {
-              const float2 tv = *reinterpret_cast<const float2*>(tcol + i * NTOK + 8 * j);
-              llo[j][0] = fmaf(al, tv.x, llo[j][0]);
-              llo[j][1] = fmaf(al, tv.y, llo[j][1]);
-              lhi[j][0] = fmaf(ah, tv.x, lhi[j][0]);
-              lhi[j][1] = fmaf(ah, tv.y, lhi[j][1]);
-            }
-          };
-          int i = 0;
-          if ((rank & 3) == 0) {  // four INT8 entries per 32-bit load (rows 4-byte aligned)
-            for (; i < rank; i += 4) {
-              const uint32_t wl = *reinterpret_cast<const uint32_t*>(alo + i);
-              const uint32_t wh = *reinterpret_cast<const uint32_t*>(ahi + i);
-  #pragma unroll
-              for (int b = 0; b < 4; ++b)
-                step((float)(int8_t)(wl >> (8 * b)), (float)(int8_t)(wh >> (8 * b)), i + b);
-            }
-          }
-          for (; i < rank; ++i) step((float)alo[i], (float)ahi[i], i);
-          const float sl = part == 0 ? sac_lo : saw_lo, sh = part == 0 ? sac_hi : saw_hi;
-  #pragma unroll
-          for (int j = 0; j < NT8; ++j) {
-            y[j][0] = fmaf(sl, llo[j][0], y[j][0]);
-            y[j][1] = fmaf(sl, llo[j][1], y[j][1]);
-            y[j][2] = fmaf(sh, lhi[j][0], y[j][2]);
-            y[j][3] = fmaf(sh, lhi[j][1], y[j][3]);
-          }
-        }
-      }
-      // the logits of the scaled tokens (8 j + 2 tq + e): times 2^e_n
-#pragma unroll
-      for (int j = 0; j < NT8; ++j) {
-        const float2 tk = *reinterpret_cast<const float2*>(
-            smem + m.h + (size_t)NTOK * D * 2 + (size_t)nkb * NTOK * 8 + (8 * j + 2 * tq) * 4);
-        y[j][0] *= tk.x;
-        y[j][1] *= tk.y;
-        y[j][2] *= tk.x;
-        y[j][3] *= tk.y;
-      }
-      if (MODE == 0) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int64_t v = h ? v_hi : v_lo;
-          if (v >= p.V) continue;
+        } else {
+          // ---- fused NLL: per token (max, sum exp) over the row group's rows, target logit ----
 #pragma unroll
           for (int j = 0; j < NT8; ++j)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-              const int64_t tok = 8 * j + 2 * tq + e;
-              if (tok < p.N) __stcs(p.Y + tok * p.V + v, y[j][2 * h + e]);
+              float mx = NEG_INF;
+              if (v_lo < p.V) mx = fmaxf(mx, y[j][e]);
+              if (v_hi < p.V) mx = fmaxf(mx, y[j][2 + e]);
+              float sm = 0.f;
+              if (v_lo < p.V) sm += __expf(y[j][e] - mx);
+              if (v_hi < p.V) sm += __expf(y[j][2 + e] - mx);
+#pragma unroll
+              for (int o = 4; o < 32; o <<= 1) {  // the 8 lanes sharing this token
+                const float mo = __shfl_xor_sync(0xffffffffu, mx, o);
+                const float so = __shfl_xor_sync(0xffffffffu, sm, o);
+                const float mn = fmaxf(mx, mo);
+                sm = (mx == NEG_INF ? 0.f : sm * __expf(mx - mn)) +
+                     (mo == NEG_INF ? 0.f : so * __expf(mo - mn));
+                mx = mn;
+              }
+              const int n = 8 * j + 2 * tq + e;
+              if (gid == 0) red[(RG * wg + r) * NTOK + n] = make_float2(mx, sm);
+              if (n < p.N) {
+                const int64_t tgt = __ldg(p.targets + n);
+                if (v_lo == tgt && v_lo < p.V) p.tlogit[n] = y[j][e];
+                if (v_hi == tgt && v_hi < p.V) p.tlogit[n] = y[j][2 + e];
+              }
             }
         }
-      } else {
-        // ---- fused NLL: per token (max, sum exp) over the tile's rows, target logit ----
-#pragma unroll
-        for (int j = 0; j < NT8; ++j)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            float mx = NEG_INF;
-            if (v_lo < p.V) mx = fmaxf(mx, y[j][e]);
-            if (v_hi < p.V) mx = fmaxf(mx, y[j][2 + e]);
-            float sm = 0.f;
-            if (v_lo < p.V) sm += __expf(y[j][e] - mx);
-            if (v_hi < p.V) sm += __expf(y[j][2 + e] - mx);
-#pragma unroll
-            for (int o = 4; o < 32; o <<= 1) {  // the 8 lanes sharing this token
-              const float mo = __shfl_xor_sync(0xffffffffu, mx, o);
-              const float so = __shfl_xor_sync(0xffffffffu, sm, o);
-              const float mn = fmaxf(mx, mo);
-              sm = (mx == NEG_INF ? 0.f : sm * __expf(mx - mn)) +
-                   (mo == NEG_INF ? 0.f : so * __expf(mo - mn));
-              mx = mn;
-            }
-            const int n = 8 * j + 2 * tq + e;
-            if (gid == 0) red[warp * NTOK + n] = make_float2(mx, sm);
-            if (n < p.N) {
-              const int64_t tgt = __ldg(p.targets + n);
-              if (v_lo == tgt && v_lo < p.V) p.tlogit[n] = y[j][e];
-              if (v_hi == tgt && v_hi < p.V) p.tlogit[n] = y[j][2 + e];
-            }
-          }
-        asm volatile("bar.sync 1, 256;\n" ::: "memory");
-        for (int n = ctid; n < NTOK; n += kDecRows * 32) {
+      }
+      if (MODE != 0) {
+        // the tile's (max, sum exp) per token from its eight row groups
+        asm volatile("bar.sync 1, %0;\n" ::"r"(WPP * 32) : "memory");
+        for (int n = etid; n < NTOK; n += WPP * 32) {
           if (n >= p.N) continue;
           float mx = NEG_INF, sm = 0.f;
           for (int w = 0; w < kDecRows; ++w) {
@@ -889,7 +955,7 @@ __global__ void __launch_bounds__(DecCfg<NT8>::THREADS, 1)
           }
           p.part[(int64_t)n * p.n_vtiles + T] = make_float2(mx, sm);
         }
-        asm volatile("bar.sync 1, 256;\n" ::: "memory");
+        asm volatile("bar.sync 1, %0;\n" ::"r"(WPP * 32) : "memory");
       }
     }
     __syncwarp();
@@ -906,7 +972,7 @@ cudaError_t launch_dec_cfg(const DecParams& p, int grid, cudaStream_t st) {
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  if (DecCfg<NT8>::PAR == 2 && p.sp % 2 != 0) return cudaErrorInvalidValue;
+  if (p.sp % DecCfg<NT8>::PAR != 0) return cudaErrorInvalidValue;
   return launch_dependent(kern, grid, DecCfg<NT8>::THREADS, smem, st, p);
 }
 
@@ -917,15 +983,15 @@ cudaError_t launch_dec_nt(const DecParams& p, int g, int grid, cudaStream_t st) 
   return launch_dec_cfg<NT8, 1, MODE>(p, grid, st);
 }
 
-// Paired warps take stages by the parity of the global stage index; with an even number
-// of ring slots every use of a slot then goes to the same warp, which never waits on a
-// slot's mbarrier more than one phase ahead (an odd count would let a fast warp skip a
-// phase and alias the parity test).
+// The PAR warps of a row-group set take stages by the global stage index modulo PAR; with
+// a ring of a multiple of PAR slots every use of a slot then goes to the same warps, which
+// never wait on a slot's mbarrier more than one phase ahead (another count would let a
+// fast warp skip a phase and alias the parity test).
 template <int NT8, int MODE>
 int fit_sp(const Shapes& s, size_t budget) {
   const int G = (int)(s.D / s.g);
   for (int sp = kDecMaxSP; sp >= 3; --sp)
-    if ((DecCfg<NT8>::PAR == 1 || sp % 2 == 0) &&
+    if (sp % DecCfg<NT8>::PAR == 0 &&
         dec_smem<NT8, MODE>(s.D, G, s.r_c, s.r_r, sp).total <= budget)
       return sp;
   return 0;
