@@ -120,7 +120,7 @@ __host__ __device__ inline DecSmem dec_smem(int64_t D, int G, int r_c, int r_r, 
   o += (size_t)2 * NTOK * dec_ts16_stride(r_c + r_r);
   m.red = o;  // MODE 1: [8 warps][NTOK] float2
   o += MODE ? dec_round16((size_t)kDecRows * NTOK * 8) : 0;
-  m.xch = o;  // paired warps: [2][256][NT8] float4 partial sums handed over per tile
+  m.xch = o;  // [2][PAR - 1][256][NT8] float4 partial sums handed to the warps of parity 0
   o += (size_t)2 * (DecCfg<NT8>::PAR - 1) * 256 * NT8 * 16;
   m.bars = o;
   o += 256;
