@@ -208,7 +208,8 @@ int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* ta
   // a single token tile is split evenly over the CTAs (partials + per-tile counters)
   const size_t split_bytes = use_tc ? tc_split_scratch_bytes(s, plan) : 0;
   const size_t o_scr = split_bytes ? cv.take(split_bytes) : 0;
-  const size_t o_cnt = split_bytes ? cv.take((size_t)((s.V + 127) / 128) * 4) : 0;
+  // per-tile counters of a split launch, or the work counter of the dynamic item order
+  const size_t o_cnt = use_tc ? cv.take((size_t)((s.V + 127) / 128) * 4) : 0;
   const size_t o_tloc = shard ? cv.take((size_t)s.N * 4) : 0;
   void* base = nullptr;
   if (cudaMallocFromPoolAsync(&base, cv.off, ds->pool, st) != cudaSuccess) {
@@ -218,7 +219,7 @@ int run(const uint16_t* H, const archead_head* head, float* Y, const int32_t* ta
   char* b = static_cast<char*>(base);
   __half* Hh = reinterpret_cast<__half*>(b + o_hh);
   float* scr = split_bytes ? reinterpret_cast<float*>(b + o_scr) : nullptr;
-  unsigned* cnt = split_bytes ? reinterpret_cast<unsigned*>(b + o_cnt) : nullptr;
+  unsigned* cnt = use_tc ? reinterpret_cast<unsigned*>(b + o_cnt) : nullptr;
   float* t = reinterpret_cast<float*>(b + o_t);
   float* tsc = reinterpret_cast<float*>(b + o_tsc);
   int32_t* tloc = shard ? reinterpret_cast<int32_t*>(b + o_tloc) : nullptr;

@@ -185,8 +185,8 @@ __host__ __device__ __forceinline__ int64_t tc_image_offset(int64_t tt, int64_t 
          ((((kk >> 3) & 7) ^ (int)(nn & 7)) << 3) + (kk & 7);
 }
 // Blocked image of H (zero rows up to the token tile) and its rank blocks.
-// counters: the per-tile counters of a split launch (ceil(V/128) words, zeroed here), or
-// nullptr.
+// counters: ceil(V/128) words zeroed here (the per-tile counters of a split launch, or
+// the work counter of the dynamic item order), or nullptr.
 cudaError_t launch_prologue_blocked(const uint16_t* H, const archead_head* head,
                                     const Shapes& s, const TcPlan& plan, __half* Hb, float* tsc,
                                     unsigned* counters, unsigned* err, cudaStream_t st,
@@ -197,7 +197,8 @@ size_t tc_split_scratch_bytes(const Shapes& s, const TcPlan& plan);
 // Y != nullptr: write logits.  Y == nullptr: fused NLL, writing (max, sum exp) partials
 // into part[N x ceil(V/128)] and target logits into tlogit[N] (see launch_nll_combine).
 // scratch / counters (tc_split_scratch_bytes, launch_prologue_blocked): the split of a
-// single token tile over the CTAs, or nullptr for whole tiles per CTA.
+// single token tile over the CTAs; with several token tiles, counters[0] is the work
+// counter from which the CTAs take their items in order (nullptr: a fixed round-robin).
 cudaError_t launch_residual_tc(const __half* Hb, const float* tsc, const archead_head* head,
                                const Shapes& s, const TcPlan& plan, float* Y,
                                const int32_t* targets,

@@ -36,8 +36,11 @@
 //    reduced on chip into split-vocabulary log-sum-exp partials (fused NLL).
 // Scheduling: with a single token tile (decode) the (tile, K block) units are split evenly
 // over the CTAs and a tile at the edge of two ranges is finished from two partial
-// accumulators; otherwise items are dealt round-robin with the token tile varying
-// fastest, so CTAs working on the same rows run together and re-read them from L2.
+// accumulators; otherwise the CTAs take items in order (the token tile varying fastest
+// inside L2-sized bands) from a work counter: the packed producer claims them two items
+// ahead of its stream and hands the indices to the other roles through a small queue in
+// shared memory, so all CTAs stay within a few items of one another and the readers of a
+// vocabulary tile find its packed blocks in L2.
 // Every mbarrier wait is bounded (about a second of SM cycles); a wait that gives up sets
 // the device error word, the CTA drains what it issued and frees its tensor memory.
 #include "tc_common.cuh"
@@ -49,6 +52,9 @@ constexpr int kTcThreads = 352;  // warps 0-3 dequant, 4-7 epilogue, 8 and 10 pr
 constexpr int kPkBytes = 8192;   // packed block of one 128-row tile (128 columns)
 constexpr int kMaxSB = 8;        // deepest B ring
 constexpr int kMaxSP = 8;        // deepest packed ring
+constexpr int kItemQ = 8;        // item queue slots (dynamic order)
+constexpr int kItemAhead = 2;    // items the packed producer claims ahead of its stream
+constexpr int kItemUsers = 10;   // releases per item: B producer, MMA warp, 4 dequant, 4 epilogue
 
 struct TcParams {
   const __half* Hb;  // B image: [token tile][nkb + nrb blocks][NT x 128]
@@ -80,6 +86,10 @@ struct TcParams {
   // ([CTA][slot 0: first item, 1: last item][NT][128] FP32); the part that arrives second
   // at the tile's counter (zeroed by the prologue) adds the two and finishes the tile.
   int split;
+  // Several token tiles: the items are taken in order from a work counter (counters[0],
+  // zeroed by the prologue) instead of a fixed round-robin, so all CTAs stay within a few
+  // items of one another and the readers of a vocabulary tile share its reads through L2.
+  int dyn;
   float* scratch;
   unsigned* counters;
   unsigned* err;
@@ -118,7 +128,7 @@ template <int NT>
 size_t tc_smem_bytes(int sb, int sp, int G, bool nll) {
   using C = TcCfg<NT>;
   return (size_t)sb * C::HSTAGE + (size_t)sp * kPkBytes + 2 * round16((size_t)128 * G) +
-         (nll ? nll_scratch_bytes<NT>() : 0) + (size_t)NT * 4 + 512;
+         (nll ? nll_scratch_bytes<NT>() : 0) + (size_t)NT * 4 + 1024;
 }
 
 // The k-th work item of this CTA: its tile's first row, its row limit, its token tile.
@@ -128,6 +138,26 @@ struct Item {
   int kb0, kb1;  // the item's K blocks [kb0, kb1) of the tile's nkb + nrb
   int part;      // 0: whole tile; 1: head part (blocks from 0); 2: tail part (to the end)
 };
+
+// Item gi of the several-token-tile order: bands of tt_band token tiles; inside a band the
+// token tile varies fastest, so CTAs reading the same vocabulary rows run together and the
+// band's B image is reused from L2 across all vocabulary tiles.  False past the last item.
+__device__ __forceinline__ bool item_of(const TcParams& p, int64_t gi, Item& it) {
+  if (gi >= p.n_vtiles * p.n_tok_tiles) return false;
+  const int64_t band_items = p.n_vtiles * p.tt_band;
+  const int64_t band = gi / band_items;
+  const int64_t local = gi - band * band_items;
+  const int64_t tt0 = band * p.tt_band;
+  const int64_t nb = p.n_tok_tiles - tt0 < p.tt_band ? p.n_tok_tiles - tt0 : p.tt_band;
+  it.vt = local / nb;
+  it.tt = (int)(tt0 + (local - it.vt * nb));
+  it.kb0 = 0;
+  it.kb1 = (int)(p.D >> 7) + p.nrb;
+  it.part = 0;
+  it.row0 = it.vt * 128;
+  it.row_end = it.row0 + 128 < p.V ? it.row0 + 128 : p.V;
+  return true;
+}
 
 __device__ __forceinline__ bool get_item(const TcParams& p, int k, Item& it) {
   const int nkbt = (int)(p.D >> 7) + p.nrb;
@@ -154,22 +184,41 @@ __device__ __forceinline__ bool get_item(const TcParams& p, int k, Item& it) {
     if (it.vt >= t1) return false;
     it.tt = 0;
   } else {
-    // bands of tt_band token tiles; inside a band the token tile varies fastest, so CTAs
-    // reading the same vocabulary rows run together and the band's B image is reused
-    // from L2 across all vocabulary tiles
-    const int64_t gi = blockIdx.x + (int64_t)k * gridDim.x;
-    if (gi >= p.n_vtiles * p.n_tok_tiles) return false;
-    const int64_t band_items = p.n_vtiles * p.tt_band;
-    const int64_t band = gi / band_items;
-    const int64_t local = gi - band * band_items;
-    const int64_t tt0 = band * p.tt_band;
-    const int64_t nb = p.n_tok_tiles - tt0 < p.tt_band ? p.n_tok_tiles - tt0 : p.tt_band;
-    it.vt = local / nb;
-    it.tt = (int)(tt0 + (local - it.vt * nb));
+    if (!item_of(p, blockIdx.x + (int64_t)k * gridDim.x, it)) return false;
   }
   it.row0 = it.vt * 128;
   it.row_end = it.row0 + 128 < p.V ? it.row0 + 128 : p.V;
   return true;
+}
+
+// The k-th item of this CTA.  The fixed orders come from get_item; the dynamic order from
+// the item queue that the packed producer fills: the caller waits for slot k's phase, reads
+// the item index, and its warp releases the slot (one arrival per warp, by lane 0 after
+// all its lanes have read; `solo` for a single-thread role).
+struct ItemQueue {
+  const int64_t* ids;
+  uint64_t* full;
+  uint64_t* empty;
+};
+__device__ __forceinline__ bool next_item(const TcParams& p, const ItemQueue& q, int64_t k,
+                                          Item& it, bool& ok, bool solo) {
+  if (!p.dyn) return get_item(p, (int)k, it);
+  if (!ok) return false;  // warp-uniform for warp callers: only set from warp-wide outcomes
+  const int slot = (int)(k % kItemQ);
+  bool got = tc::mbar_wait(&q.full[slot], (uint32_t)(k / kItemQ) & 1u, p.err);
+  if (!solo) got = __all_sync(0xffffffffu, got);  // the lanes agree before __syncwarp below
+  if (!got) {
+    ok = false;
+    return false;
+  }
+  const int64_t gi = *reinterpret_cast<const volatile int64_t*>(q.ids + slot);
+  if (solo) {
+    tc::mbar_arrive(&q.empty[slot]);
+  } else {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) tc::mbar_arrive(&q.empty[slot]);
+  }
+  return item_of(p, gi, it);
 }
 
 // The row scales of vocabulary row v (clamped into range; rows past V only pad a tile).
@@ -268,8 +317,12 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
   uint64_t* acc_full = a_empty + C::SA;  // [2]
   uint64_t* acc_empty = acc_full + 2;    // [2]
   uint64_t* mma_done = acc_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* item_full = mma_done + 1;        // [kItemQ]
+  uint64_t* item_empty = item_full + kItemQ;  // [kItemQ]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(item_empty + kItemQ);
   int* ep_flag = reinterpret_cast<int*>(tmem_slot + 1);  // epilogue: a tile counter's value
+  int64_t* item_ids = reinterpret_cast<int64_t*>(tmem_slot + 2);  // [kItemQ]
+  const ItemQueue iq = {item_ids, item_full, item_empty};
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -293,6 +346,10 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
       tc::mbar_init(&a_empty[s], 1);
     }
     tc::mbar_init(mma_done, 1);
+    for (int s = 0; s < kItemQ; ++s) {
+      tc::mbar_init(&item_full[s], 1);
+      tc::mbar_init(&item_empty[s], kItemUsers);
+    }
     tc::mbar_fence_init();
   }
   if (warp == 9) tc::tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -310,11 +367,38 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
     // by a constant stride: the thread is on the critical path of the pipeline.  A wait
     // that gives up drains the copies in flight.
     if (lane == 0) {
+      bool ok = true;
+      // dynamic order: claim items from the work counter (zeroed by the prologue kernel,
+      // hence the dependency wait) kItemAhead ahead of the stream, into the item queue
+      int64_t claimed = 0;
+      bool more = true;
+      const int64_t total = p.n_vtiles * p.n_tok_tiles;
+      if (p.dyn) grid_dependency_wait();
+      auto claim_to = [&](int64_t upto) {
+        while (ok && more && claimed <= upto) {
+          const int slot = (int)(claimed % kItemQ);
+          if (claimed >= kItemQ &&
+              !tc::mbar_wait(&item_empty[slot], (uint32_t)((claimed / kItemQ) - 1) & 1u, p.err)) {
+            ok = false;
+            break;
+          }
+          const int64_t gi = (int64_t)atomicAdd(p.counters, 1u);
+          item_ids[slot] = gi;
+          tc::mbar_arrive(&item_full[slot]);  // releases the index to the waiting roles
+          ++claimed;
+          if (gi >= total) more = false;
+        }
+      };
+      auto p_next = [&](int64_t k, Item& it) -> bool {
+        if (!p.dyn) return get_item(p, (int)k, it);
+        claim_to(k + kItemAhead);
+        if (!ok || k >= claimed) return false;
+        return item_of(p, item_ids[k % kItemQ], it);
+      };
       Item pit;
-      bool p_have = get_item(p, 0, pit);
+      bool p_have = p_next(0, pit);
       int ip = 0, np = 0, nc = 0, ps = 0, cs = 0;
       uint32_t pph = 0, cph = 0;  // phase parities of the next refill of slot ps / cs
-      bool ok = true;
       while (ok && p_have) {
         if (nc >= 2 && !tc::mbar_wait(&c_empty[cs], cph ^ 1u, p.err)) {
           ok = false;
@@ -346,7 +430,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
             pph ^= 1u;
           }
         }
-        p_have = get_item(p, ++ip, pit);
+        p_have = p_next(++ip, pit);
       }
       if (!ok) {  // drain copies still in flight before the CTA exits
         for (int q = np - SPK < 0 ? 0 : np - SPK; q < np; ++q)
@@ -363,10 +447,10 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
     if (lane == 0) {
       grid_dependency_wait();
       Item hit;
-      bool h_have = get_item(p, 0, hit);
+      bool ok = true;
+      bool h_have = next_item(p, iq, 0, hit, ok, true);
       int ih = 0, nb = 0, hs = 0;
       uint32_t hph = 0;
-      bool ok = true;
       while (ok && h_have) {
         const unsigned char* hsrc = reinterpret_cast<const unsigned char*>(p.Hb) +
                                     ((int64_t)hit.tt * nkbt + hit.kb0) * C::HSTAGE;
@@ -384,7 +468,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
             hph ^= 1u;
           }
         }
-        h_have = get_item(p, ++ih, hit);
+        h_have = next_item(p, iq, ++ih, hit, ok, true);
       }
       if (!ok) {
         for (int q = nb - SB < 0 ? 0 : nb - SB; q < nb; ++q)
@@ -407,7 +491,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
       uint32_t pa = 0, pb = 0;
       bool ok = true;
       Item it;
-      for (int i = 0; ok && get_item(p, i, it); ++i) {
+      for (int i = 0; ok && __all_sync(0xffffffffu, next_item(p, iq, i, it, ok, false)); ++i) {
         const int ab = i % C::NACC, use = i / C::NACC;
         if (i >= C::NACC &&
             !__all_sync(0xffffffffu, tc::mbar_wait(&acc_empty[ab], (use - 1) & 1, p.err)))
@@ -478,13 +562,13 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
     bool p_ready = false, a_ready = false;  // the next stage's barriers, probed early
     bool ok = true;
     Item it;
-    bool have = get_item(p, 0, it);
+    bool have = __all_sync(0xffffffffu, next_item(p, iq, 0, it, ok, false));
     RowIn rin = {0.f, 0.f, 0.f};
     if (have) rin = load_row(p, it.row0 + tid);
     for (int i = 0; ok && have; ++i) {
       // the next item's row scales load while this one runs
       Item nx;
-      const bool have_nx = get_item(p, i + 1, nx);
+      const bool have_nx = __all_sync(0xffffffffu, next_item(p, iq, i + 1, nx, ok, false));
       RowIn rnx = rin;
       if (have_nx) rnx = load_row(p, nx.row0 + tid);
       const int64_t v = it.row0 + tid;
@@ -620,7 +704,9 @@ __global__ void __launch_bounds__(kTcThreads, 2) residual_tc_kernel(const TcPara
     const uint32_t lane_off = (uint32_t)(32 * (warp - 4)) << 16;
     int cur_tt = -1;
     Item it;
-    for (int i = 0; get_item(p, i, it); ++i) {
+    bool qok = true;
+    // one outcome for all four epilogue warps: they share named barriers below
+    for (int i = 0; tc::bar_and(1, 128, next_item(p, iq, i, it, qok, false)); ++i) {
       const int ab = i % C::NACC, use = i / C::NACC;
       const int64_t tok0 = (int64_t)it.tt * NT;
       if (it.tt != cur_tt) {  // the token tile's scales (and targets)
@@ -994,6 +1080,7 @@ cudaError_t launch_residual_tc(const __half* Hb, const float* tsc, const archead
   }
   p.n_vtiles = (s.V + 127) / 128;
   p.split = (p.n_tok_tiles == 1 && scratch && counters) ? 1 : 0;
+  p.dyn = (p.n_tok_tiles > 1 && counters && p.n_vtiles * p.n_tok_tiles < (1ll << 31)) ? 1 : 0;
   p.scratch = scratch;
   p.counters = counters;
   if (plan.nt == 0 || plan.sb < 2 || plan.sb > kMaxSB || plan.sp < 2 || plan.sp > kMaxSP)
