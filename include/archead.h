@@ -199,6 +199,13 @@ int archead_nll_merge(const float* partials, int G, int64_t N, float* nll_out, v
  * the device, evaluates, copies Y back into Y_host (float N x V), and synchronises
  * `stream` before returning.  Pinned host memory gives asynchronous copies.  The device
  * staging buffers come from the library's stream-ordered pool.
+ *   When Y holds at least about 6 MB, the vocabulary is evaluated in chunks (at most 8,
+ * each a multiple of 128 rows, about 3 MB of Y) and each chunk's logits are copied to
+ * Y_host on a library-owned second stream while the next chunks run, so the host copy,
+ * which takes longer than the kernels for all but the smallest N, overlaps them.  Each
+ * chunk is an ordinary archead_logits call on a view of the head's rows; the chunks' FP32
+ * sums may round differently from one call over the whole head (within 1e-4 max|Y|).
+ * archead_last_launches() then counts the launches of all chunks.
  */
 int archead_logits_host(const uint16_t* H_host, const archead_head* head, float* Y_host,
                         int64_t N, int64_t V, int64_t D, int r_c, int r_r, int g,

@@ -1,5 +1,6 @@
 // C ABI of the ARCHead packed LM-head library: argument validation, stream-ordered
 // scratch, the per-device error word and kernel dispatch.  See include/archead.h.
+#include <algorithm>
 #include <mutex>
 
 #include "archead_internal.cuh"
@@ -17,6 +18,7 @@ struct DeviceState {
   bool ready = false;
   unsigned* err = nullptr;       // device address of g_error_word on this device
   cudaMemPool_t pool = nullptr;  // library-owned stream-ordered pool
+  cudaStream_t copy = nullptr;   // device-to-host copies of archead_logits_host
 };
 
 std::mutex g_mu;
@@ -68,6 +70,54 @@ int current_state(DeviceState** out) {
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// The non-blocking stream on which archead_logits_host copies Y to the host (created on
+// first use, kept for the life of the process).
+int copy_stream(DeviceState* ds, cudaStream_t* out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!ds->copy && cudaStreamCreateWithFlags(&ds->copy, cudaStreamNonBlocking) != cudaSuccess) {
+    ds->copy = nullptr;
+    cudaGetLastError();
+    return ARCHEAD_ERR_CUDA;
+  }
+  *out = ds->copy;
+  return ARCHEAD_OK;
+}
+
+// The rows [v0, v0 + rows) of a head as a head of its own (v0 a multiple of 128): every
+// per-row array is row-major, and the device nibble layout is tile-major with 128 x D/2
+// bytes per 128-row tile, so the view is the same pointers advanced by v0 rows.
+archead_head head_rows(const archead_head& h, int64_t v0, int64_t rows) {
+  archead_head s = h;
+  s.V = rows;
+  if (h.format == ARCHEAD_FMT_ROW8) {
+    s.r_nib = h.r_nib + v0 * h.D;
+    s.row_scale = h.row_scale + v0;
+    return s;
+  }
+  s.r_nib = h.r_nib + v0 * (h.D / 2);
+  s.r_code = h.r_code + v0 * (h.D / h.g);
+  s.r_super = h.r_super + v0;
+  if (h.Ac) s.Ac = h.Ac + v0 * h.r_c;
+  if (h.sAc) s.sAc = h.sAc + v0;
+  if (h.Aw) s.Aw = h.Aw + v0 * h.r_r;
+  if (h.sAw) s.sAw = h.sAw + v0;
+  return s;
+}
+
+// archead_logits_host splits the vocabulary into chunks of about this many bytes of Y (at
+// most kMaxHostChunks, each a multiple of 128 rows) and copies each chunk's logits to the
+// host while the next chunks are evaluated: the copy of 4 bytes per logit over the host
+// link takes longer than the kernels for all but the smallest N.
+constexpr size_t kHostChunkBytes = 3u << 20;
+constexpr int kMaxHostChunks = 8;
+
+int64_t host_chunk_rows(int64_t N, int64_t V) {
+  const size_t yb = (size_t)N * V * 4;
+  const int64_t c = (int64_t)std::min<size_t>(kMaxHostChunks, yb / kHostChunkBytes);
+  if (c < 2 || V < 256) return V;
+  return (int64_t)round_up((size_t)((V + c - 1) / c), 128);
+}
 
 int check_head(const archead_head* h, int64_t N, int64_t V, int64_t D, int r_c, int r_r,
                int g) {
@@ -440,9 +490,50 @@ int archead_logits_host(const uint16_t* H_host, const archead_head* head, float*
   rc = ARCHEAD_OK;
   if (cudaMemcpyAsync(Hd, H_host, hb, cudaMemcpyHostToDevice, st) != cudaSuccess)
     rc = ARCHEAD_ERR_CUDA;
-  if (!rc) rc = archead_logits(Hd, head, Yd, N, V, D, r_c, r_r, g, stream);
-  if (!rc && cudaMemcpyAsync(Y_host, Yd, yb, cudaMemcpyDeviceToHost, st) != cudaSuccess)
-    rc = ARCHEAD_ERR_CUDA;
+  const int64_t rows = host_chunk_rows(N, V);
+  if (rows >= V) {
+    if (!rc) rc = archead_logits(Hd, head, Yd, N, V, D, r_c, r_r, g, stream);
+    if (!rc && cudaMemcpyAsync(Y_host, Yd, yb, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+      rc = ARCHEAD_ERR_CUDA;
+  } else {
+    // chunk i: its kernels on `stream` write the N x vc block Yd + N v0 (its own row-major
+    // logits), an event marks their end, and the copy stream waits for it and copies the
+    // block into columns [v0, v0 + vc) of Y_host
+    cudaStream_t cs = nullptr;
+    cudaEvent_t ev[kMaxHostChunks + 1];
+    int nev = 0;
+    if (!rc) rc = copy_stream(ds, &cs);
+    while (!rc && nev <= kMaxHostChunks) {
+      if (cudaEventCreateWithFlags(&ev[nev], cudaEventDisableTiming) != cudaSuccess)
+        rc = ARCHEAD_ERR_CUDA;
+      else
+        ++nev;
+    }
+    int launches = 0, i = 0;
+    for (int64_t v0 = 0; !rc && v0 < V; v0 += rows, ++i) {
+      const int64_t vc = std::min(rows, V - v0);
+      const archead_head part = head_rows(*head, v0, vc);
+      float* Yc = Yd + N * v0;
+      rc = archead_logits(Hd, &part, Yc, N, vc, D, r_c, r_r, g, stream);
+      if (rc) break;
+      launches += t_last_launches;
+      if (cudaEventRecord(ev[i], st) != cudaSuccess ||
+          cudaStreamWaitEvent(cs, ev[i], 0) != cudaSuccess ||
+          cudaMemcpy2DAsync(Y_host + v0, (size_t)V * 4, Yc, (size_t)vc * 4, (size_t)vc * 4,
+                            (size_t)N, cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+        rc = ARCHEAD_ERR_CUDA;
+    }
+    // the staging buffer goes back to the pool on `stream` only after the last copy
+    if (cs && nev == kMaxHostChunks + 1 &&
+        (cudaEventRecord(ev[kMaxHostChunks], cs) != cudaSuccess ||
+         cudaStreamWaitEvent(st, ev[kMaxHostChunks], 0) != cudaSuccess)) {
+      cudaStreamSynchronize(cs);
+      if (!rc) rc = ARCHEAD_ERR_CUDA;
+    }
+    if (cs && nev < kMaxHostChunks + 1) cudaStreamSynchronize(cs);
+    if (!rc) t_last_launches = launches;
+    for (int j = 0; j < nev; ++j) cudaEventDestroy(ev[j]);
+  }
   cudaFreeAsync(base, st);
   if (cudaStreamSynchronize(st) != cudaSuccess && !rc) rc = ARCHEAD_ERR_CUDA;
   return rc;
