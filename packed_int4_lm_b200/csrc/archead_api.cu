@@ -344,7 +344,8 @@ const char* archead_strerror(int status) {
     case ARCHEAD_ERR_NULLPTR: return "a required pointer is NULL";
     case ARCHEAD_ERR_ALIGN: return "a pointer is not suitably aligned (16 bytes)";
     case ARCHEAD_ERR_SHAPE: return "sizes disagree with the head or break a limit";
-    case ARCHEAD_ERR_RANGE_H: return "an entry of H is not finite, or a scaled rank product exceeds the FP16 range";
+    case ARCHEAD_ERR_RANGE_H:
+      return "an entry of H is not finite, or a scaled rank product exceeds the FP16 range";
     case ARCHEAD_ERR_TARGET: return "a target id is outside [0, V)";
     case ARCHEAD_ERR_TIMEOUT: return "a bounded device wait gave up";
     case ARCHEAD_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
